@@ -1,0 +1,155 @@
+"""Pins for the oracle's backward: adjoint identities (the forward is linear
+in the value and in the weights) and central finite differences for the
+location gradients and for the fused chain (offsets, reference points,
+logits).  CPU only."""
+import numpy as np
+
+import oracle
+from scale_deformable_attention_02_b200 import workloads as wl
+
+
+def _kink_mask(loc, shapes, tol):
+    """True where a sample sits within tol (pixels) of a cell boundary in x
+    or y, where the interpolant has a kink and a finite difference is not a
+    derivative."""
+    mask = np.zeros(loc.shape[:-1], bool)
+    for l, (h, w) in enumerate(shapes):
+        x = loc[..., l, :, 0] * w - 0.5
+        y = loc[..., l, :, 1] * h - 0.5
+        fx = x - np.floor(x)
+        fy = y - np.floor(y)
+        near = (np.minimum(fx, 1 - fx) < tol) | (np.minimum(fy, 1 - fy) < tol)
+        mask[..., l, :] = near
+    return mask
+
+
+def test_adjoint_value_and_weights():
+    """<g, F(v', A)> = <dF/dv^T g, v'> for any v' (F is linear in v), and
+    <g, F(v, A')> = <dF/dA^T g, A'> for any A' (F is linear in A)."""
+    for seed in range(3):
+        d = wl.make_random_problem(seed, N=2, Lq=9, M=3, D=4, K=3,
+                                   shapes=((6, 5), (3, 3), (2, 1)))
+        shapes, value = d["spatial_shapes"], d["value"]
+        loc = d["sampling_locations"]
+        A = oracle.softmax(d["logits"])
+        g = d["grad_out"].astype(np.float64)
+        gv, gl, ga = oracle.backward(value, shapes, loc, A, g)
+        rng = np.random.default_rng(100 + seed)
+        v2 = rng.uniform(-1, 1, size=value.shape).astype(np.float32)
+        lhs = np.sum(g * oracle.forward(v2, shapes, loc, A))
+        rhs = np.sum(gv * v2.astype(np.float64))
+        assert abs(lhs - rhs) <= 1e-12 * (1 + abs(lhs))
+        A2 = rng.uniform(-1, 1, size=A.shape)
+        lhs = np.sum(g * oracle.forward(value, shapes, loc, A2))
+        rhs = np.sum(ga * A2)
+        assert abs(lhs - rhs) <= 1e-12 * (1 + abs(lhs))
+
+
+def test_adjoint_on_tiny_workload_bf16_value():
+    d = wl.make_random_problem(5, N=1, Lq=16, M=2, D=8, K=2, shapes=wl.TINY_SHAPES,
+                               value_dtype="bf16")
+    shapes = d["spatial_shapes"]
+    A = oracle.softmax(d["logits"])
+    g = d["grad_out"].astype(np.float64)
+    out_bits = oracle.forward(d["value"], shapes, d["sampling_locations"], A)
+    out_f32 = oracle.forward(d["value_f32"], shapes, d["sampling_locations"], A)
+    np.testing.assert_array_equal(out_bits, out_f32)  # bf16 widening is exact
+    gv, _, ga = oracle.backward(d["value"], shapes, d["sampling_locations"], A, g)
+    assert abs(np.sum(g * out_bits) - np.sum(ga * A)) < 1e-12
+
+
+def _fd_check_loc(value, shapes, loc64, A, g, h=1e-6, kink_tol=1e-3):
+    _, gl, _ = oracle.backward(value, shapes, loc64, A, g, loc_f32=False)
+    skip = _kink_mask(loc64, shapes, kink_tol)
+    idx = np.argwhere(~skip)
+    assert len(idx) > 0
+    checked = 0
+    for ii in idx:
+        ii = tuple(ii)
+        for c in range(2):
+            lp = loc64.copy()
+            lm = loc64.copy()
+            lp[ii + (c,)] += h
+            lm[ii + (c,)] -= h
+            fp = np.sum(g * oracle.forward(value, shapes, lp, A, loc_f32=False))
+            fm = np.sum(g * oracle.forward(value, shapes, lm, A, loc_f32=False))
+            fd = (fp - fm) / (2 * h)
+            an = gl[ii + (c,)]
+            assert abs(fd - an) <= 1e-6 * (1 + abs(an)), (ii, c, fd, an)
+            checked += 1
+    return checked
+
+
+def test_finite_differences_location_gradient_tiny():
+    """Central differences of <g, out> in every location coordinate of the
+    tiny workload (fp64 oracle), away from cell-boundary kinks.  The
+    interpolant is linear in x inside a cell, so the difference is exact up
+    to rounding."""
+    d = wl.make_inputs(wl.TINY)
+    loc64 = d["sampling_locations"].astype(np.float64)
+    A = oracle.softmax(d["logits"])
+    g = d["grad_out"].astype(np.float64)
+    n = _fd_check_loc(d["value"], d["spatial_shapes"], loc64, A, g)
+    assert n >= 200  # 128 samples x 2 coordinates, minus kinks
+
+
+def test_finite_differences_location_gradient_encoder_subsample():
+    """Same check on encoder-shaped problems (D = 32, 4 levels of the
+    encoder shapes) for a handful of queries; the other queries are removed
+    because they do not affect the chosen queries' outputs."""
+    d = wl.make_inputs(wl.ENCODER_BWD)
+    rng = np.random.default_rng(44)
+    qs = np.sort(rng.choice(wl.ENCODER_BWD.queries, size=6, replace=False))
+    loc32 = oracle.locations_f32(d["reference_points"][:1, qs], d["offsets"][:1, qs],
+                                 d["spatial_shapes"])
+    A = oracle.softmax(d["logits"][:1, qs])
+    g = d["grad_out"][:1, qs].astype(np.float64)
+    # only one batch entry's value matters for batch entry 0
+    value = np.ascontiguousarray(d["value"][:1])
+    n = _fd_check_loc(value, d["spatial_shapes"], loc32.astype(np.float64), A, g)
+    assert n > 6 * 8 * 16
+
+
+def test_finite_differences_fused_chain():
+    """The chain from sampled-point gradients to the fused inputs: central
+    differences of <g, F(ref, off, logits)> with F composed in fp64."""
+    d = wl.make_random_problem(9, N=1, Lq=3, M=2, D=3, K=2,
+                               shapes=((5, 6), (3, 4)), offset_std=1.0)
+    shapes, value = d["spatial_shapes"], d["value"]
+    ref = d["reference_points"].astype(np.float64)
+    off = d["offsets"].astype(np.float64)
+    z = d["logits"].astype(np.float64)
+    g = d["grad_out"].astype(np.float64)
+
+    def F(ref_, off_, z_):
+        loc = oracle.locations_f64(ref_, off_, shapes)
+        return np.sum(g * oracle.forward(value, shapes, loc, oracle.softmax(z_), loc_f32=False))
+
+    loc = oracle.locations_f64(ref, off, shapes)
+    A = oracle.softmax(z)
+    _, gl, ga = oracle.backward(value, shapes, loc, A, g, loc_f32=False)
+    g_ref, g_off, g_z = oracle.fused_chain(gl, ga, A, shapes)
+    h = 1e-6
+    skip = _kink_mask(loc, shapes, 1e-3)
+    for ii in np.ndindex(*off.shape[:-1]):
+        if skip[ii]:
+            continue
+        for c in range(2):
+            p, m = off.copy(), off.copy()
+            p[ii + (c,)] += h
+            m[ii + (c,)] -= h
+            fd = (F(ref, p, z) - F(ref, m, z)) / (2 * h)
+            assert abs(fd - g_off[ii + (c,)]) <= 1e-6 * (1 + abs(fd))
+    for ii in np.ndindex(*z.shape):
+        p, m = z.copy(), z.copy()
+        p[ii] += h
+        m[ii] -= h
+        fd = (F(ref, off, p) - F(ref, off, m)) / (2 * h)
+        assert abs(fd - g_z[ii]) <= 1e-6 * (1 + abs(fd))
+    if not skip.any():
+        for ii in np.ndindex(*ref.shape):
+            p, m = ref.copy(), ref.copy()
+            p[ii] += h
+            m[ii] -= h
+            fd = (F(p, off, z) - F(m, off, z)) / (2 * h)
+            assert abs(fd - g_ref[ii]) <= 1e-6 * (1 + abs(fd))
