@@ -1,0 +1,531 @@
+#!/usr/bin/env python
+"""Benchmark of the MSDeformAttn core on B200: one step = the fused forward
+(softmax, location map, bilinear gather; it also writes the locations and
+weights the backward needs) followed by the backward (grad_value scatter,
+grad_sampling_locations, grad_attention_weights) over one batch of the chosen
+synthetic workload.  Prints ONE JSON line on rank 0.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload encoder]
+  python bench.py --impl reference ...   # the CPU oracle, timed on host cores
+
+Timing: W untimed warm-up steps; then K steps, each preceded by an L2 flush
+(a memset of twice the L2 size, outside the timed events), each timed with
+CUDA events on the launching stream; the K-step region is bracketed by a
+barrier and torch.cuda.synchronize() on both sides; the reported time is the
+max over ranks.  Multi-GPU: every rank runs its own batch (weak scaling; the
+batch entries are independent, so there is no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from scale_deformable_attention_02_b200 import workloads as wl  # noqa: E402
+
+METRIC = "MSDeformAttn fwd+bwd queries/sec and effective HBM GB/s (% roofline) on 1 B200"
+FALLBACK_HBM_GBS = 6650.0
+
+WORKLOAD_TEXT = {
+    "encoder": "encoder-shaped fused fwd+bwd, fp32 value: N=2, Lq=S=17821 (one query per "
+               "pixel of 100x134, 50x67, 25x34, 13x17), M=8, D=32, L=4, K=4",
+    "encoder_bf16": "encoder-shaped fused fwd+bwd, bf16 value, fp32 accumulation: N=2, "
+                    "Lq=S=17821, M=8, D=32, L=4, K=4",
+    "stress": "high-resolution stress fused fwd+bwd, bf16 value, fp32 accumulation: N=8, "
+              "Lq=S=37150 (167x167, 84x84, 42x42, 21x21), M=8, D=32, L=4, K=8, 5% of "
+              "samples pushed out of range",
+    "decoder": "decoder-shaped fused fwd+bwd, fp32 value: N=2, Lq=300, M=8, D=32, L=4, K=4, "
+               "S=17821",
+}
+
+
+# ---------------------------------------------------------------------------
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(WORKLOAD_TEXT), default="encoder")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle leg")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def rank_workload(name: str, rank: int) -> wl.Workload:
+    w = wl.WORKLOADS[name]
+    return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+# ---------------------------------------------------------------------------
+# algorithmic (unique) bytes per launch
+# ---------------------------------------------------------------------------
+def algorithmic_bytes(w: wl.Workload) -> dict:
+    """Minimum HBM traffic of each launch: every input read once, every
+    output written once (the value map counted once although its rows are
+    gathered many times; the backward's zero-fill of grad_value is not
+    counted)."""
+    N, Lq, S, M, D, L, K = (w.N, w.queries, w.S, w.M, w.D, w.L, w.K)
+    esz = 2 if w.value_dtype == "bf16" else 4
+    samples = N * Lq * M * L * K
+    value = N * S * M * D * esz
+    ref = N * Lq * 2 * 4
+    outb = N * Lq * M * D * 4
+    fwd = value + ref + samples * 8 + samples * 4 + outb + samples * 8 + samples * 4
+    bwd = value + samples * 8 + samples * 4 + outb + N * S * M * D * 4 + samples * 8 + samples * 4
+    return {"fwd": fwd, "bwd": bwd, "samples": samples}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "scale_deformable_attention_02_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + b"\0" + fh.read())
+    return h.hexdigest()
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def read_traffic(workload: str, kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d[workload][kernel]
+        if e.get("source_sha256") != kernel_source_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; nothing is changed)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, pci_bus_id: str | None, fallback_index: int, period_s: float = 0.002):
+        self.samples = []
+        self.period = period_s
+        self._stop = threading.Event()
+        self._t = None
+        self.max_mhz = None
+        self.error = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            self.h = None
+            if pci_bus_id:
+                try:
+                    self.h = pynvml.nvmlDeviceGetHandleByPciBusId(pci_bus_id.encode())
+                except Exception:
+                    self.h = None
+            if self.h is None:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(fallback_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.nvml = None
+            self.error = repr(e)
+
+    def _run(self):
+        nv = self.nvml
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((time.perf_counter(), sm, rs))
+            except Exception as e:  # pragma: no cover
+                self.error = repr(e)
+                return
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nvml is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "note": self.error or "no samples"}
+        mhz = [s[1] for s in self.samples]
+        active = 0
+        for s in self.samples:
+            active |= s[2]
+        reasons = [k for k, bit in self.REASONS.items() if active & bit and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(self.samples),
+                "sm_mhz_min": min(mhz), "source": "NVML, every 2 ms during the timed steps"}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    from scale_deformable_attention_02_b200 import msda_backward, msda_forward_fused
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                device_id=device)
+    w = rank_workload(args.workload, rank)
+    inp = wl.make_inputs(w)
+    sh = inp["spatial_shapes"]
+
+    def dev_tensor(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+        return torch.from_numpy(a).to(device)
+
+    value = dev_tensor(inp["value"])
+    ref = dev_tensor(inp["reference_points"])
+    off = dev_tensor(inp["offsets"])
+    logits = dev_tensor(inp["logits"])
+    gout = dev_tensor(inp["grad_out"])
+    out = torch.empty((w.N, w.queries, w.M * w.D), device=device)
+    loc = torch.empty_like(off)
+    attn = torch.empty_like(logits)
+    gval = torch.empty((w.N, w.S, w.M, w.D), device=device)
+    gloc = torch.empty_like(off)
+    gattn = torch.empty_like(logits)
+    starts, _ = __import__("scale_deformable_attention_02_b200").msda_level_start_index(sh)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        msda_forward_fused(value, sh, starts, ref, off, logits, out=out,
+                           sampling_locations_out=loc, attention_weights_out=attn,
+                           stream=stream)
+
+    def step_bwd():
+        msda_backward(value, sh, starts, loc, attn, gout, grad_value=gval,
+                      grad_sampling_locations=gloc, grad_attention_weights=gattn,
+                      stream=stream)
+
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flush = torch.empty(max(2 * l2, 64 << 20), dtype=torch.uint8, device=device)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+        step_bwd()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    clocks = ClockSampler(_pci_bus_id(torch, device), _nvml_index(local))
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+        step_bwd()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    clocks.stop()
+    if world > 1:
+        dist.barrier()
+    fwd_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    bwd_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
+    t = torch.tensor([statistics.fmean(step_ms), statistics.fmean(fwd_ms),
+                      statistics.fmean(bwd_ms)], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step, ms_fwd, ms_bwd = (float(x) for x in t.tolist())
+    queries = w.N * w.queries
+    value_qps = queries * world / (ms_step / 1e3)
+
+    # ---- end to end through the binding with host buffers -----------------
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value,
+                      queries)
+
+    # ---- roofline of the dominant launch ----------------------------------
+    peak, peak_kind = read_peaks()
+    ab = algorithmic_bytes(w)
+    dom = "bwd" if ms_bwd >= ms_fwd else "fwd"
+    dom_ms = ms_bwd if dom == "bwd" else ms_fwd
+    achieved = ab[dom] / (dom_ms / 1e3) / 1e9
+    kernels = {
+        "fwd": {"kernel": "fwd_kernel (msda_forward_fused)", "ms": ms_fwd,
+                "algorithmic_bytes": ab["fwd"],
+                "GB_s": ab["fwd"] / (ms_fwd / 1e3) / 1e9},
+        "bwd": {"kernel": "memset + bwd_kernel (msda_backward)", "ms": ms_bwd,
+                "algorithmic_bytes": ab["bwd"],
+                "GB_s": ab["bwd"] / (ms_bwd / 1e3) / 1e9},
+    }
+    for k in kernels.values():
+        k["frac_of_" + peak_kind] = k["GB_s"] / peak
+    roofline = {
+        "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+        "frac": achieved / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+        if peak_kind == "measured" else "fallback 6.65 TB/s",
+        "traffic": read_traffic(args.workload, dom), "kernel": kernels[dom]["kernel"],
+        "algorithmic_bytes_per_launch": ab[dom],
+    }
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, inp)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC,
+            "value": value_qps,
+            "unit": "queries/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": ms_step,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic (seeded numpy PCG64; shapes of the Deformable DETR "
+                    "encoder/decoder, no dataset or trained weights)",
+            "config": {
+                "workload": WORKLOAD_TEXT[args.workload],
+                "value_dtype": w.value_dtype,
+                "global_batch": w.N * world,
+                "queries_per_step": queries * world,
+                "parallelism": f"dp{world} (independent batches, no collective)",
+                "l2": "flushed before every timed step (memset of 2x L2, outside the events)",
+            },
+            "effective_GB_s": (ab["fwd"] + ab["bwd"]) / (ms_step / 1e3) / 1e9,
+            "kernels": kernels,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": 2 * K,
+            "clocks": clocks.summary(),
+            "impl": "ours",
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def _pci_bus_id(torch, device):
+    try:
+        p = torch.cuda.get_device_properties(device)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        return None
+
+
+def _nvml_index(local: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    parts = [p for p in vis.split(",") if p.strip()]
+    try:
+        return int(parts[local])
+    except Exception:
+        return local
+
+
+def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_dev, queries):
+    """The same step through the public binding, starting from pinned host
+    buffers: H2D of the step's inputs, fused forward, backward, D2H of the
+    step's results (out, grad_value, grad_sampling_locations,
+    grad_attention_weights), all inside the timed events."""
+    from scale_deformable_attention_02_b200 import msda_backward, msda_forward_fused
+
+    def pinned(a):
+        a = np.ascontiguousarray(a)
+        t = torch.from_numpy(a.view(np.int16) if a.dtype == np.uint16 else a)
+        return t.pin_memory()
+
+    names = ["value", "reference_points", "offsets", "logits", "grad_out"]
+    h_in = {k: pinned(inp[k]) for k in names}
+    d_in = {k: torch.empty(h_in[k].shape, dtype=h_in[k].dtype, device=device) for k in names}
+    res_shapes = {"out": (w.N, w.queries, w.M * w.D), "grad_value": (w.N, w.S, w.M, w.D),
+                  "grad_loc": tuple(inp["offsets"].shape), "grad_attn": tuple(inp["logits"].shape)}
+    h_out = {k: torch.empty(s, dtype=torch.float32).pin_memory() for k, s in res_shapes.items()}
+    d_out = {k: torch.empty(s, dtype=torch.float32, device=device) for k, s in res_shapes.items()}
+    loc = torch.empty(tuple(inp["offsets"].shape), device=device)
+    attn = torch.empty(tuple(inp["logits"].shape), device=device)
+    bf16 = w.value_dtype == "bf16"
+
+    def one():
+        for k in names:
+            d_in[k].copy_(h_in[k], non_blocking=True)
+        v = d_in["value"].view(torch.bfloat16) if bf16 else d_in["value"]
+        msda_forward_fused(v, sh, starts, d_in["reference_points"], d_in["offsets"],
+                           d_in["logits"], out=d_out["out"], sampling_locations_out=loc,
+                           attention_weights_out=attn, stream=stream)
+        msda_backward(v, sh, starts, loc, attn, d_in["grad_out"],
+                      grad_value=d_out["grad_value"], grad_sampling_locations=d_out["grad_loc"],
+                      grad_attention_weights=d_out["grad_attn"], stream=stream)
+        for k in res_shapes:
+            h_out[k].copy_(d_out[k], non_blocking=True)
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize()
+    n = max(1, args.e2e_steps)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n):
+        one()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t = torch.tensor([e0.elapsed_time(e1) / n], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    h2d = sum(h_in[k].numel() * h_in[k].element_size() for k in names)
+    d2h = sum(h_out[k].numel() * h_out[k].element_size() for k in res_shapes)
+    return {"value": queries * world / (ms / 1e3), "unit": "queries/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
+            "api": "scale_deformable_attention_02_b200.msda_forward_fused + msda_backward "
+                   "on pinned host buffers copied in and out every step"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs (the oracle is test infrastructure; only these legs run it)
+# ---------------------------------------------------------------------------
+def _oracle_sample(w, inp, frac_queries: int):
+    """Every frac-th query of every batch entry (the oracle's cost per query
+    is uniform, so a strided sample keeps the workload's mix)."""
+    qs = np.arange(0, w.queries, frac_queries)
+    pick = lambda a: np.ascontiguousarray(a[:, qs])  # noqa: E731
+    return {"value": inp["value"], "spatial_shapes": inp["spatial_shapes"],
+            "reference_points": pick(inp["reference_points"]), "offsets": pick(inp["offsets"]),
+            "logits": pick(inp["logits"]), "grad_out": pick(inp["grad_out"]),
+            "queries": w.N * len(qs)}
+
+
+def _oracle_step(oracle, s):
+    out, loc, A = oracle.forward_fused(s["value"], s["spatial_shapes"], s["reference_points"],
+                                       s["offsets"], s["logits"])
+    oracle.backward(s["value"], s["spatial_shapes"], loc, A, s["grad_out"])
+
+
+def cpu_baseline(w, inp, min_seconds: float = 10.0):
+    import oracle
+    threads = os.cpu_count() or 1
+    oracle.set_threads(threads)
+    s = _oracle_sample(w, inp, 1)
+    t0 = time.perf_counter()
+    passes = 0
+    while True:
+        _oracle_step(oracle, s)
+        passes += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or passes >= 20:
+            break
+    return {"value": s["queries"] * passes / el, "unit": "queries/s", "cores": threads,
+            "kind": "oracle",
+            "sample": f"{passes} full pass(es) of the workload ({s['queries']} queries each: "
+                      f"fused forward + backward) on the plain C oracle, fp64 accumulation, "
+                      f"OpenMP over {threads} threads, {el:.1f} s"}
+
+
+def run_reference(args):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    w = rank_workload(args.workload, 0)
+    inp = wl.make_inputs(w)
+    stride = 8 if args.workload == "stress" else 4
+    s = _oracle_sample(w, inp, stride)
+    threads = os.cpu_count() or 1
+    oracle.set_threads(threads)
+    for _ in range(args.warmup):
+        _oracle_step(oracle, s)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        _oracle_step(oracle, s)
+        times.append(time.perf_counter() - t0)
+    sec = statistics.fmean(times)
+    qps = s["queries"] / sec
+    sample = (f"every {stride}th query of each of the {w.N} batch entries ({s['queries']} "
+              f"queries per step), fused forward + backward on the plain C oracle")
+    line = {
+        "metric": METRIC, "value": qps, "unit": "queries/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded numpy PCG64)",
+        "config": {"workload": WORKLOAD_TEXT[args.workload], "value_dtype": w.value_dtype,
+                   "global_batch": w.N, "parallelism": "host cores (OpenMP)"},
+        "impl": "reference",
+        "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": qps, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

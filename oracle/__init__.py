@@ -67,6 +67,8 @@ def lib():
             _lib.ora_softmax.argtypes = [P, P, I64, I64]
             _lib.ora_locations_f32.restype = None
             _lib.ora_locations_f32.argtypes = [P, P, P, Dims, P]
+            _lib.ora_locations_box_f32.restype = None
+            _lib.ora_locations_box_f32.argtypes = [P, P, Dims, P]
             _lib.ora_locations_f64.restype = None
             _lib.ora_locations_f64.argtypes = [P, P, P, Dims, P]
             _lib.ora_backward.restype = None
@@ -134,6 +136,17 @@ def locations_f32(ref: np.ndarray, off: np.ndarray, shapes: np.ndarray) -> np.nd
     loc = np.empty_like(off)
     lib().ora_locations_f32(_ptr(ref), _ptr(off), _ptr(shapes),
                             Dims(N, Lq, 0, M, 0, L, K), _ptr(loc))
+    return loc
+
+
+def locations_box_f32(box: np.ndarray, off: np.ndarray) -> np.ndarray:
+    """Box references (cx, cy, w, h): loc = (cx, cy) + off * (w, h), fp32."""
+    box = np.ascontiguousarray(box, dtype=np.float32)
+    off = np.ascontiguousarray(off, dtype=np.float32)
+    N, Lq, M, L, K, _ = off.shape
+    assert box.shape == (N, Lq, 4)
+    loc = np.empty_like(off)
+    lib().ora_locations_box_f32(_ptr(box), _ptr(off), Dims(N, Lq, 0, M, 0, L, K), _ptr(loc))
     return loc
 
 

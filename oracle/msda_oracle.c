@@ -269,6 +269,30 @@ void ora_locations_f32(const float *ref, const float *off, const int64_t *shapes
                     }
 }
 
+/*
+ * Box reference (iterative bounding-box refinement, "Deformable DETR" wiki
+ * page, "Variants"): the previous layer's box (cx, cy, w, h) is the reference
+ * and the offsets are scaled by the box size, so in normalised units
+ * loc_x = cx + off_x * w, loc_y = cy + off_y * h (offsets in box units; the
+ * page's 1/(2K) scaling of the initial offsets is a property of the offsets,
+ * not of this map).  fp32: one IEEE multiply, then one IEEE add.
+ *   box [N,Lq,4]   off [N,Lq,M,L,K,2]   loc [N,Lq,M,L,K,2]
+ */
+void ora_locations_box_f32(const float *box, const float *off, ora_dims d, float *loc)
+{
+    const int64_t N = d.N, Lq = d.Lq, M = d.M, L = d.L, K = d.K;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t q = 0; q < Lq; ++q)
+            for (int64_t j = 0; j < M * L * K; ++j) {
+                const int64_t i = (n * Lq + q) * M * L * K + j;
+                const float *b = box + 4 * (n * Lq + q);
+                float dx = off[2 * i] * b[2];
+                float dy = off[2 * i + 1] * b[3];
+                loc[2 * i] = b[0] + dx;
+                loc[2 * i + 1] = b[1] + dy;
+            }
+}
+
 /* The same map in fp64 (finite-difference checks of the fused chain). */
 void ora_locations_f64(const double *ref, const double *off, const int64_t *shapes,
                        ora_dims d, double *loc)

@@ -1,0 +1,15 @@
+"""Multi-scale deformable attention (MSDeformAttn) core for NVIDIA B200.
+
+The compute path is libmsda.so (hand-written sm_100a CUDA kernels behind the
+C ABI in include/msda.h); this package is its thin Python binding, plus the
+seeded synthetic workloads used by the tests and the benchmark.
+"""
+from ._lib import LIB_PATH, MSDA_BF16, MSDA_F32
+from .api import (MsdaError, msda_backward, msda_debug_sample_points, msda_forward,
+                  msda_forward_fused, msda_level_start_index)
+
+__all__ = [
+    "LIB_PATH", "MSDA_BF16", "MSDA_F32", "MsdaError", "msda_backward",
+    "msda_debug_sample_points", "msda_forward", "msda_forward_fused",
+    "msda_level_start_index",
+]

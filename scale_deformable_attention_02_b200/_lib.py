@@ -1,0 +1,66 @@
+"""ctypes view of libmsda.so (the C ABI in include/msda.h and
+include/msda_debug.h).  No fallback: if the library is missing or does not
+load, every call raises."""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmsda.so")
+
+MSDA_F32 = 0
+MSDA_BF16 = 1
+
+STATUS_NAMES = {
+    0: "MSDA_OK", 1: "MSDA_ERR_NULL", 2: "MSDA_ERR_SHAPE", 3: "MSDA_ERR_LEVELS",
+    4: "MSDA_ERR_DTYPE", 5: "MSDA_ERR_ALIGN", 6: "MSDA_ERR_ALIAS",
+    7: "MSDA_ERR_UNSUPPORTED", 8: "MSDA_ERR_CUDA",
+}
+
+# Every function declared in include/*.h, with its ctypes signature.
+P = ctypes.c_void_p
+I64 = ctypes.c_int64
+INT = ctypes.c_int
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_int64) for k in ("N", "Lq", "S", "M", "D", "L", "K")]
+
+
+SIGNATURES = {
+    "msda_status_string": (ctypes.c_char_p, [INT]),
+    "msda_abi_version": (INT, []),
+    "msda_last_cuda_error": (INT, []),
+    "msda_level_start_index": (INT, [P, I64, P, P]),
+    "msda_forward": (INT, [P, INT, P, P, P, P, P, Dims, P]),
+    "msda_forward_fused": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, Dims, P]),
+    "msda_backward": (INT, [P, INT, P, P, P, P, P, P, P, P, Dims, P]),
+    "msda_debug_sample_points": (INT, [P, P, P, Dims, P, P, P, P, P, P, P]),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libmsda.so (built in-tree by scale_deformable_attention_02_b200.build)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(
+                    f"{LIB_PATH} is not built; run `python -m "
+                    "scale_deformable_attention_02_b200.build` (needs nvcc)")
+            lib = ctypes.CDLL(LIB_PATH)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(lib, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = lib
+        return _lib
+
+
+def status_string(code: int) -> str:
+    return load().msda_status_string(int(code)).decode()

@@ -1,0 +1,247 @@
+"""Python binding of the C ABI: argument marshalling only.
+
+Each function takes torch CUDA tensors, checks that their dtypes, devices,
+shapes and contiguity agree, allocates missing outputs with torch, and calls
+the C entry point of the same name on the current (or given) CUDA stream.
+Every step of the computation runs in libmsda.so's kernels; there is no
+other code path.
+
+Layouts (see include/msda.h):
+  value [N,S,M,D] float32 | bfloat16, sampling_locations [N,Lq,M,L,K,2],
+  attention_weights / logits [N,Lq,M,L,K], reference_points [N,Lq,2|4],
+  offsets [N,Lq,M,L,K,2], out / grad_out [N,Lq,M*D] (all float32 except value),
+  spatial_shapes [L,2] int64 (H, W) and level_start_index [L] int64 on the host.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from . import _lib
+
+
+class MsdaError(RuntimeError):
+    """A non-OK status from libmsda.so."""
+
+    def __init__(self, status: int, where: str):
+        self.status = int(status)
+        msg = f"{where}: {_lib.status_string(status)}"
+        if self.status == 8:
+            msg += f" (cudaError {_lib.load().msda_last_cuda_error()})"
+        super().__init__(msg)
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise MsdaError(status, where)
+
+
+def _host_i64(x, name: str) -> np.ndarray:
+    if isinstance(x, torch.Tensor):
+        x = x.detach().to("cpu").numpy()
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.int64))
+    if a.ndim == 0:
+        raise ValueError(f"{name} must be an array")
+    return a
+
+
+def _hptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(device: torch.device, stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    if isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    return ctypes.c_void_p(int(stream))
+
+
+def _value_dtype(value: torch.Tensor) -> int:
+    if value.dtype == torch.float32:
+        return _lib.MSDA_F32
+    if value.dtype == torch.bfloat16:
+        return _lib.MSDA_BF16
+    raise TypeError(f"value must be float32 or bfloat16, got {value.dtype}")
+
+
+def _need(t: torch.Tensor, name: str, shape, device, dtype=torch.float32):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _levels(spatial_shapes, level_start_index):
+    shapes = _host_i64(spatial_shapes, "spatial_shapes").reshape(-1, 2)
+    if level_start_index is None:
+        starts, _ = msda_level_start_index(shapes)
+    else:
+        starts = _host_i64(level_start_index, "level_start_index").reshape(-1)
+    return shapes, starts
+
+
+def msda_level_start_index(spatial_shapes) -> tuple[np.ndarray, int]:
+    """Level start rows (exclusive prefix sum of H*W) and S, from the C ABI."""
+    shapes = _host_i64(spatial_shapes, "spatial_shapes").reshape(-1, 2)
+    starts = np.zeros(shapes.shape[0], dtype=np.int64)
+    S = ctypes.c_int64(0)
+    _check(_lib.load().msda_level_start_index(_hptr(shapes), shapes.shape[0], _hptr(starts),
+                                              ctypes.byref(S)), "msda_level_start_index")
+    return starts, int(S.value)
+
+
+def _value_dims(value: torch.Tensor, shapes: np.ndarray, lead):
+    if value.dim() != 4:
+        raise ValueError("value must be [N, S, M, D]")
+    N, S, M, D = value.shape
+    L = shapes.shape[0]
+    if len(lead) < 5:
+        raise ValueError("per-sample tensors must be [N, Lq, M, L, K(, 2)]")
+    if lead[0] != N or lead[2] != M or lead[3] != L:
+        raise ValueError(f"per-sample tensor shape {tuple(lead)} disagrees with value "
+                         f"{tuple(value.shape)} and L={L}")
+    Lq, K = lead[1], lead[4]
+    return _lib.Dims(N, Lq, S, M, D, L, K)
+
+
+def msda_forward(value: torch.Tensor, spatial_shapes, level_start_index,
+                 sampling_locations: torch.Tensor, attention_weights: torch.Tensor,
+                 out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[n,q,m*D:(m+1)*D] = sum_{l,k} A * bilinear(value level l, head m, loc)."""
+    dev = value.device
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    d = _value_dims(value, shapes, tuple(sampling_locations.shape))
+    _need(sampling_locations, "sampling_locations", (d.N, d.Lq, d.M, d.L, d.K, 2), dev)
+    _need(attention_weights, "attention_weights", (d.N, d.Lq, d.M, d.L, d.K), dev)
+    if not value.is_contiguous():
+        raise ValueError("value must be contiguous")
+    if out is None:
+        out = torch.empty((d.N, d.Lq, d.M * d.D), device=dev, dtype=torch.float32)
+    _need(out, "out", (d.N, d.Lq, d.M * d.D), dev)
+    _check(_lib.load().msda_forward(_dptr(value), _value_dtype(value), _hptr(shapes),
+                                    _hptr(starts), _dptr(sampling_locations),
+                                    _dptr(attention_weights), _dptr(out), d,
+                                    _stream_handle(dev, stream)), "msda_forward")
+    return out
+
+
+def msda_forward_fused(value: torch.Tensor, spatial_shapes, level_start_index,
+                       reference_points: torch.Tensor, offsets: torch.Tensor,
+                       logits: torch.Tensor, out: torch.Tensor | None = None,
+                       sampling_locations_out: torch.Tensor | None = None,
+                       attention_weights_out: torch.Tensor | None = None,
+                       return_sampling: bool = False, stream=None):
+    """Fused forward: softmax over the L*K logits of each head and the
+    location map (ref + off/W_l, or box: (cx,cy) + off*(w,h)) inside the
+    kernel.  Returns out, or (out, sampling_locations, attention_weights) when
+    return_sampling is true (those outputs are then allocated if not given)."""
+    dev = value.device
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    d = _value_dims(value, shapes, tuple(offsets.shape))
+    rdim = reference_points.shape[-1] if reference_points.dim() == 3 else -1
+    if rdim not in (2, 4):
+        raise ValueError("reference_points must be [N, Lq, 2] or [N, Lq, 4]")
+    _need(reference_points, "reference_points", (d.N, d.Lq, rdim), dev)
+    _need(offsets, "offsets", (d.N, d.Lq, d.M, d.L, d.K, 2), dev)
+    _need(logits, "logits", (d.N, d.Lq, d.M, d.L, d.K), dev)
+    if not value.is_contiguous():
+        raise ValueError("value must be contiguous")
+    if out is None:
+        out = torch.empty((d.N, d.Lq, d.M * d.D), device=dev, dtype=torch.float32)
+    _need(out, "out", (d.N, d.Lq, d.M * d.D), dev)
+    if return_sampling:
+        if sampling_locations_out is None:
+            sampling_locations_out = torch.empty_like(offsets)
+        if attention_weights_out is None:
+            attention_weights_out = torch.empty_like(logits)
+    if sampling_locations_out is not None:
+        _need(sampling_locations_out, "sampling_locations_out", tuple(offsets.shape), dev)
+    if attention_weights_out is not None:
+        _need(attention_weights_out, "attention_weights_out", tuple(logits.shape), dev)
+    _check(_lib.load().msda_forward_fused(
+        _dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
+        _dptr(reference_points), int(rdim), _dptr(offsets), _dptr(logits), _dptr(out),
+        _dptr(sampling_locations_out), _dptr(attention_weights_out), d,
+        _stream_handle(dev, stream)), "msda_forward_fused")
+    if return_sampling:
+        return out, sampling_locations_out, attention_weights_out
+    return out
+
+
+def msda_backward(value: torch.Tensor, spatial_shapes, level_start_index,
+                  sampling_locations: torch.Tensor, attention_weights: torch.Tensor,
+                  grad_out: torch.Tensor, grad_value: torch.Tensor | None = None,
+                  grad_sampling_locations: torch.Tensor | None = None,
+                  grad_attention_weights: torch.Tensor | None = None,
+                  need_sampling_grad: bool = True, need_weight_grad: bool = True,
+                  stream=None):
+    """Gradients of msda_forward.  Returns (grad_value [fp32], grad_loc or
+    None, grad_attn or None)."""
+    dev = value.device
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    d = _value_dims(value, shapes, tuple(sampling_locations.shape))
+    _need(sampling_locations, "sampling_locations", (d.N, d.Lq, d.M, d.L, d.K, 2), dev)
+    _need(attention_weights, "attention_weights", (d.N, d.Lq, d.M, d.L, d.K), dev)
+    _need(grad_out, "grad_out", (d.N, d.Lq, d.M * d.D), dev)
+    if not value.is_contiguous():
+        raise ValueError("value must be contiguous")
+    if grad_value is None:
+        grad_value = torch.empty(tuple(value.shape), device=dev, dtype=torch.float32)
+    _need(grad_value, "grad_value", tuple(value.shape), dev)
+    if grad_sampling_locations is None and need_sampling_grad:
+        grad_sampling_locations = torch.empty_like(sampling_locations)
+    if grad_attention_weights is None and need_weight_grad:
+        grad_attention_weights = torch.empty_like(attention_weights)
+    if grad_sampling_locations is not None:
+        _need(grad_sampling_locations, "grad_sampling_locations",
+              tuple(sampling_locations.shape), dev)
+    if grad_attention_weights is not None:
+        _need(grad_attention_weights, "grad_attention_weights",
+              tuple(attention_weights.shape), dev)
+    _check(_lib.load().msda_backward(
+        _dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
+        _dptr(sampling_locations), _dptr(attention_weights), _dptr(grad_out),
+        _dptr(grad_value), _dptr(grad_sampling_locations), _dptr(grad_attention_weights), d,
+        _stream_handle(dev, stream)), "msda_backward")
+    return grad_value, grad_sampling_locations, grad_attention_weights
+
+
+def msda_debug_sample_points(spatial_shapes, level_start_index,
+                             sampling_locations: torch.Tensor, stream=None) -> dict:
+    """Per-sample cell record computed by the kernels' own cell arithmetic."""
+    dev = sampling_locations.device
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    if sampling_locations.dim() != 6:
+        raise ValueError("sampling_locations must be [N, Lq, M, L, K, 2]")
+    N, Lq, M, L, K, _ = sampling_locations.shape
+    S = int(sum(int(h) * int(w) for h, w in shapes))
+    d = _lib.Dims(N, Lq, S, M, 4, L, K)
+    _need(sampling_locations, "sampling_locations", (N, Lq, M, L, K, 2), dev)
+    n = N * Lq * M * L * K
+    r = {
+        "valid": torch.empty(n, device=dev, dtype=torch.int32),
+        "x0": torch.empty(n, device=dev, dtype=torch.int32),
+        "y0": torch.empty(n, device=dev, dtype=torch.int32),
+        "x": torch.empty(n, device=dev, dtype=torch.float32),
+        "y": torch.empty(n, device=dev, dtype=torch.float32),
+        "rows": torch.empty((n, 4), device=dev, dtype=torch.int64),
+    }
+    _check(_lib.load().msda_debug_sample_points(
+        _hptr(shapes), _hptr(starts), _dptr(sampling_locations), d, _dptr(r["valid"]),
+        _dptr(r["x0"]), _dptr(r["y0"]), _dptr(r["x"]), _dptr(r["y"]), _dptr(r["rows"]),
+        _stream_handle(dev, stream)), "msda_debug_sample_points")
+    return r

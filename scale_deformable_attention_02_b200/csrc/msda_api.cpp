@@ -1,0 +1,351 @@
+// msda_api.cpp -- the C entry points: argument checks, then launches.
+//
+// Every check runs before any CUDA call, so a rejected call has no side
+// effect at all (and the checks themselves work on a machine without a GPU).
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "msda.h"
+#include "msda_debug.h"
+#include "msda_internal.h"
+
+namespace {
+
+using msda::Levels;
+using msda::kMaxLK;
+
+constexpr int kAbiVersion = 10000;  // 1.0.0
+constexpr int64_t kI32Max = 2147483647LL;
+constexpr int64_t kGuard = (int64_t)1 << 62;
+
+thread_local int g_last_cuda_error = 0;
+
+// a * b with a, b >= 0; false if the product exceeds `limit`.
+bool mul_le(int64_t a, int64_t b, int64_t limit, int64_t *out)
+{
+    if (a != 0 && b > limit / a) return false;
+    *out = a * b;
+    return *out <= limit;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+struct Span {
+    const void *p;
+    int64_t bytes;
+};
+
+bool overlap(Span a, Span b)
+{
+    if (!a.p || !b.p || a.bytes <= 0 || b.bytes <= 0) return false;
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(a.p);
+    const uintptr_t pb = reinterpret_cast<uintptr_t>(b.p);
+    return pa < pb + (uintptr_t)b.bytes && pb < pa + (uintptr_t)a.bytes;
+}
+
+// True if any output overlaps any input or another output.
+bool any_alias(const Span *outs, int nout, const Span *ins, int nin)
+{
+    for (int i = 0; i < nout; ++i) {
+        for (int j = 0; j < nin; ++j)
+            if (overlap(outs[i], ins[j])) return true;
+        for (int j = i + 1; j < nout; ++j)
+            if (overlap(outs[i], outs[j])) return true;
+    }
+    return false;
+}
+
+// Validated problem: element counts and launch-side metadata.
+struct Problem {
+    int64_t items;    // N*Lq*M
+    int64_t samples;  // N*Lq*M*L*K
+    int64_t n_value;  // N*S*M*D
+    int64_t n_out;    // N*Lq*M*D
+    int esz;          // value element size
+    int nchunks;      // 16-byte chunks per value row
+    int lanes;        // lanes per row: next power of two >= nchunks
+    Levels lv;
+};
+
+// Dims, level metadata and size limits (no pointers).
+msda_status check_dims(msda_dtype dt, const int64_t *shapes, const int64_t *starts,
+                       const msda_dims &d, Problem *pr)
+{
+    if (!shapes || !starts) return MSDA_ERR_NULL;
+    if (dt != MSDA_F32 && dt != MSDA_BF16) return MSDA_ERR_DTYPE;
+    if (d.N < 0 || d.Lq < 0 || d.S < 0 || d.M < 1 || d.D < 1 || d.L < 1 || d.K < 1)
+        return MSDA_ERR_SHAPE;
+    if (d.L > kMaxLK || d.K > kMaxLK || d.L * d.K > kMaxLK) return MSDA_ERR_UNSUPPORTED;
+    memset(&pr->lv, 0, sizeof pr->lv);
+    int64_t acc = 0;
+    for (int64_t l = 0; l < d.L; ++l) {
+        const int64_t H = shapes[2 * l], W = shapes[2 * l + 1];
+        if (H < 0 || W < 0) return MSDA_ERR_SHAPE;
+        if (H > kI32Max || W > kI32Max) return MSDA_ERR_UNSUPPORTED;
+        if (starts[l] != acc) return MSDA_ERR_LEVELS;
+        acc += H * W;  // < 2^62: both factors < 2^31
+        if (acc > kI32Max) return MSDA_ERR_UNSUPPORTED;
+        pr->lv.H[l] = (int)H;
+        pr->lv.W[l] = (int)W;
+        pr->lv.start[l] = (int)starts[l];
+    }
+    if (acc != d.S) return MSDA_ERR_LEVELS;
+    pr->esz = dt == MSDA_F32 ? 4 : 2;
+    if (d.D > 512) return MSDA_ERR_UNSUPPORTED;
+    const int64_t rowbytes = d.D * pr->esz;
+    if (rowbytes % 16 != 0) return MSDA_ERR_ALIGN;
+    if (rowbytes > 512) return MSDA_ERR_UNSUPPORTED;  // at most one 16-byte chunk per lane
+    if (d.Lq > kI32Max || d.M > kI32Max) return MSDA_ERR_UNSUPPORTED;
+    int64_t smd, md, t;
+    if (!mul_le(d.M, d.D, kI32Max, &md) || !mul_le(d.S, md, kI32Max, &smd))
+        return MSDA_ERR_UNSUPPORTED;  // row offsets inside one batch entry are int32
+    if (!mul_le(d.N, smd, kGuard, &pr->n_value)) return MSDA_ERR_UNSUPPORTED;
+    if (!mul_le(d.N, d.Lq, kGuard, &t) || !mul_le(t, d.M, kGuard, &pr->items))
+        return MSDA_ERR_UNSUPPORTED;
+    if (!mul_le(pr->items, d.L * d.K * 2, kGuard, &t)) return MSDA_ERR_UNSUPPORTED;
+    pr->samples = pr->items * d.L * d.K;
+    pr->n_out = pr->items * d.D;
+    pr->nchunks = (int)(rowbytes / 16);
+    int lanes = 1;
+    while (lanes < pr->nchunks) lanes <<= 1;
+    pr->lanes = lanes;
+    return MSDA_OK;
+}
+
+msda_status cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess) return MSDA_OK;
+    g_last_cuda_error = (int)e;
+    return MSDA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *msda_status_string(msda_status status)
+{
+    switch (status) {
+    case MSDA_OK: return "MSDA_OK";
+    case MSDA_ERR_NULL: return "MSDA_ERR_NULL: a required pointer is NULL";
+    case MSDA_ERR_SHAPE: return "MSDA_ERR_SHAPE: a dimension is out of range";
+    case MSDA_ERR_LEVELS:
+        return "MSDA_ERR_LEVELS: spatial_shapes, level_start_index and S disagree";
+    case MSDA_ERR_DTYPE: return "MSDA_ERR_DTYPE: unknown value dtype";
+    case MSDA_ERR_ALIGN: return "MSDA_ERR_ALIGN: a pointer or row size breaks the alignment rule";
+    case MSDA_ERR_ALIAS: return "MSDA_ERR_ALIAS: an output overlaps an input or another output";
+    case MSDA_ERR_UNSUPPORTED: return "MSDA_ERR_UNSUPPORTED: outside this build's limits";
+    case MSDA_ERR_CUDA: return "MSDA_ERR_CUDA: the CUDA runtime reported an error";
+    }
+    return "MSDA_ERR_UNKNOWN";
+}
+
+int msda_abi_version(void) { return kAbiVersion; }
+
+int msda_last_cuda_error(void) { return g_last_cuda_error; }
+
+msda_status msda_level_start_index(const int64_t *spatial_shapes, int64_t L,
+                                   int64_t *level_start_index, int64_t *S_out)
+{
+    if (!spatial_shapes || !level_start_index) return MSDA_ERR_NULL;
+    if (L < 1) return MSDA_ERR_SHAPE;
+    int64_t acc = 0;
+    for (int64_t l = 0; l < L; ++l) {
+        const int64_t H = spatial_shapes[2 * l], W = spatial_shapes[2 * l + 1];
+        if (H < 0 || W < 0) return MSDA_ERR_SHAPE;
+        int64_t hw;
+        if (!mul_le(H, W, kGuard, &hw) || acc > kGuard - hw) return MSDA_ERR_UNSUPPORTED;
+        level_start_index[l] = acc;
+        acc += hw;
+    }
+    if (S_out) *S_out = acc;
+    return MSDA_OK;
+}
+
+msda_status msda_forward(const void *value, msda_dtype value_dtype,
+                         const int64_t *spatial_shapes, const int64_t *level_start_index,
+                         const float *sampling_locations, const float *attention_weights,
+                         float *out, msda_dims d, msda_stream_t stream)
+{
+    Problem pr;
+    msda_status st = check_dims(value_dtype, spatial_shapes, level_start_index, d, &pr);
+    if (st != MSDA_OK) return st;
+    if (pr.n_out > 0 && (!sampling_locations || !attention_weights || !out))
+        return MSDA_ERR_NULL;
+    if (pr.n_out > 0 && pr.n_value > 0 && !value) return MSDA_ERR_NULL;
+    if (!aligned(value, 16) || !aligned(out, 16) || !aligned(sampling_locations, 8) ||
+        !aligned(attention_weights, 4))
+        return MSDA_ERR_ALIGN;
+    const Span outs[] = {{out, pr.n_out * 4}};
+    const Span ins[] = {{value, pr.n_value * pr.esz},
+                        {sampling_locations, pr.samples * 8},
+                        {attention_weights, pr.samples * 4}};
+    if (any_alias(outs, 1, ins, 3)) return MSDA_ERR_ALIAS;
+    if (pr.n_out == 0) return MSDA_OK;
+
+    msda::FwdParams p;
+    memset(&p, 0, sizeof p);
+    p.value = value;
+    p.loc = sampling_locations;
+    p.attn = attention_weights;
+    p.out = out;
+    p.items = pr.items;
+    p.Lq = (int)d.Lq;
+    p.S = (int)d.S;
+    p.M = (int)d.M;
+    p.D = (int)d.D;
+    p.L = (int)d.L;
+    p.K = (int)d.K;
+    p.nchunks = pr.nchunks;
+    p.lv = pr.lv;
+    return cuda_status(msda::launch_forward(p, value_dtype == MSDA_BF16, false, pr.lanes,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+msda_status msda_forward_fused(const void *value, msda_dtype value_dtype,
+                               const int64_t *spatial_shapes,
+                               const int64_t *level_start_index,
+                               const float *reference_points, int reference_dim,
+                               const float *offsets, const float *logits, float *out,
+                               float *sampling_locations_out, float *attention_weights_out,
+                               msda_dims d, msda_stream_t stream)
+{
+    Problem pr;
+    msda_status st = check_dims(value_dtype, spatial_shapes, level_start_index, d, &pr);
+    if (st != MSDA_OK) return st;
+    if (reference_dim != 2 && reference_dim != 4) return MSDA_ERR_SHAPE;
+    if (pr.n_out > 0 && (!reference_points || !offsets || !logits || !out))
+        return MSDA_ERR_NULL;
+    if (pr.n_out > 0 && pr.n_value > 0 && !value) return MSDA_ERR_NULL;
+    if (!aligned(value, 16) || !aligned(out, 16) || !aligned(reference_points, 8) ||
+        !aligned(offsets, 8) || !aligned(logits, 4) || !aligned(sampling_locations_out, 8) ||
+        !aligned(attention_weights_out, 4))
+        return MSDA_ERR_ALIGN;
+    const int64_t nq = pr.items / d.M;
+    const Span outs[] = {{out, pr.n_out * 4},
+                         {sampling_locations_out, pr.samples * 8},
+                         {attention_weights_out, pr.samples * 4}};
+    const Span ins[] = {{value, pr.n_value * pr.esz},
+                        {reference_points, nq * reference_dim * 4},
+                        {offsets, pr.samples * 8},
+                        {logits, pr.samples * 4}};
+    if (any_alias(outs, 3, ins, 4)) return MSDA_ERR_ALIAS;
+    if (pr.n_out == 0) return MSDA_OK;
+
+    msda::FwdParams p;
+    memset(&p, 0, sizeof p);
+    p.value = value;
+    p.ref = reference_points;
+    p.ref_dim = reference_dim;
+    p.off = offsets;
+    p.logits = logits;
+    p.out = out;
+    p.loc_out = sampling_locations_out;
+    p.attn_out = attention_weights_out;
+    p.items = pr.items;
+    p.Lq = (int)d.Lq;
+    p.S = (int)d.S;
+    p.M = (int)d.M;
+    p.D = (int)d.D;
+    p.L = (int)d.L;
+    p.K = (int)d.K;
+    p.nchunks = pr.nchunks;
+    p.lv = pr.lv;
+    return cuda_status(msda::launch_forward(p, value_dtype == MSDA_BF16, true, pr.lanes,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+msda_status msda_backward(const void *value, msda_dtype value_dtype,
+                          const int64_t *spatial_shapes, const int64_t *level_start_index,
+                          const float *sampling_locations, const float *attention_weights,
+                          const float *grad_out, float *grad_value,
+                          float *grad_sampling_locations, float *grad_attention_weights,
+                          msda_dims d, msda_stream_t stream)
+{
+    Problem pr;
+    msda_status st = check_dims(value_dtype, spatial_shapes, level_start_index, d, &pr);
+    if (st != MSDA_OK) return st;
+    if (pr.n_value > 0 && !grad_value) return MSDA_ERR_NULL;
+    if (pr.n_out > 0 && (!sampling_locations || !attention_weights || !grad_out))
+        return MSDA_ERR_NULL;
+    if (pr.n_out > 0 && pr.n_value > 0 && !value) return MSDA_ERR_NULL;
+    if (!aligned(value, 16) || !aligned(grad_out, 16) || !aligned(grad_value, 16) ||
+        !aligned(sampling_locations, 8) || !aligned(attention_weights, 4) ||
+        !aligned(grad_sampling_locations, 8) || !aligned(grad_attention_weights, 4))
+        return MSDA_ERR_ALIGN;
+    const Span outs[] = {{grad_value, pr.n_value * 4},
+                         {grad_sampling_locations, pr.samples * 8},
+                         {grad_attention_weights, pr.samples * 4}};
+    const Span ins[] = {{value, pr.n_value * pr.esz},
+                        {sampling_locations, pr.samples * 8},
+                        {attention_weights, pr.samples * 4},
+                        {grad_out, pr.n_out * 4}};
+    if (any_alias(outs, 3, ins, 4)) return MSDA_ERR_ALIAS;
+
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (pr.n_value > 0) {
+        st = cuda_status(cudaMemsetAsync(grad_value, 0, (size_t)pr.n_value * 4, s));
+        if (st != MSDA_OK) return st;
+    }
+    if (pr.n_out == 0) return MSDA_OK;
+
+    msda::BwdParams p;
+    memset(&p, 0, sizeof p);
+    p.value = value;
+    p.loc = sampling_locations;
+    p.attn = attention_weights;
+    p.grad_out = grad_out;
+    p.grad_value = grad_value;
+    p.grad_loc = grad_sampling_locations;
+    p.grad_attn = grad_attention_weights;
+    p.items = pr.items;
+    p.Lq = (int)d.Lq;
+    p.S = (int)d.S;
+    p.M = (int)d.M;
+    p.D = (int)d.D;
+    p.L = (int)d.L;
+    p.K = (int)d.K;
+    p.nchunks = pr.nchunks;
+    p.lv = pr.lv;
+    return cuda_status(
+        msda::launch_backward(p, value_dtype == MSDA_BF16, pr.lanes, s));
+}
+
+msda_status msda_debug_sample_points(const int64_t *spatial_shapes,
+                                     const int64_t *level_start_index,
+                                     const float *sampling_locations, msda_dims d,
+                                     int32_t *valid, int32_t *x0, int32_t *y0, float *x,
+                                     float *y, int64_t *rows, msda_stream_t stream)
+{
+    Problem pr;
+    msda_status st = check_dims(MSDA_F32, spatial_shapes, level_start_index, d, &pr);
+    if (st != MSDA_OK) return st;
+    if (pr.samples > 0 && (!sampling_locations || !valid || !x0 || !y0 || !x || !y || !rows))
+        return MSDA_ERR_NULL;
+    if (!aligned(sampling_locations, 8) || !aligned(valid, 4) || !aligned(x0, 4) ||
+        !aligned(y0, 4) || !aligned(x, 4) || !aligned(y, 4) || !aligned(rows, 8))
+        return MSDA_ERR_ALIGN;
+    const int64_t n = pr.samples;
+    const Span outs[] = {{valid, n * 4}, {x0, n * 4}, {y0, n * 4},
+                         {x, n * 4},     {y, n * 4},  {rows, n * 32}};
+    const Span ins[] = {{sampling_locations, n * 8}};
+    if (any_alias(outs, 6, ins, 1)) return MSDA_ERR_ALIAS;
+    if (n == 0) return MSDA_OK;
+    msda::PointsParams p;
+    memset(&p, 0, sizeof p);
+    p.loc = sampling_locations;
+    p.valid = valid;
+    p.x0 = x0;
+    p.y0 = y0;
+    p.x = x;
+    p.y = y;
+    p.rows = rows;
+    p.samples = n;
+    p.L = (int)d.L;
+    p.K = (int)d.K;
+    p.lv = pr.lv;
+    return cuda_status(msda::launch_sample_points(p, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,234 @@
+// msda_bwd.cu -- backward kernel of the MSDeformAttn core (sm_100a).
+//
+// Gradients flow through the bilinear interpolation to the value map, the
+// sampling locations and the attention weights ("Deformable DETR" wiki
+// page, "Deformable attention module"; "Deformable Attention" glossary
+// page, gradients through the interpolation grid).  Per sample, with
+// g = grad_out[n,q,m,:], corner weights w_j(fx, fy) and t_j = <v_j, g>:
+//   dA        = sum_j w_j t_j
+//   dloc_x    = A * W * sum_j (dw_j/dfx) t_j,  dloc_y = A * H * sum_j (dw_j/dfy) t_j
+//   dvalue_j += A * w_j * g            (scatter; corners inside the level)
+//
+// Work decomposition (one warp per (n, q, m), as in the forward):
+//   1. Lane j < L*K finds sample j's cell and writes, per corner, the row
+//      offset, w_j, dw_j/dfx and dw_j/dfy to shared memory.
+//   2. SPAN = min(32, 4R) lanes work on one sample (R lanes per 16-byte-chunked
+//      row, one corner per R lanes), 32/SPAN samples at a time.  Each lane
+//      gathers its chunk of a corner row, forms its part of t_j, scatters
+//      A w_j g with one vector `red.global.add.v4.f32` per chunk, and keeps
+//      three running partial sums per sample.
+//   3. Every 8 samples per lane group the 24 partial sums are reduced across
+//      the SPAN lanes with a butterfly reduce-scatter (each step halves the
+//      values a lane holds), which costs about 4 shuffles per sample instead
+//      of 15, and the lanes holding finished sums write dA and dloc.
+#include "msda_common.cuh"
+#include "msda_internal.h"
+
+namespace msda {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kBatch = 8;  // samples per lane group between reductions
+constexpr int kNV = 32;    // reduce-scatter width: 3 * kBatch used, padded
+
+struct __align__(16) CornerB {
+    int off;  // element offset of the corner row inside the (n, m) map; -1 = outside
+    float w;    // bilinear weight
+    float dwx;  // d w / d fx
+    float dwy;  // d w / d fy
+};
+
+// Butterfly reduce-scatter over aligned groups of SPAN lanes.  Before: every
+// lane holds N partial values.  After: lane (lane % SPAN) = b holds, in
+// v[0 .. N/SPAN), the group totals of values b*N/SPAN .. (b+1)*N/SPAN - 1.
+template <int SPAN, int N>
+__device__ __forceinline__ void reduce_scatter(float (&v)[kNV], int lane)
+{
+    if constexpr (SPAN > 1) {
+        constexpr int o = SPAN / 2;
+        constexpr int h = N / 2;
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < h; ++i) {
+            const float send = upper ? v[i] : v[i + h];
+            const float keep = upper ? v[i + h] : v[i];
+            v[i] = keep + __shfl_xor_sync(kFull, send, o);
+        }
+        reduce_scatter<o, h>(v, lane);
+    }
+}
+
+template <typename VT, int R>
+__global__ void __launch_bounds__(kWarps * 32)
+    bwd_kernel(const __grid_constant__ BwdParams p)
+{
+    constexpr int kVec = Chunk<VT>::kVec;
+    constexpr int kSpan = (4 * R < 32) ? 4 * R : 32;  // lanes per sample
+    constexpr int kGroups = 32 / kSpan;               // samples in flight per warp
+    constexpr int kCornerSlots = kSpan / R;           // 4, 2 or 1
+    constexpr int kCpl = 4 / kCornerSlots;            // corners per lane
+    constexpr int kPer = kNV / kSpan;                 // finished sums per lane
+
+    __shared__ CornerB corners[kWarps][kMaxLK * 4];
+    __shared__ float sA[kWarps][kMaxLK];
+    __shared__ int sH[kMaxLevels], sW[kMaxLevels], sStart[kMaxLevels];
+
+    const int tid = threadIdx.x;
+    if (tid < p.L) {
+        sH[tid] = p.lv.H[tid];
+        sW[tid] = p.lv.W[tid];
+        sStart[tid] = p.lv.start[tid];
+    }
+    __syncthreads();
+
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int64_t item = (int64_t)blockIdx.x * kWarps + warp;
+    if (item >= p.items) return;
+
+    const int M = p.M, D = p.D, K = p.K;
+    const int LK = p.L * K;
+    const int m = (int)(item % M);
+    const int64_t nq = item / M;
+    const int64_t n = nq / p.Lq;
+    const int64_t sbase = item * LK;
+
+    // ---- phase 1: cell and corner derivatives of sample `lane` -------------
+    if (lane < LK) {
+        const int l = lane / K;
+        const int H = sH[l], W = sW[l], start = sStart[l];
+        const float2 t = __ldg(reinterpret_cast<const float2 *>(p.loc) + sbase + lane);
+        sA[warp][lane] = __ldg(p.attn + sbase + lane);
+        CornerB c[4] = {{-1, 0.f, 0.f, 0.f}, {-1, 0.f, 0.f, 0.f}, {-1, 0.f, 0.f, 0.f},
+                        {-1, 0.f, 0.f, 0.f}};
+        float x, y, fx, fy;
+        int x0, y0;
+        if (msda_cell(t.x, t.y, H, W, x, y, x0, y0, fx, fy)) {
+            const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+            // corner j = (dy, dx) = (j >> 1, j & 1)
+            const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
+            const float dwx[4] = {-hy, hy, -fy, fy};
+            const float dwy[4] = {-hx, -fx, hx, fx};
+            const int MD = M * D;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = msda_row(start, H, W, y0 + (j >> 1), x0 + (j & 1));
+                c[j].off = r < 0 ? -1 : r * MD;
+                c[j].w = w[j];
+                c[j].dwx = dwx[j];
+                c[j].dwy = dwy[j];
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) corners[warp][lane * 4 + j] = c[j];
+    }
+    __syncwarp();
+
+    // ---- phase 2/3 -------------------------------------------------------
+    const int grp = lane / kSpan;
+    const int lin = lane % kSpan;
+    const int cslot = lin / R;
+    const int chunk = lin % R;
+    const bool chunk_ok = chunk < p.nchunks;
+
+    float g[kVec];
+    if (chunk_ok) {
+        const float4 *gp = reinterpret_cast<const float4 *>(
+            p.grad_out + nq * (int64_t)(M * D) + m * D + chunk * kVec);
+#pragma unroll
+        for (int i = 0; i < kVec / 4; ++i) {
+            const float4 t = __ldg(gp + i);
+            g[4 * i] = t.x;
+            g[4 * i + 1] = t.y;
+            g[4 * i + 2] = t.z;
+            g[4 * i + 3] = t.w;
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < kVec; ++i) g[i] = 0.f;
+    }
+    const int64_t rowbase = (n * p.S * M + m) * (int64_t)D + chunk * kVec;
+    const VT *vbase = static_cast<const VT *>(p.value) + rowbase;
+    float *gvbase = p.grad_value + rowbase;
+
+    const int per_batch = kBatch * kGroups;
+    for (int b0 = 0; b0 < LK; b0 += per_batch) {
+        float v[kNV];
+#pragma unroll
+        for (int i = 0; i < kNV; ++i) v[i] = 0.f;
+#pragma unroll
+        for (int it = 0; it < kBatch; ++it) {
+            const int s = b0 + it * kGroups + grp;
+            if (s < LK) {
+                const float a = sA[warp][s];
+#pragma unroll
+                for (int ci = 0; ci < kCpl; ++ci) {
+                    const CornerB e = corners[warp][s * 4 + cslot * kCpl + ci];
+                    float t = 0.f;
+                    if (e.off >= 0 && chunk_ok) {
+                        float x[kVec];
+                        Chunk<VT>::load(vbase + e.off, x);
+#pragma unroll
+                        for (int i = 0; i < kVec; ++i) t = fmaf(x[i], g[i], t);
+                        const float aw = a * e.w;
+                        float *dst = gvbase + e.off;
+#pragma unroll
+                        for (int i = 0; i < kVec; i += 4)
+                            red_add_v4(dst + i, aw * g[i], aw * g[i + 1], aw * g[i + 2],
+                                       aw * g[i + 3]);
+                    }
+                    v[it] = fmaf(e.w, t, v[it]);
+                    v[kBatch + it] = fmaf(e.dwx, t, v[kBatch + it]);
+                    v[2 * kBatch + it] = fmaf(e.dwy, t, v[2 * kBatch + it]);
+                }
+            }
+        }
+        reduce_scatter<kSpan, kNV>(v, lane);
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int idx = lin * kPer + i;
+            const int qty = idx / kBatch;
+            const int it = idx % kBatch;
+            const int s = b0 + it * kGroups + grp;
+            if (qty < 3 && s < LK) {
+                const int64_t si = sbase + s;
+                if (qty == 0) {
+                    if (p.grad_attn) p.grad_attn[si] = v[i];
+                } else if (p.grad_loc) {
+                    const int l = s / K;
+                    const float scale = (qty == 1) ? (float)sW[l] : (float)sH[l];
+                    p.grad_loc[2 * si + (qty - 1)] = sA[warp][s] * (scale * v[i]);
+                }
+            }
+        }
+    }
+}
+
+template <typename VT>
+cudaError_t launch_bwd_vt(const BwdParams &p, int R, cudaStream_t stream)
+{
+    const dim3 block(kWarps * 32);
+    const dim3 grid((unsigned)((p.items + kWarps - 1) / kWarps));
+    switch (R) {
+    case 1: bwd_kernel<VT, 1><<<grid, block, 0, stream>>>(p); break;
+    case 2: bwd_kernel<VT, 2><<<grid, block, 0, stream>>>(p); break;
+    case 4: bwd_kernel<VT, 4><<<grid, block, 0, stream>>>(p); break;
+    case 8: bwd_kernel<VT, 8><<<grid, block, 0, stream>>>(p); break;
+    case 16: bwd_kernel<VT, 16><<<grid, block, 0, stream>>>(p); break;
+    case 32: bwd_kernel<VT, 32><<<grid, block, 0, stream>>>(p); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_backward(const BwdParams &p, bool bf16, int lanes_per_row,
+                            cudaStream_t stream)
+{
+    if (p.items == 0) return cudaSuccess;
+    return bf16 ? launch_bwd_vt<__nv_bfloat16>(p, lanes_per_row, stream)
+                : launch_bwd_vt<float>(p, lanes_per_row, stream);
+}
+
+}  // namespace msda

@@ -1,0 +1,106 @@
+// msda_common.cuh -- device helpers shared by the MSDeformAttn kernels.
+//
+// Every kernel (forward, fused forward, backward, index record) derives a
+// sample's cell from its normalised location through msda_cell(), so the
+// integer cell, the corner rows and the fractions are computed by one piece
+// of code everywhere.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "msda_types.h"
+
+namespace msda {
+
+constexpr unsigned kFull = 0xffffffffu;
+
+// Pixel coordinate and cell of one sample on a level of size H x W
+// ("Deformable DETR" wiki page, "Multi-scale deformable attention": phi_l
+// rescales the normalised point by the level's size).  Pixel centres sit at
+// half-integers: x = loc_x * W - 0.5, each step one IEEE fp32 operation with
+// no contraction into an FMA.  Returns false when no corner of the cell can
+// lie inside the level (x outside (-1, W) or y outside (-1, H)); NaN and Inf
+// fail this test too.
+__device__ __forceinline__ bool msda_cell(float lx, float ly, int H, int W, float &x,
+                                          float &y, int &x0, int &y0, float &fx,
+                                          float &fy)
+{
+    x = __fadd_rn(__fmul_rn(lx, (float)W), -0.5f);
+    y = __fadd_rn(__fmul_rn(ly, (float)H), -0.5f);
+    if (!(x > -1.0f && x < (float)W && y > -1.0f && y < (float)H)) return false;
+    const float xf = floorf(x);
+    const float yf = floorf(y);
+    x0 = (int)xf;
+    y0 = (int)yf;
+    fx = __fsub_rn(x, xf);
+    fy = __fsub_rn(y, yf);
+    return true;
+}
+
+// Value row of pixel (yy, xx) on a level, or -1 outside the level (zero
+// padding: such a corner contributes nothing).
+__device__ __forceinline__ int msda_row(int start, int H, int W, int yy, int xx)
+{
+    return (xx >= 0 && xx < W && yy >= 0 && yy < H) ? start + yy * W + xx : -1;
+}
+
+// ---------------------------------------------------------------------------
+// Loads of one 16-byte chunk of a value row, widened to fp32.
+// ---------------------------------------------------------------------------
+template <typename VT>
+struct Chunk;
+
+template <>
+struct Chunk<float> {
+    static constexpr int kVec = 4;
+    __device__ __forceinline__ static void load(const float *p, float (&v)[4])
+    {
+        const float4 t = __ldg(reinterpret_cast<const float4 *>(p));
+        v[0] = t.x;
+        v[1] = t.y;
+        v[2] = t.z;
+        v[3] = t.w;
+    }
+};
+
+template <>
+struct Chunk<__nv_bfloat16> {
+    static constexpr int kVec = 8;
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float (&v)[8])
+    {
+        const uint4 t = __ldg(reinterpret_cast<const uint4 *>(p));
+        const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            // bf16 -> fp32 widening is exact: the bf16 bits become the high half.
+            v[2 * i] = __uint_as_float(w[i] << 16);
+            v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+
+// Vector atomic add of four fp32 values (sm_90+ `red.global.add.v4.f32`).
+__device__ __forceinline__ void red_add_v4(float *addr, float a, float b, float c, float d)
+{
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a),
+                 "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ float warp_max(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
+}  // namespace msda

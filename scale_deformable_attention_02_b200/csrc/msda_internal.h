@@ -1,0 +1,65 @@
+// msda_internal.h -- launch parameters shared by the host entry points and
+// the kernels.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "msda_types.h"
+
+namespace msda {
+
+// Everything a forward launch needs.  Checked on the host before launch:
+// S*M*D < 2^31 (row offsets are int32), L*K <= 32, rows of 16..512 bytes.
+struct FwdParams {
+    const void *value;
+    // unfused inputs
+    const float *loc;   // [N,Lq,M,L,K,2]
+    const float *attn;  // [N,Lq,M,L,K]
+    // fused inputs
+    const float *ref;     // [N,Lq,ref_dim]
+    const float *off;     // [N,Lq,M,L,K,2]
+    const float *logits;  // [N,Lq,M,L,K]
+    int ref_dim;
+    // outputs
+    float *out;       // [N,Lq,M*D]
+    float *loc_out;   // nullable (fused)
+    float *attn_out;  // nullable (fused)
+    int64_t items;    // N*Lq*M (one warp each)
+    int Lq, S, M, D, L, K;
+    int nchunks;  // 16-byte chunks per value row
+    Levels lv;
+};
+
+struct BwdParams {
+    const void *value;
+    const float *loc;
+    const float *attn;
+    const float *grad_out;
+    float *grad_value;
+    float *grad_loc;   // nullable
+    float *grad_attn;  // nullable
+    int64_t items;
+    int Lq, S, M, D, L, K;
+    int nchunks;
+    Levels lv;
+};
+
+struct PointsParams {
+    const float *loc;
+    int32_t *valid, *x0, *y0;
+    float *x, *y;
+    int64_t *rows;
+    int64_t samples;  // N*Lq*M*L*K
+    int L, K;
+    Levels lv;
+};
+
+// Launchers (return the launch's cudaError_t).
+cudaError_t launch_forward(const FwdParams &p, bool bf16, bool fused, int lanes_per_row,
+                           cudaStream_t stream);
+cudaError_t launch_backward(const BwdParams &p, bool bf16, int lanes_per_row,
+                            cudaStream_t stream);
+cudaError_t launch_sample_points(const PointsParams &p, cudaStream_t stream);
+
+}  // namespace msda

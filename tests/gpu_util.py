@@ -1,0 +1,58 @@
+"""Helpers shared by the GPU parity tests: device transfer and the
+elementwise tolerance check |gpu - oracle| <= atol + rtol * |oracle|."""
+import numpy as np
+import torch
+
+# Tolerances: fp32 outputs and weights (1e-5 relative, 1e-6 absolute);
+# gradients accumulated with atomics or reduced across lanes (1e-4 relative,
+# 1e-5 absolute); bf16 value against the fp32-value oracle (2e-2 relative).
+F32 = dict(rtol=1e-5, atol=1e-6)
+GRAD = dict(rtol=1e-4, atol=1e-5)
+
+
+def dev():
+    return torch.device("cuda:0")
+
+
+def to_dev(a: np.ndarray) -> torch.Tensor:
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:  # bf16 bit patterns
+        return torch.from_numpy(a.view(np.int16)).to(dev()).view(torch.bfloat16)
+    return torch.from_numpy(a).to(dev())
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu").numpy()
+
+
+def assert_close(gpu, ora, rtol, atol, what=""):
+    g = np.asarray(gpu, dtype=np.float64)
+    o = np.asarray(ora, dtype=np.float64)
+    assert g.shape == o.shape, (what, g.shape, o.shape)
+    fin = np.isfinite(o)
+    assert np.array_equal(np.isfinite(g), fin), f"{what}: non-finite entries differ"
+    g = np.where(fin, g, 0.0)
+    o = np.where(fin, o, 0.0)
+    err = np.abs(g - o)
+    bound = atol + rtol * np.abs(o)
+    bad = err > bound
+    if bad.any():
+        i = np.unravel_index(np.argmax(err - bound), err.shape)
+        raise AssertionError(
+            f"{what}: {int(bad.sum())} of {bad.size} elements outside "
+            f"atol={atol} rtol={rtol}; worst at {i}: gpu={g[i]!r} oracle={o[i]!r} "
+            f"err={err[i]:.3e} bound={bound[i]:.3e}")
+
+
+def assert_bits_equal(gpu, ora, what=""):
+    g = np.asarray(gpu)
+    o = np.asarray(ora)
+    assert g.shape == o.shape, (what, g.shape, o.shape)
+    if g.dtype == np.float32:
+        g = g.view(np.uint32)
+        o = np.asarray(o, dtype=np.float32).view(np.uint32)
+    mism = g != o
+    if mism.any():
+        i = np.argwhere(mism)[0]
+        raise AssertionError(f"{what}: {int(mism.sum())} mismatches; first at {tuple(i)}: "
+                             f"gpu={g[tuple(i)]} oracle={o[tuple(i)]}")

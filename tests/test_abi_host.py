@@ -1,0 +1,212 @@
+"""The C ABI on the host: the library loads, exports every symbol the headers
+declare, computes the level metadata, and rejects bad arguments with the
+documented status codes before any device work.  CPU only: every call here
+returns before touching CUDA (pointers are fake and never dereferenced)."""
+import ctypes
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from scale_deformable_attention_02_b200 import _lib
+from scale_deformable_attention_02_b200 import build as msda_build
+from scale_deformable_attention_02_b200 import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+OK, NULL, SHAPE, LEVELS, DTYPE, ALIGN, ALIAS, UNSUP = range(8)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    msda_build.build()
+    return _lib.load()
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names += re.findall(r"^MSDA_API\s+[\w\s\*]*?\b(msda_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_headers_declare_the_entry_points():
+    names = declared_functions()
+    for must in ("msda_forward", "msda_forward_fused", "msda_backward",
+                 "msda_level_start_index", "msda_status_string", "msda_debug_sample_points"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert name in _lib.SIGNATURES, f"binding lacks {name}"
+
+
+def test_library_exports_nothing_else():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = sorted({ln.split()[-1] for ln in out.splitlines() if " T " in ln})
+    assert exported == declared_functions()
+
+
+def test_status_strings_and_version(lib):
+    for code, name in _lib.STATUS_NAMES.items():
+        assert lib.msda_status_string(code).decode().startswith(name)
+    assert lib.msda_abi_version() == 10000
+
+
+@pytest.mark.parametrize("shapes", [wl.TINY_SHAPES, wl.ENCODER_SHAPES, wl.STRESS_SHAPES,
+                                    ((0, 5), (3, 0), (1, 1)), ((7, 3),)])
+def test_level_start_index_bit_exact_with_oracle(lib, shapes):
+    from scale_deformable_attention_02_b200 import msda_level_start_index
+    s = wl.spatial_shapes_array(shapes)
+    starts, S = msda_level_start_index(s)
+    ostarts, oS = oracle.level_start_index(s)
+    assert starts.tolist() == ostarts.tolist() and S == oS
+
+
+def test_level_start_index_errors(lib):
+    s = np.array([[3, -1]], dtype=np.int64)
+    out = np.zeros(1, dtype=np.int64)
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)  # noqa: E731
+    assert lib.msda_level_start_index(p(s), 1, p(out), None) == SHAPE
+    assert lib.msda_level_start_index(None, 1, p(out), None) == NULL
+    assert lib.msda_level_start_index(p(s), 0, p(out), None) == SHAPE
+
+
+# ---------------------------------------------------------------------------
+# Argument checks of the compute entry points (fake device pointers).
+# ---------------------------------------------------------------------------
+BASE = 1 << 32  # fake, 256-byte aligned device addresses, far apart
+GAP = 1 << 28
+
+
+def fake(i, off=0):
+    return ctypes.c_void_p(BASE + i * GAP + off)
+
+
+class Prob:
+    def __init__(self, N=2, Lq=5, M=2, D=8, K=2, shapes=((4, 6), (2, 3)), dtype=0):
+        self.shapes = np.array(shapes, dtype=np.int64).reshape(-1, 2)
+        self.starts, S = oracle.level_start_index(self.shapes)
+        self.dims = _lib.Dims(N, Lq, S, M, D, len(shapes), K)
+        self.dtype = dtype
+
+    def sp(self):
+        return self.shapes.ctypes.data_as(ctypes.c_void_p)
+
+    def st(self):
+        return self.starts.ctypes.data_as(ctypes.c_void_p)
+
+
+def fwd(lib, pr, value=None, loc=None, attn=None, out=None, dims=None, dtype=None,
+        shapes=None, starts=None):
+    return lib.msda_forward(value or fake(0), pr.dtype if dtype is None else dtype,
+                            shapes or pr.sp(), starts or pr.st(), loc or fake(1),
+                            attn or fake(2), out or fake(3), dims or pr.dims, None)
+
+
+def test_forward_argument_errors(lib):
+    pr = Prob()
+    assert fwd(lib, pr, dtype=7) == DTYPE
+    bad = Prob()
+    bad.dims.M = 0
+    assert fwd(lib, bad) == SHAPE
+    bad = Prob()
+    bad.dims.N = -1
+    assert fwd(lib, bad) == SHAPE
+    # L*K beyond one lane per sample
+    big = Prob(K=17)
+    assert fwd(lib, big) == UNSUP
+    # level metadata that disagrees with S or with the prefix sum
+    bad = Prob()
+    bad.dims.S += 1
+    assert fwd(lib, bad) == LEVELS
+    bad = Prob()
+    bad.starts[1] += 1
+    assert fwd(lib, bad) == LEVELS
+    bad = Prob(shapes=((4, -6), (2, 3)))
+    assert fwd(lib, bad) == SHAPE
+    # row sizes: fp32 D = 3 (12 B), bf16 D = 4 (8 B) are not 16-byte multiples
+    assert fwd(lib, Prob(D=3)) == ALIGN
+    assert fwd(lib, Prob(D=4, dtype=1)) == ALIGN
+    assert fwd(lib, Prob(D=256)) == UNSUP  # 1 KB rows
+    # pointers
+    assert lib.msda_forward(fake(0), 0, None, pr.st(), fake(1), fake(2), fake(3), pr.dims,
+                            None) == NULL
+    assert fwd(lib, pr, value=fake(0, 8)) == ALIGN
+    assert fwd(lib, pr, out=fake(3, 4)) == ALIGN
+    assert fwd(lib, pr, loc=fake(1, 4)) == ALIGN
+    assert fwd(lib, pr, attn=fake(2, 2)) == ALIGN
+    assert lib.msda_forward(fake(0), 0, pr.sp(), pr.st(), None, fake(2), fake(3), pr.dims,
+                            None) == NULL
+    # out overlapping an input
+    assert fwd(lib, pr, out=fake(1)) == ALIAS
+    assert fwd(lib, pr, out=fake(0, 64)) == ALIAS
+    # int32 row offsets: S*M*D must stay below 2^31
+    huge = Prob(M=8, D=32, shapes=((4096, 2049),))
+    assert fwd(lib, huge) == UNSUP
+
+
+def test_empty_problems_are_no_ops(lib):
+    """N = 0 or Lq = 0: nothing to compute, null tensors allowed, no launch."""
+    for N, Lq in ((0, 5), (2, 0)):
+        pr = Prob(N=N, Lq=Lq)
+        assert lib.msda_forward(None, 0, pr.sp(), pr.st(), None, None, None, pr.dims,
+                                None) == OK
+        assert lib.msda_forward_fused(None, 0, pr.sp(), pr.st(), None, 2, None, None, None,
+                                      None, None, pr.dims, None) == OK
+    pr = Prob(N=0)
+    assert lib.msda_backward(None, 0, pr.sp(), pr.st(), None, None, None, None, None, None,
+                             pr.dims, None) == OK
+
+
+def test_fused_argument_errors(lib):
+    pr = Prob()
+
+    def call(ref=None, rdim=2, off=None, logits=None, out=None, loc_out=None, attn_out=None):
+        return lib.msda_forward_fused(fake(0), 0, pr.sp(), pr.st(), ref or fake(1), rdim,
+                                      off or fake(2), logits or fake(4), out or fake(3),
+                                      loc_out, attn_out, pr.dims, None)
+
+    assert call(rdim=3) == SHAPE
+    assert call(ref=fake(1, 4)) == ALIGN
+    assert call(off=fake(2, 4)) == ALIGN
+    assert call(loc_out=fake(5, 4)) == ALIGN
+    assert call(loc_out=fake(2)) == ALIAS          # writes over the offsets
+    assert call(attn_out=fake(3, 16)) == ALIAS     # overlaps out
+    assert call(out=fake(5), loc_out=fake(5, 32)) == ALIAS
+    assert lib.msda_forward_fused(fake(0), 0, pr.sp(), pr.st(), None, 2, fake(2), fake(4),
+                                  fake(3), None, None, pr.dims, None) == NULL
+
+
+def test_backward_argument_errors(lib):
+    pr = Prob()
+
+    def call(gv=None, gl=None, ga=None, g=None, loc=None):
+        return lib.msda_backward(fake(0), 0, pr.sp(), pr.st(), loc or fake(1), fake(2),
+                                 g or fake(3), gv or fake(4), gl, ga, pr.dims, None)
+
+    assert call(gv=fake(4, 8)) == ALIGN
+    assert call(gl=fake(5, 4)) == ALIGN
+    assert call(gv=fake(3)) == ALIAS          # grad_value over grad_out
+    assert call(gl=fake(4, 64)) == ALIAS      # grad_loc inside grad_value
+    assert call(ga=fake(1)) == ALIAS          # grad_attn over the locations
+    assert lib.msda_backward(fake(0), 0, pr.sp(), pr.st(), fake(1), fake(2), fake(3), None,
+                             None, None, pr.dims, None) == NULL
+
+
+def test_binding_rejects_mismatched_tensors():
+    torch = pytest.importorskip("torch")
+    from scale_deformable_attention_02_b200 import msda_forward
+    value = torch.zeros(1, 80, 2, 8)
+    loc = torch.zeros(1, 4, 2, 2, 2, 2)
+    attn = torch.zeros(1, 4, 2, 2, 3)  # K mismatch
+    with pytest.raises(ValueError):
+        msda_forward(value, wl.TINY_SHAPES, None, loc, attn)

@@ -296,6 +296,33 @@ def test_locations_zero_offset_and_exact_steps():
         np.testing.assert_allclose(px, off64[..., l, :, 0], rtol=0, atol=1e-11)
 
 
+def test_box_locations():
+    """Box references: zero offset gives the box centre bit for bit, and an
+    offset of +-1/2 box unit lands on the box edges (dyadic boxes keep every
+    step exact) -- the iterative-refinement reading that offsets are scaled
+    by the previous box's width and height ("Deformable DETR" wiki page,
+    "Variants")."""
+    N, Lq, M, L, K = 2, 5, 3, 2, 4
+    cx = RNG.integers(8, 56, size=(N, Lq)) / 64.0
+    cy = RNG.integers(8, 56, size=(N, Lq)) / 64.0
+    w = RNG.integers(1, 8, size=(N, Lq)) / 32.0
+    h = RNG.integers(1, 8, size=(N, Lq)) / 32.0
+    box = np.stack([cx, cy, w, h], axis=-1).astype(np.float32)
+    off = np.zeros((N, Lq, M, L, K, 2), np.float32)
+    loc = oracle.locations_box_f32(box, off)
+    np.testing.assert_array_equal(loc, np.broadcast_to(box[:, :, None, None, None, :2], loc.shape))
+    off[..., 0] = 0.5
+    off[..., 1] = -0.5
+    loc = oracle.locations_box_f32(box, off)
+    np.testing.assert_array_equal(loc[..., 0], np.broadcast_to((cx + w / 2)[:, :, None, None, None], loc.shape[:-1]))
+    np.testing.assert_array_equal(loc[..., 1], np.broadcast_to((cy - h / 2)[:, :, None, None, None], loc.shape[:-1]))
+    # general offsets: within fp32 rounding of the exact map
+    off = RNG.standard_normal(off.shape).astype(np.float32)
+    loc = oracle.locations_box_f32(box, off)
+    exact = box[:, :, None, None, None, :2].astype(np.float64) + off * box[:, :, None, None, None, 2:].astype(np.float64)
+    np.testing.assert_allclose(loc, exact, rtol=0, atol=2e-7)
+
+
 # --------------------------------------------------------------------------
 # Independent brute-force formulation: tent kernels over every pixel
 # --------------------------------------------------------------------------
