@@ -74,8 +74,19 @@ def dist_env():
 
 
 def rank_workload(name: str, rank: int) -> wl.Workload:
+    """Rank r's own batch: the same shapes, its own seed (weak scaling)."""
     w = wl.WORKLOADS[name]
     return dataclasses.replace(w, seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(vals, world: int, device):
+    """Element-wise max of per-rank timings (every rank gets the result)."""
+    import torch
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=device)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
 
 
 # ---------------------------------------------------------------------------
@@ -281,11 +292,9 @@ def run_ours(args):
     fwd_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
     bwd_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
     step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
-    t = torch.tensor([statistics.fmean(step_ms), statistics.fmean(fwd_ms),
-                      statistics.fmean(bwd_ms)], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_step, ms_fwd, ms_bwd = (float(x) for x in t.tolist())
+    ms_step, ms_fwd, ms_bwd = max_over_ranks(
+        [statistics.fmean(step_ms), statistics.fmean(fwd_ms), statistics.fmean(bwd_ms)],
+        world, device)
     queries = w.N * w.queries
     value_qps = queries * world / (ms_step / 1e3)
 
@@ -429,10 +438,7 @@ def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    t = torch.tensor([e0.elapsed_time(e1) / n], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms = float(t.item())
+    ms = max_over_ranks([e0.elapsed_time(e1) / n], world, device)[0]
     h2d = sum(h_in[k].numel() * h_in[k].element_size() for k in names)
     d2h = sum(h_out[k].numel() * h_out[k].element_size() for k in res_shapes)
     return {"value": queries * world / (ms / 1e3), "unit": "queries/s", "ms_per_step": ms,

@@ -72,7 +72,7 @@ def lib():
             _lib.ora_locations_f64.restype = None
             _lib.ora_locations_f64.argtypes = [P, P, P, Dims, P]
             _lib.ora_backward.restype = None
-            _lib.ora_backward.argtypes = [P, I, P, P, P, I, P, P, P, P, P, Dims]
+            _lib.ora_backward.argtypes = [P, I, P, P, P, I, P, P, P, P, P, P, P, Dims]
             _lib.ora_fused_chain.restype = None
             _lib.ora_fused_chain.argtypes = [P, P, P, P, Dims, P, P, P]
             _lib.ora_sample_points_f32.restype = None
@@ -185,9 +185,10 @@ def forward_fused(value, shapes, ref, off, logits):
     return forward(value, shapes, loc, a, loc_f32=True), loc, a
 
 
-def backward(value, shapes, loc, attn, grad_out, loc_f32: bool = True):
+def backward(value, shapes, loc, attn, grad_out, loc_f32: bool = True, with_mass=False):
     """Returns (grad_value [N,S,M,D], grad_loc like loc, grad_attn like attn),
-    all float64."""
+    all float64; with_mass=True appends (grad_loc_mass, grad_attn_mass), the
+    sums of absolute terms that scale a finite-precision rounding bound."""
     v, bf = _value_arg(value)
     shapes = np.ascontiguousarray(shapes, dtype=np.int64)
     starts, S = level_start_index(shapes)
@@ -199,9 +200,14 @@ def backward(value, shapes, loc, attn, grad_out, loc_f32: bool = True):
     gv = np.empty(v.shape, dtype=np.float64)
     gl = np.empty(loc64.shape, dtype=np.float64)
     ga = np.empty(a64.shape, dtype=np.float64)
+    glm = np.empty(loc64.shape, dtype=np.float64) if with_mass else None
+    gam = np.empty(a64.shape, dtype=np.float64) if with_mass else None
     lib().ora_backward(_ptr(v), bf, _ptr(shapes), _ptr(starts), _ptr(loc64),
                        1 if loc_f32 else 0, _ptr(a64), _ptr(g64), _ptr(gv),
-                       _ptr(gl), _ptr(ga), d)
+                       _ptr(gl), _ptr(ga), None if glm is None else _ptr(glm),
+                       None if gam is None else _ptr(gam), d)
+    if with_mass:
+        return gv, gl, ga, glm, gam
     return gv, gl, ga
 
 

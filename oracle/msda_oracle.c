@@ -324,11 +324,18 @@ void ora_locations_f64(const double *ref, const double *off, const int64_t *shap
  * (dx/dloc_x = W by R1; dfx/dx = 1 by R6; outside corners have v_j = 0.)
  * grad_value [N,S,M,D] is overwritten.  Serial per (n, m): rows of different
  * (n, m) are disjoint, so the result is deterministic.
+ *
+ * grad_loc_mass / grad_attn_mass (may be NULL) receive the absolute mass of
+ * each sum, the same expression with every term replaced by its absolute
+ * value (e.g. A*W*sum_j |dw_j/dfx| sum_c |v_jc g_c|).  They are not part of
+ * the method: they scale the rounding-error bound of a finite-precision
+ * evaluation of the same sum, |fl(sum) - sum| <= n*u*mass.
  */
 void ora_backward(const void *value, int value_bf16, const int64_t *shapes,
                   const int64_t *starts, const double *loc, int loc_f32,
                   const double *attn, const double *grad_out, double *grad_value,
-                  double *grad_loc, double *grad_attn, ora_dims d)
+                  double *grad_loc, double *grad_attn, double *grad_loc_mass,
+                  double *grad_attn_mass, ora_dims d)
 {
     const int64_t N = d.N, Lq = d.Lq, S = d.S, M = d.M, D = d.D, L = d.L, K = d.K;
     memset(grad_value, 0, sizeof(double) * (size_t)(N * S * M * D));
@@ -346,10 +353,17 @@ void ora_backward(const void *value, int value_bf16, const int64_t *shapes,
                         grad_attn[i] = 0.0;
                         grad_loc[2 * i] = 0.0;
                         grad_loc[2 * i + 1] = 0.0;
+                        if (grad_loc_mass) {
+                            grad_loc_mass[2 * i] = 0.0;
+                            grad_loc_mass[2 * i + 1] = 0.0;
+                        }
+                        if (grad_attn_mass)
+                            grad_attn_mass[i] = 0.0;
                         continue;
                     }
                     const double a = attn[i];
                     double dA = 0.0, dfx = 0.0, dfy = 0.0;
+                    double mA = 0.0, mfx = 0.0, mfy = 0.0;
                     for (int cy = 0; cy < 2; ++cy)
                         for (int cx = 0; cx < 2; ++cx) {
                             const double wx = cx ? p.fx : 1.0 - p.fx;
@@ -360,19 +374,29 @@ void ora_backward(const void *value, int value_bf16, const int64_t *shapes,
                             const int64_t r = pixel_row(shapes, starts, l, p.y0 + cy, p.x0 + cx);
                             if (r < 0)
                                 continue; /* v = 0: no term, no scatter */
-                            double vg = 0.0;
+                            double vg = 0.0, vg_abs = 0.0;
                             for (int64_t c = 0; c < D; ++c) {
                                 const int64_t e = ((n * S + r) * M + m) * D + c;
                                 vg += value_at(value, value_bf16, e) * g[c];
+                                vg_abs += fabs(value_at(value, value_bf16, e) * g[c]);
                                 grad_value[e] += a * w * g[c];
                             }
                             dA += w * vg;
                             dfx += sx * wy * vg;
                             dfy += sy * wx * vg;
+                            mA += w * vg_abs;
+                            mfx += wy * vg_abs;
+                            mfy += wx * vg_abs;
                         }
                     grad_attn[i] = dA;
                     grad_loc[2 * i] = a * (double)W * dfx;
                     grad_loc[2 * i + 1] = a * (double)H * dfy;
+                    if (grad_loc_mass) {
+                        grad_loc_mass[2 * i] = fabs(a) * (double)W * mfx;
+                        grad_loc_mass[2 * i + 1] = fabs(a) * (double)H * mfy;
+                    }
+                    if (grad_attn_mass)
+                        grad_attn_mass[i] = mA;
                 }
             }
         }

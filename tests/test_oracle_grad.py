@@ -153,3 +153,18 @@ def test_finite_differences_fused_chain():
             m[ii] -= h
             fd = (F(p, off, z) - F(m, off, z)) / (2 * h)
             assert abs(fd - g_ref[ii]) <= 1e-6 * (1 + abs(fd))
+
+
+def test_backward_mass_bounds_the_sums():
+    """The absolute masses bound the gradients (|sum| <= sum of |terms|) and
+    equal them when every term has the same sign (non-negative value and
+    upstream gradient make every <v_j, g> >= 0, so grad_attn = its mass)."""
+    d = wl.make_random_problem(21, N=1, Lq=7, M=2, D=4, K=3, shapes=((5, 6), (3, 3)))
+    sh, loc = d["spatial_shapes"], d["sampling_locations"]
+    A = oracle.softmax(d["logits"])
+    _, gl, ga, mgl, mga = oracle.backward(d["value"], sh, loc, A, d["grad_out"], with_mass=True)
+    assert np.all(np.abs(gl) <= mgl * (1 + 1e-12)) and np.all(np.abs(ga) <= mga * (1 + 1e-12))
+    v = np.abs(d["value"])
+    g = np.abs(d["grad_out"])
+    _, _, ga2, _, mga2 = oracle.backward(v, sh, loc, A, g, with_mass=True)
+    np.testing.assert_allclose(ga2, mga2, rtol=1e-13, atol=0)
