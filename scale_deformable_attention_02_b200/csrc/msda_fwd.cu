@@ -4,43 +4,95 @@
 // page, "Multi-scale deformable attention" equation):
 //   out[n,q,m,:] = sum_{l,k} A[n,q,m,l,k] * bilinear(value[n, level l, m, :], loc)
 //
-// Work decomposition (one warp per (n, q, m)):
-//   1. Lane j < L*K owns sample j.  It reads the sample's location and weight
-//      (fused: forms them from the reference point, the pixel offset and the
-//      logit; the softmax runs across the lanes with shuffles), finds the cell
-//      and writes four (row offset, weight) corner entries to shared memory.
-//      The attention weight is folded into the corner weights.
-//   2. The warp walks the 4*L*K (sample, corner) pairs.  A value row of one
-//      head (D elements) is split into 16-byte chunks: R lanes cover a row and
-//      32/R rows are gathered per warp instruction, so every corner read is a
-//      coalesced 16-byte-per-lane load of a whole row (fp32 D = 32: 8 lanes x
-//      16 B, four corners per instruction; bf16 D = 32: 4 lanes, two samples
-//      per instruction).  Each lane accumulates its chunk in fp32 registers.
-//   3. The 32/R partial sums of a chunk are combined with xor shuffles and
-//      lanes 0..R-1 store the head's D outputs.
-// The gather is the whole cost ("Deformable DETR" wiki page, "Limitations":
-// deformable sampling means unordered memory access); there is no dense
-// contraction, so no tensor-core path.
+// Work decomposition.  An "item" is one (n, q, m); it has L*K samples.  A warp
+// owns 32/P consecutive items, where P = max(4, next power of two >= L*K) is
+// the number of lanes given to one item in phase 1.
+//   1. Every lane owns one sample (lane j of an item's P-lane segment owns
+//      sample j).  It reads the sample's location and weight -- or, fused,
+//      forms them: the joint softmax over the item's L*K logits runs inside
+//      the P-lane segment with xor shuffles, and the location map is an IEEE
+//      divide and add -- finds the cell and writes four corner entries
+//      (row offset, attention weight x bilinear weight) to shared memory.
+//   2. The warp walks the 4*L*K (sample, corner) pairs of its items together.
+//      A (pixel, head) row of D elements is split into 16-byte chunks; R lanes
+//      cover one row and 32/R rows are gathered per warp instruction, so every
+//      corner read is a coalesced 16-byte-per-lane load of whole rows (fp32,
+//      D = 32: 8 lanes x 16 B, the four corners of a sample in one
+//      instruction; bf16, D = 32: 4 lanes, two samples per instruction).
+//      Lanes accumulate their chunk in fp32 with packed FMA (`__ffma2_rn`).
+//   3. Xor shuffles combine the 32/R partial sums of a chunk, and lanes
+//      0..R-1 store each item's D outputs.
+// Single-use data (locations, weights, logits, offsets, outputs) is read and
+// written with evict-first hints so that the value map, which every sample
+// gathers from, keeps the L2.  The gather is the whole cost ("Deformable
+// DETR" wiki page, "Limitations": deformable sampling means unordered memory
+// access); there is no dense contraction, so no tensor-core path.
 #include "msda_common.cuh"
 #include "msda_internal.h"
 
 namespace msda {
 namespace {
 
-constexpr int kWarps = 8;  // warps (items) per CTA
+constexpr int kWarps = 8;  // warps per CTA
 
-struct __align__(8) Corner {
-    int off;  // element offset of the corner row inside the (n, m) map; -1 = outside
-    float w;  // bilinear weight times the attention weight
+struct __align__(16) Corner {
+    int off;    // element offset of the corner row inside the (n, m) map; -1 = outside
+    int pad;
+    float2 w;   // (w, w): bilinear weight times the attention weight, twice
 };
 
-template <typename VT, int R, bool kFused>
+template <int P>
+__device__ __forceinline__ float seg_max(float v)
+{
+#pragma unroll
+    for (int o = P / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+    return v;
+}
+
+template <int P>
+__device__ __forceinline__ float seg_sum(float v)
+{
+#pragma unroll
+    for (int o = P / 2; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
+// One 16-byte chunk of a value row as kVec/2 float pairs.
+template <typename VT>
+struct Pairs;
+
+template <>
+struct Pairs<float> {
+    static constexpr int kN = 2;
+    __device__ __forceinline__ static void load(const float *p, float2 (&v)[2])
+    {
+        const float4 t = __ldg(reinterpret_cast<const float4 *>(p));
+        v[0] = make_float2(t.x, t.y);
+        v[1] = make_float2(t.z, t.w);
+    }
+};
+
+template <>
+struct Pairs<__nv_bfloat16> {
+    static constexpr int kN = 4;
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float2 (&v)[4])
+    {
+        const uint4 t = __ldg(reinterpret_cast<const uint4 *>(p));
+        const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)  // exact widening: bf16 bits become the high half
+            v[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+    }
+};
+
+template <typename VT, int R, int P, bool kFused, bool kExact>
 __global__ void __launch_bounds__(kWarps * 32)
     fwd_kernel(const __grid_constant__ FwdParams p)
 {
-    constexpr int kVec = Chunk<VT>::kVec;
-    constexpr int kSlots = 32 / R;  // (sample, corner) pairs per warp instruction
-    __shared__ Corner corners[kWarps][kMaxLK * 4];
+    constexpr int kNP = Pairs<VT>::kN;   // float pairs per 16-byte chunk
+    constexpr int kSlots = 32 / R;       // (sample, corner) pairs per warp instruction
+    constexpr int kItems = 32 / P;       // items per warp
+    __shared__ Corner corners[kWarps][kItems][4 * P];
     __shared__ int sH[kMaxLevels], sW[kMaxLevels], sStart[kMaxLevels];
 
     const int tid = threadIdx.x;
@@ -53,124 +105,168 @@ __global__ void __launch_bounds__(kWarps * 32)
 
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int64_t item = (int64_t)blockIdx.x * kWarps + warp;
-    if (item >= p.items) return;  // whole warp leaves together
+    const int64_t item0 = ((int64_t)blockIdx.x * kWarps + warp) * kItems;
+    if (item0 >= p.items) return;  // whole warp leaves together
 
     const int M = p.M, D = p.D, K = p.K;
     const int LK = p.L * K;
-    const int m = (int)(item % M);
-    const int64_t nq = item / M;  // n * Lq + q
-    const int64_t n = nq / p.Lq;
-    const int64_t sbase = item * LK;  // first sample of this (n, q, m)
-    const bool act = lane < LK;
-    const int l = act ? lane / K : 0;
+    const int MD = M * D;
 
-    // ---- phase 1: location and weight of sample `lane` --------------------
-    float lx = 0.f, ly = 0.f, a = 0.f;
-    if constexpr (kFused) {
-        // Joint softmax over the L*K logits of this head, max-subtracted.
-        const float z = act ? __ldg(p.logits + sbase + lane) : -INFINITY;
-        const float mx = warp_max(z);
-        const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
-        const float s = warp_sum(e);
-        a = __fdiv_rn(e, s);
-        if (act) {
-            const float2 o = __ldg(reinterpret_cast<const float2 *>(p.off) + sbase + lane);
-            if (p.ref_dim == 2) {
-                // point reference: offsets are level-l pixels -> divide by the level size
-                const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
-                lx = __fadd_rn(r.x, __fdiv_rn(o.x, (float)sW[l]));
-                ly = __fadd_rn(r.y, __fdiv_rn(o.y, (float)sH[l]));
-            } else {
-                // box reference (cx, cy, w, h): offsets are in box units
-                const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
-                const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
-                lx = __fadd_rn(c.x, __fmul_rn(o.x, s2.x));
-                ly = __fadd_rn(c.y, __fmul_rn(o.y, s2.y));
+    // ---- phase 1: one sample per lane -------------------------------------
+    {
+        const int seg = lane / P;  // item within the warp
+        const int j = lane % P;    // sample within the item
+        const int64_t item = item0 + seg;
+        const bool act = j < LK && item < p.items;
+        const int64_t si = item * LK + j;
+        const int l = act ? j / K : 0;
+        float lx = 0.f, ly = 0.f, a = 0.f;
+        if constexpr (kFused) {
+            const float z = act ? __ldcs(p.logits + si) : -INFINITY;
+            const float mx = seg_max<P>(z);
+            const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
+            const float s = seg_sum<P>(e);
+            a = __fdiv_rn(e, s);
+            if (act) {
+                const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + si);
+                const int64_t nq = item / M;
+                if (p.ref_dim == 2) {
+                    // point reference: offsets are level-l pixels
+                    const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
+                    lx = __fadd_rn(r.x, __fdiv_rn(o.x, (float)sW[l]));
+                    ly = __fadd_rn(r.y, __fdiv_rn(o.y, (float)sH[l]));
+                } else {
+                    // box reference (cx, cy, w, h): offsets are in box units
+                    const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
+                    const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
+                    lx = __fadd_rn(c.x, __fmul_rn(o.x, s2.x));
+                    ly = __fadd_rn(c.y, __fmul_rn(o.y, s2.y));
+                }
+                if (p.loc_out)
+                    __stcs(reinterpret_cast<float2 *>(p.loc_out) + si, make_float2(lx, ly));
+                if (p.attn_out) __stcs(p.attn_out + si, a);
             }
-            if (p.loc_out)
-                reinterpret_cast<float2 *>(p.loc_out)[sbase + lane] = make_float2(lx, ly);
-            if (p.attn_out) p.attn_out[sbase + lane] = a;
-        }
-    } else {
-        if (act) {
-            const float2 t = __ldg(reinterpret_cast<const float2 *>(p.loc) + sbase + lane);
+        } else if (act) {
+            const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
             lx = t.x;
             ly = t.y;
-            a = __ldg(p.attn + sbase + lane);
+            a = __ldcs(p.attn + si);
         }
-    }
-    if (act) {
-        const int H = sH[l], W = sW[l], start = sStart[l];
-        Corner c[4] = {{-1, 0.f}, {-1, 0.f}, {-1, 0.f}, {-1, 0.f}};
-        float x, y, fx, fy;
-        int x0, y0;
-        if (msda_cell(lx, ly, H, W, x, y, x0, y0, fx, fy)) {
-            const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
-            const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
-            const int MD = M * D;
+        if (j < LK) {  // items past the end get four "outside" entries
+            const int H = sH[l], W = sW[l], start = sStart[l];
+            Corner c[4];
 #pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = msda_row(start, H, W, y0 + (j >> 1), x0 + (j & 1));
-                c[j].off = r < 0 ? -1 : r * MD;
-                c[j].w = w[j] * a;
+            for (int q = 0; q < 4; ++q) c[q] = {-1, 0, make_float2(0.f, 0.f)};
+            float x, y, fx, fy;
+            int x0, y0;
+            if (act && msda_cell(lx, ly, H, W, x, y, x0, y0, fx, fy)) {
+                const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+                const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int r = msda_row(start, H, W, y0 + (q >> 1), x0 + (q & 1));
+                    const float wa = w[q] * a;
+                    c[q].off = r < 0 ? -1 : r * MD;
+                    c[q].w = make_float2(wa, wa);
+                }
             }
-        }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) corners[warp][lane * 4 + j] = c[j];
+            for (int q = 0; q < 4; ++q) corners[warp][seg][j * 4 + q] = c[q];
+        }
     }
     __syncwarp();
 
-    // ---- phase 2: gather the corner rows ---------------------------------
+    // ---- phase 2: gather the corner rows of every item of the warp --------
     const int slot = lane / R;
     const int chunk = lane % R;
-    const bool chunk_ok = chunk < p.nchunks;
-    const VT *vbase = static_cast<const VT *>(p.value) + (n * p.S * M + m) * (int64_t)D +
-                      chunk * kVec;
-    float acc[kVec];
+    const bool chunk_ok = kExact || chunk < p.nchunks;
+    const VT *vbase[kItems];
+    float2 acc[kItems][kNP];
 #pragma unroll
-    for (int i = 0; i < kVec; ++i) acc[i] = 0.f;
+    for (int it = 0; it < kItems; ++it) {
+        const int64_t item = item0 + it;
+        const int m = (int)(item % M);
+        const int64_t n = item / M / p.Lq;
+        vbase[it] = static_cast<const VT *>(p.value) + (n * p.S * M + m) * (int64_t)D +
+                    chunk * (2 * kNP);
+#pragma unroll
+        for (int i = 0; i < kNP; ++i) acc[it][i] = make_float2(0.f, 0.f);
+    }
     const int npairs = 4 * LK;
-#pragma unroll 4
+#pragma unroll 2
     for (int t = slot; t < npairs; t += kSlots) {
-        const Corner e = corners[warp][t];
-        if (e.off >= 0 && chunk_ok) {
-            float v[kVec];
-            Chunk<VT>::load(vbase + e.off, v);
 #pragma unroll
-            for (int i = 0; i < kVec; ++i) acc[i] = fmaf(e.w, v[i], acc[i]);
+        for (int it = 0; it < kItems; ++it) {
+            const Corner e = corners[warp][it][t];
+            float2 v[kNP];
+#pragma unroll
+            for (int i = 0; i < kNP; ++i) v[i] = make_float2(0.f, 0.f);
+            if (e.off >= 0 && chunk_ok) Pairs<VT>::load(vbase[it] + e.off, v);
+#pragma unroll
+            for (int i = 0; i < kNP; ++i) acc[it][i] = __ffma2_rn(e.w, v[i], acc[it][i]);
         }
     }
 
-    // ---- phase 3: combine the slots, store the head's output --------------
+    // ---- phase 3: combine the slots, store each item's output -------------
 #pragma unroll
-    for (int o = R; o < 32; o <<= 1)
+    for (int it = 0; it < kItems; ++it) {
 #pragma unroll
-        for (int i = 0; i < kVec; ++i) acc[i] += __shfl_xor_sync(kFull, acc[i], o);
-    if (slot == 0 && chunk_ok) {
-        float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)(M * D) + m * D +
-                                                 chunk * kVec);
+        for (int o = R; o < 32; o <<= 1)
 #pragma unroll
-        for (int i = 0; i < kVec / 4; ++i)
-            dst[i] = make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+            for (int i = 0; i < kNP; ++i) {
+                acc[it][i].x += __shfl_xor_sync(kFull, acc[it][i].x, o);
+                acc[it][i].y += __shfl_xor_sync(kFull, acc[it][i].y, o);
+            }
+        const int64_t item = item0 + it;
+        if (slot == 0 && chunk_ok && item < p.items) {
+            const int64_t nq = item / M;
+            const int m = (int)(item % M);
+            float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D +
+                                                     chunk * (2 * kNP));
+#pragma unroll
+            for (int i = 0; i < kNP / 2; ++i)
+                __stcs(dst + i, make_float4(acc[it][2 * i].x, acc[it][2 * i].y,
+                                            acc[it][2 * i + 1].x, acc[it][2 * i + 1].y));
+        }
     }
+}
+
+template <typename VT, int R, int P, bool kFused>
+cudaError_t launch_p(const FwdParams &p, bool exact, cudaStream_t stream)
+{
+    constexpr int kItemsPerCta = kWarps * (32 / P);
+    const dim3 block(kWarps * 32);
+    const dim3 grid((unsigned)((p.items + kItemsPerCta - 1) / kItemsPerCta));
+    if (exact)
+        fwd_kernel<VT, R, P, kFused, true><<<grid, block, 0, stream>>>(p);
+    else
+        fwd_kernel<VT, R, P, kFused, false><<<grid, block, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename VT, int R, bool kFused>
+cudaError_t launch_r(const FwdParams &p, bool exact, cudaStream_t stream)
+{
+    const int LK = p.L * p.K;
+    if (LK <= 4) return launch_p<VT, R, 4, kFused>(p, exact, stream);
+    if (LK <= 8) return launch_p<VT, R, 8, kFused>(p, exact, stream);
+    if (LK <= 16) return launch_p<VT, R, 16, kFused>(p, exact, stream);
+    return launch_p<VT, R, 32, kFused>(p, exact, stream);
 }
 
 template <typename VT, bool kFused>
 cudaError_t launch_fwd_vt(const FwdParams &p, int R, cudaStream_t stream)
 {
-    const dim3 block(kWarps * 32);
-    const dim3 grid((unsigned)((p.items + kWarps - 1) / kWarps));
+    const bool exact = p.nchunks == R;
     switch (R) {
-    case 1: fwd_kernel<VT, 1, kFused><<<grid, block, 0, stream>>>(p); break;
-    case 2: fwd_kernel<VT, 2, kFused><<<grid, block, 0, stream>>>(p); break;
-    case 4: fwd_kernel<VT, 4, kFused><<<grid, block, 0, stream>>>(p); break;
-    case 8: fwd_kernel<VT, 8, kFused><<<grid, block, 0, stream>>>(p); break;
-    case 16: fwd_kernel<VT, 16, kFused><<<grid, block, 0, stream>>>(p); break;
-    case 32: fwd_kernel<VT, 32, kFused><<<grid, block, 0, stream>>>(p); break;
+    case 1: return launch_r<VT, 1, kFused>(p, exact, stream);
+    case 2: return launch_r<VT, 2, kFused>(p, exact, stream);
+    case 4: return launch_r<VT, 4, kFused>(p, exact, stream);
+    case 8: return launch_r<VT, 8, kFused>(p, exact, stream);
+    case 16: return launch_r<VT, 16, kFused>(p, exact, stream);
+    case 32: return launch_r<VT, 32, kFused>(p, exact, stream);
     default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace

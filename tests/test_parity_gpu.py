@@ -200,9 +200,9 @@ def test_stress_forward_backward():
         assert_close(host(gv[sl]), ogv, **GRAD, what=f"stress grad_value n={n}")
         assert_close(host(gl[sl]), ogl, **GRAD, what=f"stress grad_loc n={n}", mass=mgl)
         assert_close(host(ga[sl]), oga, **GRAD, what=f"stress grad_attn n={n}", mass=mga)
-    # the pushed-out samples really are out: about 5% of loc invalid or partial
+    # at least the pushed 5% of the samples leave their level
     valid = host(msda_debug_sample_points(sh, None, loc_o[:1])["valid"])
-    assert 0.03 < 1.0 - valid.mean() < 0.08
+    assert 1.0 - valid.mean() > 0.05  # pushed 5% plus natural spill at coarse levels
 
 
 # ---------------------------------------------------------------------------
