@@ -58,9 +58,31 @@ __device__ __forceinline__ void reduce_scatter(float (&v)[kNV], int lane)
     }
 }
 
+// Butterfly reduce-scatter of N values over aligned groups of SPAN lanes
+// (N a multiple of SPAN): afterwards lane b = lane % SPAN holds in v[0, N/SPAN)
+// the group totals of values b*N/SPAN ... (b+1)*N/SPAN - 1.
+template <int SPAN, int N>
+__device__ __forceinline__ void reduce_scatter_n(float (&v)[N], int lane)
+{
+    if constexpr (SPAN > 1) {
+        constexpr int o = SPAN / 2;
+        constexpr int h = N / 2;
+        const bool upper = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < h; ++i) {
+            const float send = upper ? v[i] : v[i + h];
+            const float keep = upper ? v[i + h] : v[i];
+            v[i] = keep + __shfl_xor_sync(kFull, send, o);
+        }
+        reduce_scatter_n<o, N>(v, lane);  // the low halves now hold the partial sums
+    }
+}
+
+// Generic path (any row width): one warp per item, partial sums of 32 lanes
+// reduced every 8 samples.  Used for rows wider than 128 bytes.
 template <typename VT, int R>
 __global__ void __launch_bounds__(kWarps * 32)
-    bwd_kernel(const __grid_constant__ BwdParams p)
+    bwd_kernel_wide(const __grid_constant__ BwdParams p)
 {
     constexpr int kVec = Chunk<VT>::kVec;
     constexpr int kSpan = (4 * R < 32) ? 4 * R : 32;  // lanes per sample
@@ -204,18 +226,237 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
 }
 
+// Fast path for rows of at most 128 bytes (R <= 8, so a warp instruction
+// covers 32/R >= 4 (sample, corner) pairs: kSG = 8/R samples of four corners).
+//   - Persistent CTAs sweep contiguous item ranges (L1 locality), a warp
+//     takes 32/P items per round and phase 1 gives every lane one sample.
+//   - Per item, 16 samples at a time (8 for bf16 rows of 128 bytes): all corner rows are loaded before any
+//     is used; each lane forms t = <v_chunk, g_chunk> and scatters
+//     A*w*g_chunk with a vector reduction.
+//   - The 16 partial t of a lane are reduced over the R chunk lanes with a
+//     butterfly reduce-scatter (each lane keeps two finished <v_c, g>), then
+//     weighted by (w, dw/dfx, dw/dfy) of its corner and summed over the four
+//     corner lanes with two xor steps: about 1.6 shuffles per sample.
+template <typename VT, int R, int P>
+__global__ void __launch_bounds__(kWarps * 32, 2)
+    bwd_kernel(const __grid_constant__ BwdParams p)
+{
+    static_assert(R <= 8, "fast path needs at least four pairs per instruction");
+    constexpr int kVec = Chunk<VT>::kVec;  // value elements per 16-byte chunk
+    constexpr int kSlots = 32 / R;         // pairs per warp instruction
+    constexpr int kSG = kSlots / 4;        // samples per warp instruction
+    // instructions per batch: 16 samples, or fewer if the loaded chunks would
+    // exceed 64 registers (bf16 with 128-byte rows: 8 samples)
+    constexpr int kB = (2 * R < 64 / kVec) ? 2 * R : 64 / kVec;
+    constexpr int kBS = kB * kSG;          // samples per batch
+    constexpr int kItems = 32 / P;
+    static_assert(kB % R == 0, "a batch must split evenly over the chunk lanes");
+    constexpr int kKeep = kB / R;          // finished <v_c, g> per lane after stage A
+
+    __shared__ CornerB corners[kWarps][kItems][4 * P];
+    __shared__ float sA[kWarps][kItems][P];
+    __shared__ int sH[kMaxLevels], sW[kMaxLevels], sStart[kMaxLevels];
+
+    const int tid = threadIdx.x;
+    if (tid < p.L) {
+        sH[tid] = p.lv.H[tid];
+        sW[tid] = p.lv.W[tid];
+        sStart[tid] = p.lv.start[tid];
+    }
+    __syncthreads();
+
+    const int warp = tid >> 5;
+    const int lane = tid & 31;
+    const int M = p.M, D = p.D, K = p.K;
+    const int LK = p.L * K;
+    const int MD = M * D;
+    const int slot = lane / R;
+    const int chunk = lane % R;
+    const int corner = slot & 3;
+    const int sg = slot >> 2;
+    const bool chunk_ok = chunk < p.nchunks;
+
+    const int64_t begin = (int64_t)blockIdx.x * p.chunk;
+    const int64_t end = begin + p.chunk < p.items ? begin + p.chunk : p.items;
+
+    for (int64_t item0 = begin + warp * kItems; item0 < end; item0 += kWarps * kItems) {
+        // ---- phase 1: cell and corner derivatives, one sample per lane ----
+        {
+            const int seg = lane / P;
+            const int j = lane % P;
+            const int64_t item = item0 + seg;
+            const bool act = j < LK && item < end;
+            if (j < LK) {
+                const int l = j / K;
+                const int H = sH[l], W = sW[l], start = sStart[l];
+                CornerB c[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) c[q] = {-1, 0.f, 0.f, 0.f};
+                float a = 0.f;
+                if (act) {
+                    const int64_t si = item * LK + j;
+                    const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
+                    a = __ldcs(p.attn + si);
+                    float x, y, fx, fy;
+                    int x0, y0;
+                    if (msda_cell(t.x, t.y, H, W, x, y, x0, y0, fx, fy)) {
+                        const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+                        const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
+                        const float dwx[4] = {-hy, hy, -fy, fy};
+                        const float dwy[4] = {-hx, -fx, hx, fx};
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            const int r = msda_row(start, H, W, y0 + (q >> 1), x0 + (q & 1));
+                            c[q] = {r < 0 ? -1 : r * MD, w[q], dwx[q], dwy[q]};
+                        }
+                    }
+                }
+                sA[warp][seg][j] = a;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) corners[warp][seg][j * 4 + q] = c[q];
+            }
+        }
+        __syncwarp();
+
+        // ---- phase 2: per item, 16 samples at a time ----------------------
+#pragma unroll 1
+        for (int it = 0; it < kItems; ++it) {
+            const int64_t item = item0 + it;
+            if (item >= end) break;  // uniform
+            const int m = (int)(item % M);
+            const int64_t nq = item / M;
+            const int64_t n = nq / p.Lq;
+            const int64_t sbase = item * LK;
+            float g[kVec];
+            if (chunk_ok) {
+                const float4 *gp = reinterpret_cast<const float4 *>(
+                    p.grad_out + nq * (int64_t)MD + m * D + chunk * kVec);
+#pragma unroll
+                for (int i = 0; i < kVec / 4; ++i) {
+                    const float4 t = __ldcs(gp + i);
+                    g[4 * i] = t.x;
+                    g[4 * i + 1] = t.y;
+                    g[4 * i + 2] = t.z;
+                    g[4 * i + 3] = t.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < kVec; ++i) g[i] = 0.f;
+            }
+            const int64_t rowbase = (n * p.S * M + m) * (int64_t)D + chunk * kVec;
+            const VT *vb = static_cast<const VT *>(p.value) + rowbase;
+            float *gvb = p.grad_value + rowbase;
+
+            for (int s0 = 0; s0 < LK; s0 += kBS) {
+                // loads: instruction b covers samples s0 + b*kSG + (0..kSG-1)
+                float v[kB][kVec];
+                int off[kB];
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    const int s = s0 + b * kSG + sg;
+                    off[b] = s < LK ? corners[warp][it][s * 4 + corner].off : -1;
+#pragma unroll
+                    for (int i = 0; i < kVec; ++i) v[b][i] = 0.f;
+                    if (off[b] >= 0 && chunk_ok) Chunk<VT>::load(vb + off[b], v[b]);
+                }
+                float t[kB];
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    t[b] = 0.f;
+#pragma unroll
+                    for (int i = 0; i < kVec; ++i) t[b] = fmaf(v[b][i], g[i], t[b]);
+                    if (off[b] >= 0 && chunk_ok) {
+                        const int s = s0 + b * kSG + sg;
+                        const float aw = sA[warp][it][s] * corners[warp][it][s * 4 + corner].w;
+                        float *dst = gvb + off[b];
+#pragma unroll
+                        for (int i = 0; i < kVec; i += 4)
+                            red_add_v4(dst + i, aw * g[i], aw * g[i + 1], aw * g[i + 2],
+                                       aw * g[i + 3]);
+                    }
+                }
+                // stage A: reduce t over the R chunk lanes (lane bits below R)
+                reduce_scatter_n<R, kB>(t, lane);
+                // lane now holds <v_corner, g> of instructions b = chunk*kKeep + k
+                float q[3][kKeep];
+#pragma unroll
+                for (int k = 0; k < kKeep; ++k) {
+                    const int b = chunk * kKeep + k;
+                    const int s = s0 + b * kSG + sg;
+                    CornerB e = {-1, 0.f, 0.f, 0.f};
+                    if (s < LK) e = corners[warp][it][s * 4 + corner];
+                    q[0][k] = e.w * t[k];
+                    q[1][k] = e.dwx * t[k];
+                    q[2][k] = e.dwy * t[k];
+                }
+                // stage B: sum over the four corner lanes of each sample
+#pragma unroll
+                for (int o = R; o < 4 * R; o <<= 1)
+#pragma unroll
+                    for (int k = 0; k < kKeep; ++k) {
+                        q[0][k] += __shfl_xor_sync(kFull, q[0][k], o);
+                        q[1][k] += __shfl_xor_sync(kFull, q[1][k], o);
+                        q[2][k] += __shfl_xor_sync(kFull, q[2][k], o);
+                    }
+                if (corner == 0) {
+#pragma unroll
+                    for (int k = 0; k < kKeep; ++k) {
+                        const int b = chunk * kKeep + k;
+                        const int s = s0 + b * kSG + sg;
+                        if (s < LK) {
+                            const int64_t si = sbase + s;
+                            if (p.grad_attn) __stcs(p.grad_attn + si, q[0][k]);
+                            if (p.grad_loc) {
+                                const int l = s / K;
+                                const float a = sA[warp][it][s];
+                                __stcs(reinterpret_cast<float2 *>(p.grad_loc) + si,
+                                       make_float2(a * ((float)sW[l] * q[1][k]),
+                                                   a * ((float)sH[l] * q[2][k])));
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        __syncwarp();
+    }
+}
+
+template <typename VT, int R, int P>
+cudaError_t launch_fast(BwdParams p, cudaStream_t stream)
+{
+    constexpr int kRound = kWarps * (32 / P);
+    auto kern = bwd_kernel<VT, R, P>;
+    const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kRound);
+    p.chunk = (p.items + ctas - 1) / ctas;
+    p.chunk = (p.chunk + kRound - 1) / kRound * kRound;
+    const dim3 grid((unsigned)((p.items + p.chunk - 1) / p.chunk));
+    kern<<<grid, kWarps * 32, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename VT, int R>
+cudaError_t launch_fast_r(const BwdParams &p, cudaStream_t stream)
+{
+    const int LK = p.L * p.K;
+    if (LK <= 4) return launch_fast<VT, R, 4>(p, stream);
+    if (LK <= 8) return launch_fast<VT, R, 8>(p, stream);
+    if (LK <= 16) return launch_fast<VT, R, 16>(p, stream);
+    return launch_fast<VT, R, 32>(p, stream);
+}
+
 template <typename VT>
 cudaError_t launch_bwd_vt(const BwdParams &p, int R, cudaStream_t stream)
 {
     const dim3 block(kWarps * 32);
     const dim3 grid((unsigned)((p.items + kWarps - 1) / kWarps));
     switch (R) {
-    case 1: bwd_kernel<VT, 1><<<grid, block, 0, stream>>>(p); break;
-    case 2: bwd_kernel<VT, 2><<<grid, block, 0, stream>>>(p); break;
-    case 4: bwd_kernel<VT, 4><<<grid, block, 0, stream>>>(p); break;
-    case 8: bwd_kernel<VT, 8><<<grid, block, 0, stream>>>(p); break;
-    case 16: bwd_kernel<VT, 16><<<grid, block, 0, stream>>>(p); break;
-    case 32: bwd_kernel<VT, 32><<<grid, block, 0, stream>>>(p); break;
+    case 1: return launch_fast_r<VT, 1>(p, stream);
+    case 2: return launch_fast_r<VT, 2>(p, stream);
+    case 4: return launch_fast_r<VT, 4>(p, stream);
+    case 8: return launch_fast_r<VT, 8>(p, stream);
+    case 16: bwd_kernel_wide<VT, 16><<<grid, block, 0, stream>>>(p); break;
+    case 32: bwd_kernel_wide<VT, 32><<<grid, block, 0, stream>>>(p); break;
     default: return cudaErrorInvalidValue;
     }
     return cudaGetLastError();

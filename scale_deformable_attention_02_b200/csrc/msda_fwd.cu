@@ -35,10 +35,9 @@ namespace {
 
 constexpr int kWarps = 8;  // warps per CTA
 
-struct __align__(16) Corner {
-    int off;    // element offset of the corner row inside the (n, m) map; -1 = outside
-    int pad;
-    float2 w;   // (w, w): bilinear weight times the attention weight, twice
+struct __align__(8) Corner {
+    int off;  // element offset of the corner row inside the (n, m) map; -1 = outside
+    float w;  // bilinear weight times the attention weight
 };
 
 template <int P>
@@ -86,12 +85,16 @@ struct Pairs<__nv_bfloat16> {
 };
 
 template <typename VT, int R, int P, bool kFused, bool kExact>
-__global__ void __launch_bounds__(kWarps * 32)
+__global__ void __launch_bounds__(kWarps * 32, 2)
     fwd_kernel(const __grid_constant__ FwdParams p)
 {
-    constexpr int kNP = Pairs<VT>::kN;   // float pairs per 16-byte chunk
-    constexpr int kSlots = 32 / R;       // (sample, corner) pairs per warp instruction
-    constexpr int kItems = 32 / P;       // items per warp
+    constexpr int kNP = Pairs<VT>::kN;  // float pairs per 16-byte chunk
+    constexpr int kSlots = 32 / R;      // (sample, corner) pairs per warp instruction
+    constexpr int kItems = 32 / P;      // items per warp per round
+    // gathers issued before the first is consumed (64 pairs = 16 samples)
+    // (at most 64 registers of loaded data: 16 fp32 chunks or 8 bf16 chunks)
+    constexpr int kB0 = (64 / kSlots) < 4 ? 4 : ((64 / kSlots) > 16 ? 16 : 64 / kSlots);
+    constexpr int kB = kB0 < 32 / kNP ? kB0 : 32 / kNP;
     __shared__ Corner corners[kWarps][kItems][4 * P];
     __shared__ int sH[kMaxLevels], sW[kMaxLevels], sStart[kMaxLevels];
 
@@ -105,142 +108,146 @@ __global__ void __launch_bounds__(kWarps * 32)
 
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int64_t item0 = ((int64_t)blockIdx.x * kWarps + warp) * kItems;
-    if (item0 >= p.items) return;  // whole warp leaves together
-
     const int M = p.M, D = p.D, K = p.K;
     const int LK = p.L * K;
     const int MD = M * D;
-
-    // ---- phase 1: one sample per lane -------------------------------------
-    {
-        const int seg = lane / P;  // item within the warp
-        const int j = lane % P;    // sample within the item
-        const int64_t item = item0 + seg;
-        const bool act = j < LK && item < p.items;
-        const int64_t si = item * LK + j;
-        const int l = act ? j / K : 0;
-        float lx = 0.f, ly = 0.f, a = 0.f;
-        if constexpr (kFused) {
-            const float z = act ? __ldcs(p.logits + si) : -INFINITY;
-            const float mx = seg_max<P>(z);
-            const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
-            const float s = seg_sum<P>(e);
-            a = __fdiv_rn(e, s);
-            if (act) {
-                const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + si);
-                const int64_t nq = item / M;
-                if (p.ref_dim == 2) {
-                    // point reference: offsets are level-l pixels
-                    const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
-                    lx = __fadd_rn(r.x, __fdiv_rn(o.x, (float)sW[l]));
-                    ly = __fadd_rn(r.y, __fdiv_rn(o.y, (float)sH[l]));
-                } else {
-                    // box reference (cx, cy, w, h): offsets are in box units
-                    const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
-                    const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
-                    lx = __fadd_rn(c.x, __fmul_rn(o.x, s2.x));
-                    ly = __fadd_rn(c.y, __fmul_rn(o.y, s2.y));
-                }
-                if (p.loc_out)
-                    __stcs(reinterpret_cast<float2 *>(p.loc_out) + si, make_float2(lx, ly));
-                if (p.attn_out) __stcs(p.attn_out + si, a);
-            }
-        } else if (act) {
-            const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
-            lx = t.x;
-            ly = t.y;
-            a = __ldcs(p.attn + si);
-        }
-        if (j < LK) {  // items past the end get four "outside" entries
-            const int H = sH[l], W = sW[l], start = sStart[l];
-            Corner c[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) c[q] = {-1, 0, make_float2(0.f, 0.f)};
-            float x, y, fx, fy;
-            int x0, y0;
-            if (act && msda_cell(lx, ly, H, W, x, y, x0, y0, fx, fy)) {
-                const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
-                const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int r = msda_row(start, H, W, y0 + (q >> 1), x0 + (q & 1));
-                    const float wa = w[q] * a;
-                    c[q].off = r < 0 ? -1 : r * MD;
-                    c[q].w = make_float2(wa, wa);
-                }
-            }
-#pragma unroll
-            for (int q = 0; q < 4; ++q) corners[warp][seg][j * 4 + q] = c[q];
-        }
-    }
-    __syncwarp();
-
-    // ---- phase 2: gather the corner rows of every item of the warp --------
+    const int npairs = 4 * LK;
     const int slot = lane / R;
     const int chunk = lane % R;
     const bool chunk_ok = kExact || chunk < p.nchunks;
-    const VT *vbase[kItems];
-    float2 acc[kItems][kNP];
-#pragma unroll
-    for (int it = 0; it < kItems; ++it) {
-        const int64_t item = item0 + it;
-        const int m = (int)(item % M);
-        const int64_t n = item / M / p.Lq;
-        vbase[it] = static_cast<const VT *>(p.value) + (n * p.S * M + m) * (int64_t)D +
-                    chunk * (2 * kNP);
-#pragma unroll
-        for (int i = 0; i < kNP; ++i) acc[it][i] = make_float2(0.f, 0.f);
-    }
-    const int npairs = 4 * LK;
-#pragma unroll 2
-    for (int t = slot; t < npairs; t += kSlots) {
-#pragma unroll
-        for (int it = 0; it < kItems; ++it) {
-            const Corner e = corners[warp][it][t];
-            float2 v[kNP];
-#pragma unroll
-            for (int i = 0; i < kNP; ++i) v[i] = make_float2(0.f, 0.f);
-            if (e.off >= 0 && chunk_ok) Pairs<VT>::load(vbase[it] + e.off, v);
-#pragma unroll
-            for (int i = 0; i < kNP; ++i) acc[it][i] = __ffma2_rn(e.w, v[i], acc[it][i]);
-        }
-    }
 
-    // ---- phase 3: combine the slots, store each item's output -------------
-#pragma unroll
-    for (int it = 0; it < kItems; ++it) {
-#pragma unroll
-        for (int o = R; o < 32; o <<= 1)
-#pragma unroll
-            for (int i = 0; i < kNP; ++i) {
-                acc[it][i].x += __shfl_xor_sync(kFull, acc[it][i].x, o);
-                acc[it][i].y += __shfl_xor_sync(kFull, acc[it][i].y, o);
+    // This CTA sweeps the contiguous item range [begin, end): neighbouring
+    // queries sample neighbouring pixels, so the sweep keeps rows in L1.
+    const int64_t begin = (int64_t)blockIdx.x * p.chunk;
+    const int64_t end = begin + p.chunk < p.items ? begin + p.chunk : p.items;
+
+    for (int64_t item0 = begin + warp * kItems; item0 < end; item0 += kWarps * kItems) {
+        // ---- phase 1: one sample per lane ---------------------------------
+        {
+            const int seg = lane / P;  // item within the round
+            const int j = lane % P;    // sample within the item
+            const int64_t item = item0 + seg;
+            const bool act = j < LK && item < end;
+            const int64_t si = item * LK + j;
+            const int l = act ? j / K : 0;
+            float lx = 0.f, ly = 0.f, a = 0.f;
+            if constexpr (kFused) {
+                const float z = act ? __ldcs(p.logits + si) : -INFINITY;
+                const float mx = seg_max<P>(z);
+                const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
+                const float s = seg_sum<P>(e);
+                a = __fdiv_rn(e, s);
+                if (act) {
+                    const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + si);
+                    const int64_t nq = item / M;
+                    if (p.ref_dim == 2) {
+                        // point reference: offsets are level-l pixels
+                        const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
+                        lx = __fadd_rn(r.x, __fdiv_rn(o.x, (float)sW[l]));
+                        ly = __fadd_rn(r.y, __fdiv_rn(o.y, (float)sH[l]));
+                    } else {
+                        // box reference (cx, cy, w, h): offsets are in box units
+                        const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
+                        const float2 s2 =
+                            __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
+                        lx = __fadd_rn(c.x, __fmul_rn(o.x, s2.x));
+                        ly = __fadd_rn(c.y, __fmul_rn(o.y, s2.y));
+                    }
+                    if (p.loc_out)
+                        __stcs(reinterpret_cast<float2 *>(p.loc_out) + si, make_float2(lx, ly));
+                    if (p.attn_out) __stcs(p.attn_out + si, a);
+                }
+            } else if (act) {
+                const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
+                lx = t.x;
+                ly = t.y;
+                a = __ldcs(p.attn + si);
             }
-        const int64_t item = item0 + it;
-        if (slot == 0 && chunk_ok && item < p.items) {
-            const int64_t nq = item / M;
-            const int m = (int)(item % M);
-            float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D +
-                                                     chunk * (2 * kNP));
+            if (j < LK) {  // items past the end get four "outside" entries
+                const int H = sH[l], W = sW[l], start = sStart[l];
+                Corner c[4];
 #pragma unroll
-            for (int i = 0; i < kNP / 2; ++i)
-                __stcs(dst + i, make_float4(acc[it][2 * i].x, acc[it][2 * i].y,
-                                            acc[it][2 * i + 1].x, acc[it][2 * i + 1].y));
+                for (int q = 0; q < 4; ++q) c[q] = {-1, 0.f};
+                float x, y, fx, fy;
+                int x0, y0;
+                if (act && msda_cell(lx, ly, H, W, x, y, x0, y0, fx, fy)) {
+                    const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+                    const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int r = msda_row(start, H, W, y0 + (q >> 1), x0 + (q & 1));
+                        c[q].off = r < 0 ? -1 : r * MD;
+                        c[q].w = w[q] * a;
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) corners[warp][seg][j * 4 + q] = c[q];
+            }
         }
+        __syncwarp();
+
+        // ---- phase 2: gather, item by item --------------------------------
+#pragma unroll 1
+        for (int it = 0; it < kItems; ++it) {
+            const int64_t item = item0 + it;
+            if (item >= end) break;  // uniform across the warp
+            const int m = (int)(item % M);
+            const int64_t nq = item / M;
+            const int64_t n = nq / p.Lq;
+            const VT *vb = static_cast<const VT *>(p.value) + (n * p.S * M + m) * (int64_t)D +
+                           chunk * (2 * kNP);
+            float2 acc[kNP];
+#pragma unroll
+            for (int i = 0; i < kNP; ++i) acc[i] = make_float2(0.f, 0.f);
+            for (int t0 = 0; t0 < npairs; t0 += kB * kSlots) {
+                float2 v[kB][kNP];
+                float w[kB];
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    const int t = t0 + b * kSlots + slot;
+                    const Corner e = t < npairs ? corners[warp][it][t] : Corner{-1, 0.f};
+                    w[b] = e.w;
+#pragma unroll
+                    for (int i = 0; i < kNP; ++i) v[b][i] = make_float2(0.f, 0.f);
+                    if (e.off >= 0 && chunk_ok) Pairs<VT>::load(vb + e.off, v[b]);
+                }
+#pragma unroll
+                for (int b = 0; b < kB; ++b)
+#pragma unroll
+                    for (int i = 0; i < kNP; ++i)
+                        acc[i] = __ffma2_rn(make_float2(w[b], w[b]), v[b][i], acc[i]);
+            }
+            // combine the slots of each chunk, store the item's D outputs
+#pragma unroll
+            for (int o = R; o < 32; o <<= 1)
+#pragma unroll
+                for (int i = 0; i < kNP; ++i) {
+                    acc[i].x += __shfl_xor_sync(kFull, acc[i].x, o);
+                    acc[i].y += __shfl_xor_sync(kFull, acc[i].y, o);
+                }
+            if (slot == 0 && chunk_ok) {
+                float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D +
+                                                         chunk * (2 * kNP));
+#pragma unroll
+                for (int i = 0; i < kNP / 2; ++i)
+                    __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
+                                                acc[2 * i + 1].y));
+            }
+        }
+        __syncwarp();  // the next round overwrites this warp's corner entries
     }
 }
 
 template <typename VT, int R, int P, bool kFused>
-cudaError_t launch_p(const FwdParams &p, bool exact, cudaStream_t stream)
+cudaError_t launch_p(FwdParams p, bool exact, cudaStream_t stream)
 {
-    constexpr int kItemsPerCta = kWarps * (32 / P);
-    const dim3 block(kWarps * 32);
-    const dim3 grid((unsigned)((p.items + kItemsPerCta - 1) / kItemsPerCta));
-    if (exact)
-        fwd_kernel<VT, R, P, kFused, true><<<grid, block, 0, stream>>>(p);
-    else
-        fwd_kernel<VT, R, P, kFused, false><<<grid, block, 0, stream>>>(p);
+    constexpr int kRound = kWarps * (32 / P);  // items per CTA round
+    auto kern = exact ? fwd_kernel<VT, R, P, kFused, true> : fwd_kernel<VT, R, P, kFused, false>;
+    const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kRound);
+    p.chunk = (p.items + ctas - 1) / ctas;
+    p.chunk = (p.chunk + kRound - 1) / kRound * kRound;
+    const dim3 grid((unsigned)((p.items + p.chunk - 1) / p.chunk));
+    kern<<<grid, kWarps * 32, 0, stream>>>(p);
     return cudaGetLastError();
 }
 

@@ -25,7 +25,8 @@ struct FwdParams {
     float *out;       // [N,Lq,M*D]
     float *loc_out;   // nullable (fused)
     float *attn_out;  // nullable (fused)
-    int64_t items;    // N*Lq*M (one warp each)
+    int64_t items;    // N*Lq*M
+    int64_t chunk;    // items per CTA (set by the launcher)
     int Lq, S, M, D, L, K;
     int nchunks;  // 16-byte chunks per value row
     Levels lv;
@@ -40,6 +41,7 @@ struct BwdParams {
     float *grad_loc;   // nullable
     float *grad_attn;  // nullable
     int64_t items;
+    int64_t chunk;  // items per CTA (set by the launcher)
     int Lq, S, M, D, L, K;
     int nchunks;
     Levels lv;
@@ -54,6 +56,10 @@ struct PointsParams {
     int L, K;
     Levels lv;
 };
+
+// CTAs for a persistent launch: (SMs x resident CTAs of `kernel`) on the
+// current device, but no more than the rounds of `round` items there are.
+int64_t persistent_ctas(const void *kernel, int threads, int64_t items, int round);
 
 // Launchers (return the launch's cudaError_t).
 cudaError_t launch_forward(const FwdParams &p, bool bf16, bool fused, int lanes_per_row,
