@@ -58,15 +58,16 @@ __device__ __forceinline__ void reduce_scatter(float (&v)[kNV], int lane)
     }
 }
 
-// Butterfly reduce-scatter of N values over aligned groups of SPAN lanes
-// (N a multiple of SPAN): afterwards lane b = lane % SPAN holds in v[0, N/SPAN)
-// the group totals of values b*N/SPAN ... (b+1)*N/SPAN - 1.
-template <int SPAN, int N>
+// Butterfly reduce-scatter of the first CNT values of v over aligned groups
+// of SPAN lanes (CNT a multiple of SPAN): afterwards lane b = lane % SPAN holds
+// in v[0, CNT/SPAN) the group totals of values b*CNT/SPAN ... (b+1)*CNT/SPAN - 1.
+template <int SPAN, int CNT, int N>
 __device__ __forceinline__ void reduce_scatter_n(float (&v)[N], int lane)
 {
+    static_assert(CNT <= N && CNT % SPAN == 0, "reduce-scatter shape");
     if constexpr (SPAN > 1) {
         constexpr int o = SPAN / 2;
-        constexpr int h = N / 2;
+        constexpr int h = CNT / 2;
         const bool upper = (lane & o) != 0;
 #pragma unroll
         for (int i = 0; i < h; ++i) {
@@ -74,7 +75,7 @@ __device__ __forceinline__ void reduce_scatter_n(float (&v)[N], int lane)
             const float keep = upper ? v[i + h] : v[i];
             v[i] = keep + __shfl_xor_sync(kFull, send, o);
         }
-        reduce_scatter_n<o, N>(v, lane);  // the low halves now hold the partial sums
+        reduce_scatter_n<o, h, N>(v, lane);  // the kept half now sits in v[0, h)
     }
 }
 
@@ -376,7 +377,7 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
                     }
                 }
                 // stage A: reduce t over the R chunk lanes (lane bits below R)
-                reduce_scatter_n<R, kB>(t, lane);
+                reduce_scatter_n<R, kB, kB>(t, lane);
                 // lane now holds <v_corner, g> of instructions b = chunk*kKeep + k
                 float q[3][kKeep];
 #pragma unroll
