@@ -38,6 +38,43 @@ struct __align__(16) CornerB {
     float dwy;  // d w / d fy
 };
 
+// A raw 16-byte chunk of a value row, widened to fp32 (bf16 widening is exact).
+template <typename VT>
+__device__ __forceinline__ void widen(const uint4 &r, float (&v)[Chunk<VT>::kVec]);
+
+template <>
+__device__ __forceinline__ void widen<float>(const uint4 &r, float (&v)[4])
+{
+    v[0] = __uint_as_float(r.x);
+    v[1] = __uint_as_float(r.y);
+    v[2] = __uint_as_float(r.z);
+    v[3] = __uint_as_float(r.w);
+}
+
+template <>
+__device__ __forceinline__ void widen<__nv_bfloat16>(const uint4 &r, float (&v)[8])
+{
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+}
+
+// Gather/scatter entry of one corner: its value row's address (already offset
+// to the batch entry and head), A*w, and the element offset of the matching
+// grad_value row inside the (n, m) map (-1: outside the level, nothing to
+// scatter).  Corners outside the level read kZeroRowB, so the gathers need no
+// predicate; only the scatter is predicated.
+struct __align__(16) CornerG {
+    const char *row;
+    float aw;
+    int goff;
+};
+
+__device__ __align__(128) float4 kZeroRowB[32] = {};
+
 // Butterfly reduce-scatter over aligned groups of SPAN lanes.  Before: every
 // lane holds N partial values.  After: lane (lane % SPAN) = b holds, in
 // v[0 .. N/SPAN), the group totals of values b*N/SPAN .. (b+1)*N/SPAN - 1.
@@ -252,9 +289,15 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
     constexpr int kBS = kB * kSG;          // samples per batch
     constexpr int kItems = 32 / P;
     static_assert(kB % R == 0, "a batch must split evenly over the chunk lanes");
+    static_assert(kBS <= P && P % kBS == 0, "a batch must stay inside the P sample slots");
     constexpr int kKeep = kB / R;          // finished <v_c, g> per lane after stage A
 
-    __shared__ CornerB corners[kWarps][kItems][4 * P];
+    // Per corner: (row offset, A*w) for the gather/scatter loop and
+    // (w, dw/dfx, dw/dfy) for the reduction; corner-major with row stride
+    // P + 2 (= 2 mod 8) so that both phases are free of bank conflicts.
+    constexpr int kStride = P + 2;
+    __shared__ CornerG cOff[kWarps][kItems][4 * kStride];
+    __shared__ float4 cDer[kWarps][kItems][4 * kStride];
     __shared__ float sA[kWarps][kItems][P];
     __shared__ int sH[kMaxLevels], sW[kMaxLevels], sStart[kMaxLevels];
 
@@ -287,12 +330,17 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
             const int j = lane % P;
             const int64_t item = item0 + seg;
             const bool act = j < LK && item < end;
-            if (j < LK) {
-                const int l = j / K;
+            {  // every sample slot up to P gets entries; unused ones read zeros
+                const int l = j < LK ? j / K : 0;
                 const int H = sH[l], W = sW[l], start = sStart[l];
-                CornerB c[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) c[q] = {-1, 0.f, 0.f, 0.f};
+                const int m = (int)(item % M);
+                const int64_t n = item / M / p.Lq;
+                const char *mapb = static_cast<const char *>(p.value) +
+                                   ((n * p.S * M + m) * (int64_t)D) * (int64_t)sizeof(VT);
+                int off[4] = {-1, -1, -1, -1};
+                float w[4] = {0.f, 0.f, 0.f, 0.f};
+                float dwx[4] = {0.f, 0.f, 0.f, 0.f};
+                float dwy[4] = {0.f, 0.f, 0.f, 0.f};
                 float a = 0.f;
                 if (act) {
                     const int64_t si = item * LK + j;
@@ -302,19 +350,36 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
                     int x0, y0;
                     if (msda_cell(t.x, t.y, H, W, x, y, x0, y0, fx, fy)) {
                         const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
-                        const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
-                        const float dwx[4] = {-hy, hy, -fy, fy};
-                        const float dwy[4] = {-hx, -fx, hx, fx};
+                        w[0] = hy * hx;
+                        w[1] = hy * fx;
+                        w[2] = fy * hx;
+                        w[3] = fy * fx;
+                        dwx[0] = -hy;
+                        dwx[1] = hy;
+                        dwx[2] = -fy;
+                        dwx[3] = fy;
+                        dwy[0] = -hx;
+                        dwy[1] = -fx;
+                        dwy[2] = hx;
+                        dwy[3] = fx;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
                             const int r = msda_row(start, H, W, y0 + (q >> 1), x0 + (q & 1));
-                            c[q] = {r < 0 ? -1 : r * MD, w[q], dwx[q], dwy[q]};
+                            off[q] = r < 0 ? -1 : r * MD;
                         }
                     }
                 }
                 sA[warp][seg][j] = a;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) corners[warp][seg][j * 4 + q] = c[q];
+                for (int q = 0; q < 4; ++q) {
+                    CornerG g;
+                    g.row = off[q] >= 0 ? mapb + (int64_t)off[q] * (int64_t)sizeof(VT)
+                                        : reinterpret_cast<const char *>(kZeroRowB);
+                    g.aw = a * w[q];
+                    g.goff = off[q];
+                    cOff[warp][seg][q * kStride + j] = g;
+                    cDer[warp][seg][q * kStride + j] = make_float4(w[q], dwx[q], dwy[q], 0.f);
+                }
             }
         }
         __syncwarp();
@@ -345,35 +410,37 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
                 for (int i = 0; i < kVec; ++i) g[i] = 0.f;
             }
             const int64_t rowbase = (n * p.S * M + m) * (int64_t)D + chunk * kVec;
-            const VT *vb = static_cast<const VT *>(p.value) + rowbase;
             float *gvb = p.grad_value + rowbase;
+            // lanes past the last chunk re-read chunk 0 (their g is zero)
+            const int lane_off = chunk_ok ? chunk * 16 : 0;
 
             for (int s0 = 0; s0 < LK; s0 += kBS) {
                 // loads: instruction b covers samples s0 + b*kSG + (0..kSG-1)
-                float v[kB][kVec];
-                int off[kB];
+                uint4 raw[kB];
+                float aw[kB];
+                int goff[kB];
 #pragma unroll
                 for (int b = 0; b < kB; ++b) {
-                    const int s = s0 + b * kSG + sg;
-                    off[b] = s < LK ? corners[warp][it][s * 4 + corner].off : -1;
-#pragma unroll
-                    for (int i = 0; i < kVec; ++i) v[b][i] = 0.f;
-                    if (off[b] >= 0 && chunk_ok) Chunk<VT>::load(vb + off[b], v[b]);
+                    const int s = s0 + b * kSG + sg;  // < P: every slot has an entry
+                    const CornerG e = cOff[warp][it][corner * kStride + s];
+                    raw[b] = __ldg(reinterpret_cast<const uint4 *>(e.row + lane_off));
+                    aw[b] = e.aw;
+                    goff[b] = e.goff;
                 }
                 float t[kB];
 #pragma unroll
                 for (int b = 0; b < kB; ++b) {
+                    float v[kVec];
+                    widen<VT>(raw[b], v);
                     t[b] = 0.f;
 #pragma unroll
-                    for (int i = 0; i < kVec; ++i) t[b] = fmaf(v[b][i], g[i], t[b]);
-                    if (off[b] >= 0 && chunk_ok) {
-                        const int s = s0 + b * kSG + sg;
-                        const float aw = sA[warp][it][s] * corners[warp][it][s * 4 + corner].w;
-                        float *dst = gvb + off[b];
+                    for (int i = 0; i < kVec; ++i) t[b] = fmaf(v[i], g[i], t[b]);
+                    if (goff[b] >= 0 && chunk_ok) {
+                        float *dst = gvb + goff[b];
 #pragma unroll
                         for (int i = 0; i < kVec; i += 4)
-                            red_add_v4(dst + i, aw * g[i], aw * g[i + 1], aw * g[i + 2],
-                                       aw * g[i + 3]);
+                            red_add_v4(dst + i, aw[b] * g[i], aw[b] * g[i + 1], aw[b] * g[i + 2],
+                                       aw[b] * g[i + 3]);
                     }
                 }
                 // stage A: reduce t over the R chunk lanes (lane bits below R)
@@ -384,11 +451,11 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
                 for (int k = 0; k < kKeep; ++k) {
                     const int b = chunk * kKeep + k;
                     const int s = s0 + b * kSG + sg;
-                    CornerB e = {-1, 0.f, 0.f, 0.f};
-                    if (s < LK) e = corners[warp][it][s * 4 + corner];
-                    q[0][k] = e.w * t[k];
-                    q[1][k] = e.dwx * t[k];
-                    q[2][k] = e.dwy * t[k];
+                    float4 e = make_float4(0.f, 0.f, 0.f, 0.f);  // (w, dw/dfx, dw/dfy, -)
+                    if (s < LK) e = cDer[warp][it][corner * kStride + s];
+                    q[0][k] = e.x * t[k];
+                    q[1][k] = e.y * t[k];
+                    q[2][k] = e.z * t[k];
                 }
                 // stage B: sum over the four corner lanes of each sample
 #pragma unroll
@@ -436,13 +503,26 @@ cudaError_t launch_fast(BwdParams p, cudaStream_t stream)
     return cudaGetLastError();
 }
 
+// Samples per batch of the fast path (compile-time, per value type and R).
+template <typename VT, int R>
+constexpr int batch_samples()
+{
+    constexpr int kVec = Chunk<VT>::kVec;
+    constexpr int kB = (2 * R < 64 / kVec) ? 2 * R : 64 / kVec;
+    return kB * (8 / R);
+}
+
 template <typename VT, int R>
 cudaError_t launch_fast_r(const BwdParams &p, cudaStream_t stream)
 {
+    // P: a power of two >= L*K and >= the samples of one batch
+    constexpr int kBS = batch_samples<VT, R>();
     const int LK = p.L * p.K;
-    if (LK <= 4) return launch_fast<VT, R, 4>(p, stream);
-    if (LK <= 8) return launch_fast<VT, R, 8>(p, stream);
-    if (LK <= 16) return launch_fast<VT, R, 16>(p, stream);
+    const int need = LK > kBS ? LK : kBS;
+    if constexpr (kBS <= 8) {
+        if (need <= 8) return launch_fast<VT, R, 8>(p, stream);
+    }
+    if (need <= 16) return launch_fast<VT, R, 16>(p, stream);
     return launch_fast<VT, R, 32>(p, stream);
 }
 

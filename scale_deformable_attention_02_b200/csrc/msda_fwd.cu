@@ -35,10 +35,18 @@ namespace {
 
 constexpr int kWarps = 8;  // warps per CTA
 
-struct __align__(8) Corner {
-    int off;  // element offset of the corner row inside the (n, m) map; -1 = outside
-    float w;  // bilinear weight times the attention weight
+// One corner of one sample: the address of its row (already offset to the
+// batch entry and head, not yet to the lane's chunk) and its weight (bilinear
+// weight times attention weight) twice, as the operand pair of __ffma2_rn.
+// A corner outside the level points at kZeroRow with weight 0, so the gather
+// loop needs neither a predicate nor a bounds check.
+struct __align__(16) Corner {
+    const char *row;
+    float2 w;
 };
+
+// 512 bytes of zeros: the row that corners outside the level read.
+__device__ __align__(128) float4 kZeroRow[32] = {};
 
 template <int P>
 __device__ __forceinline__ float seg_max(float v)
@@ -56,28 +64,28 @@ __device__ __forceinline__ float seg_sum(float v)
     return v;
 }
 
-// One 16-byte chunk of a value row as kVec/2 float pairs.
+// One 16-byte chunk of a value row: loaded raw (4 registers), widened to
+// float pairs only when it is consumed, so a batch of loads in flight costs
+// the same registers for fp32 and bf16.
 template <typename VT>
 struct Pairs;
 
 template <>
 struct Pairs<float> {
-    static constexpr int kN = 2;
-    __device__ __forceinline__ static void load(const float *p, float2 (&v)[2])
+    static constexpr int kN = 2;  // float pairs per chunk
+    __device__ __forceinline__ static void widen(const uint4 &r, float2 (&v)[2])
     {
-        const float4 t = __ldg(reinterpret_cast<const float4 *>(p));
-        v[0] = make_float2(t.x, t.y);
-        v[1] = make_float2(t.z, t.w);
+        v[0] = make_float2(__uint_as_float(r.x), __uint_as_float(r.y));
+        v[1] = make_float2(__uint_as_float(r.z), __uint_as_float(r.w));
     }
 };
 
 template <>
 struct Pairs<__nv_bfloat16> {
     static constexpr int kN = 4;
-    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float2 (&v)[4])
+    __device__ __forceinline__ static void widen(const uint4 &r, float2 (&v)[4])
     {
-        const uint4 t = __ldg(reinterpret_cast<const uint4 *>(p));
-        const uint32_t w[4] = {t.x, t.y, t.z, t.w};
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i)  // exact widening: bf16 bits become the high half
             v[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
@@ -85,17 +93,23 @@ struct Pairs<__nv_bfloat16> {
 };
 
 template <typename VT, int R, int P, bool kFused, bool kExact>
-__global__ void __launch_bounds__(kWarps * 32, 2)
+__global__ void __launch_bounds__(kWarps * 32, 3)
     fwd_kernel(const __grid_constant__ FwdParams p)
 {
     constexpr int kNP = Pairs<VT>::kN;  // float pairs per 16-byte chunk
     constexpr int kSlots = 32 / R;      // (sample, corner) pairs per warp instruction
     constexpr int kItems = 32 / P;      // items per warp per round
     // gathers issued before the first is consumed (64 pairs = 16 samples)
-    // (at most 64 registers of loaded data: 16 fp32 chunks or 8 bf16 chunks)
-    constexpr int kB0 = (64 / kSlots) < 4 ? 4 : ((64 / kSlots) > 16 ? 16 : 64 / kSlots);
-    constexpr int kB = kB0 < 32 / kNP ? kB0 : 32 / kNP;
-    __shared__ Corner corners[kWarps][kItems][4 * P];
+    // (at most 16 raw 16-byte chunks, 64 registers)
+    constexpr int kB1 = (64 / kSlots) < 4 ? 4 : ((64 / kSlots) > 16 ? 16 : 64 / kSlots);
+    // a batch covers kB*kSlots pairs and must stay inside the 4*P entries
+    constexpr int kB = kB1 * kSlots <= 4 * P ? kB1 : (4 * P) / kSlots;
+    static_assert(kB >= 1 && (4 * P) % (kB * kSlots) == 0, "batch must tile the entries");
+    // Corner entries, corner-major with row stride P + 2 (= 2 mod 8): the
+    // phase-1 stores (consecutive samples) and the phase-2 loads (four
+    // corners of one or two samples) both fall in distinct banks.
+    constexpr int kStride = P + 2;
+    __shared__ Corner corners[kWarps][kItems][4 * kStride];
     __shared__ int sH[kMaxLevels], sW[kMaxLevels], sStart[kMaxLevels];
 
     const int tid = threadIdx.x;
@@ -163,11 +177,16 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
                 ly = t.y;
                 a = __ldcs(p.attn + si);
             }
-            if (j < LK) {  // items past the end get four "outside" entries
+            {  // every sample slot up to P gets four entries; unused ones read zeros
                 const int H = sH[l], W = sW[l], start = sStart[l];
+                const int m = (int)(item % M);
+                const int64_t n = item / M / p.Lq;
+                const char *mapb = static_cast<const char *>(p.value) +
+                                   ((n * p.S * M + m) * (int64_t)D) * (int64_t)sizeof(VT);
                 Corner c[4];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) c[q] = {-1, 0.f};
+                for (int q = 0; q < 4; ++q)
+                    c[q] = {reinterpret_cast<const char *>(kZeroRow), make_float2(0.f, 0.f)};
                 float x, y, fx, fy;
                 int x0, y0;
                 if (act && msda_cell(lx, ly, H, W, x, y, x0, y0, fx, fy)) {
@@ -176,12 +195,15 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         const int r = msda_row(start, H, W, y0 + (q >> 1), x0 + (q & 1));
-                        c[q].off = r < 0 ? -1 : r * MD;
-                        c[q].w = w[q] * a;
+                        if (r >= 0) {
+                            const float wa = w[q] * a;
+                            c[q] = {mapb + (int64_t)r * MD * (int64_t)sizeof(VT),
+                                    make_float2(wa, wa)};
+                        }
                     }
                 }
 #pragma unroll
-                for (int q = 0; q < 4; ++q) corners[warp][seg][j * 4 + q] = c[q];
+                for (int q = 0; q < 4; ++q) corners[warp][seg][q * kStride + j] = c[q];
             }
         }
         __syncwarp();
@@ -193,29 +215,32 @@ __global__ void __launch_bounds__(kWarps * 32, 2)
             if (item >= end) break;  // uniform across the warp
             const int m = (int)(item % M);
             const int64_t nq = item / M;
-            const int64_t n = nq / p.Lq;
-            const VT *vb = static_cast<const VT *>(p.value) + (n * p.S * M + m) * (int64_t)D +
-                           chunk * (2 * kNP);
+            // byte offset of this lane's chunk in a row; lanes past the last chunk
+            // (D*size not a power-of-two multiple of 16 bytes) re-read chunk 0 and
+            // their sums are discarded, so no lane reads past a row
+            const int lane_off = chunk_ok ? chunk * 16 : 0;
             float2 acc[kNP];
 #pragma unroll
             for (int i = 0; i < kNP; ++i) acc[i] = make_float2(0.f, 0.f);
+            const Corner *ent = corners[warp][it];
             for (int t0 = 0; t0 < npairs; t0 += kB * kSlots) {
-                float2 v[kB][kNP];
+                uint4 raw[kB];
                 float w[kB];
 #pragma unroll
                 for (int b = 0; b < kB; ++b) {
-                    const int t = t0 + b * kSlots + slot;
-                    const Corner e = t < npairs ? corners[warp][it][t] : Corner{-1, 0.f};
-                    w[b] = e.w;
-#pragma unroll
-                    for (int i = 0; i < kNP; ++i) v[b][i] = make_float2(0.f, 0.f);
-                    if (e.off >= 0 && chunk_ok) Pairs<VT>::load(vb + e.off, v[b]);
+                    const int t = t0 + b * kSlots + slot;  // pair t = (sample t/4, corner t%4)
+                    const Corner e = ent[(t & 3) * kStride + (t >> 2)];
+                    w[b] = e.w.x;
+                    raw[b] = __ldg(reinterpret_cast<const uint4 *>(e.row + lane_off));
                 }
 #pragma unroll
-                for (int b = 0; b < kB; ++b)
+                for (int b = 0; b < kB; ++b) {
+                    float2 v[kNP];
+                    Pairs<VT>::widen(raw[b], v);
+                    const float2 wb = make_float2(w[b], w[b]);
 #pragma unroll
-                    for (int i = 0; i < kNP; ++i)
-                        acc[i] = __ffma2_rn(make_float2(w[b], w[b]), v[b][i], acc[i]);
+                    for (int i = 0; i < kNP; ++i) acc[i] = __ffma2_rn(wb, v[i], acc[i]);
+                }
             }
             // combine the slots of each chunk, store the item's D outputs
 #pragma unroll
@@ -254,10 +279,15 @@ cudaError_t launch_p(FwdParams p, bool exact, cudaStream_t stream)
 template <typename VT, int R, bool kFused>
 cudaError_t launch_r(const FwdParams &p, bool exact, cudaStream_t stream)
 {
+    // P: lanes per item in phase 1, a power of two >= L*K, and at least the 8/R
+    // samples one warp instruction gathers, so a batch never leaves the entries
     const int LK = p.L * p.K;
-    if (LK <= 4) return launch_p<VT, R, 4, kFused>(p, exact, stream);
-    if (LK <= 8) return launch_p<VT, R, 8, kFused>(p, exact, stream);
-    if (LK <= 16) return launch_p<VT, R, 16, kFused>(p, exact, stream);
+    const int need = LK > 8 / R ? LK : 8 / R;
+    if constexpr (8 / R <= 4) {
+        if (need <= 4) return launch_p<VT, R, 4, kFused>(p, exact, stream);
+    }
+    if (need <= 8) return launch_p<VT, R, 8, kFused>(p, exact, stream);
+    if (need <= 16) return launch_p<VT, R, 16, kFused>(p, exact, stream);
     return launch_p<VT, R, 32, kFused>(p, exact, stream);
 }
 
