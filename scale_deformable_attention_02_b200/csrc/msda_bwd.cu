@@ -9,18 +9,17 @@
 //   dloc_x    = A * W * sum_j (dw_j/dfx) t_j,  dloc_y = A * H * sum_j (dw_j/dfy) t_j
 //   dvalue_j += A * w_j * g            (scatter; corners inside the level)
 //
-// Work decomposition (one warp per (n, q, m), as in the forward):
-//   1. Lane j < L*K finds sample j's cell and writes, per corner, the row
-//      offset, w_j, dw_j/dfx and dw_j/dfy to shared memory.
-//   2. SPAN = min(32, 4R) lanes work on one sample (R lanes per 16-byte-chunked
-//      row, one corner per R lanes), 32/SPAN samples at a time.  Each lane
-//      gathers its chunk of a corner row, forms its part of t_j, scatters
-//      A w_j g with one vector `red.global.add.v4.f32` per chunk, and keeps
-//      three running partial sums per sample.
-//   3. Every 8 samples per lane group the 24 partial sums are reduced across
-//      the SPAN lanes with a butterfly reduce-scatter (each step halves the
-//      values a lane holds), which costs about 4 shuffles per sample instead
-//      of 15, and the lanes holding finished sums write dA and dloc.
+// Two kernels:
+//   * bwd_kernel (value rows of at most 128 bytes): a group of R lanes owns
+//     whole samples and sums their four corners inside each lane, so only
+//     the R chunk lanes need combining (see its comment).  Persistent CTAs
+//     sweep contiguous item ranges.
+//   * bwd_kernel_wide (rows wider than 128 bytes): one warp per item; lane j
+//     finds sample j's cell and stores per-corner (row offset, w, dw/dfx,
+//     dw/dfy) in shared memory; min(32, 4R) lanes work on one sample, and the
+//     per-sample partial sums are reduced every 8 samples with a butterfly
+//     reduce-scatter.
+// Both scatter A w_j g with one vector `red.global.add.v4.f32` per 16 bytes.
 #include "msda_common.cuh"
 #include "msda_internal.h"
 
@@ -62,17 +61,7 @@ __device__ __forceinline__ void widen<__nv_bfloat16>(const uint4 &r, float (&v)[
     }
 }
 
-// Gather/scatter entry of one corner: its value row's address (already offset
-// to the batch entry and head), A*w, and the element offset of the matching
-// grad_value row inside the (n, m) map (-1: outside the level, nothing to
-// scatter).  Corners outside the level read kZeroRowB, so the gathers need no
-// predicate; only the scatter is predicated.
-struct __align__(16) CornerG {
-    const char *row;
-    float aw;
-    int goff;
-};
-
+// 512 bytes of zeros: the row that corners outside the level read.
 __device__ __align__(128) float4 kZeroRowB[32] = {};
 
 // Butterfly reduce-scatter over aligned groups of SPAN lanes.  Before: every
@@ -264,266 +253,225 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
 }
 
-// Fast path for rows of at most 128 bytes (R <= 8, so a warp instruction
-// covers 32/R >= 4 (sample, corner) pairs: kSG = 8/R samples of four corners).
-//   - Persistent CTAs sweep contiguous item ranges (L1 locality), a warp
-//     takes 32/P items per round and phase 1 gives every lane one sample.
-//   - Per item, 16 samples at a time (8 for bf16 rows of 128 bytes): all corner rows are loaded before any
-//     is used; each lane forms t = <v_chunk, g_chunk> and scatters
-//     A*w*g_chunk with a vector reduction.
-//   - The 16 partial t of a lane are reduced over the R chunk lanes with a
-//     butterfly reduce-scatter (each lane keeps two finished <v_c, g>), then
-//     weighted by (w, dw/dfx, dw/dfy) of its corner and summed over the four
-//     corner lanes with two xor steps: about 1.6 shuffles per sample.
-template <typename VT, int R, int P>
+// Fast path for value rows of at most 128 bytes (R <= 8 lanes per row).
+//
+// Lane layout as in the forward fast path: G = 32/R groups of R lanes, group g
+// owns samples g, g+G, ... of the item with all four corners, lane `chunk` owns
+// 16 bytes of every row.  Per sample a lane gathers the four corner chunks,
+// forms t_c = <v_c, g_chunk>, scatters A*w_c*g_chunk with a vector reduction
+// (corners inside the level only; outside corners read a zero row), and adds
+// w_c t_c, dw_c/dfx t_c, dw_c/dfy t_c into three per-sample partial sums.
+// The four corners are summed inside the lane, so only the R chunk lanes of a
+// group have to be combined: one butterfly reduce-scatter of all the item's
+// partial sums at the end.
+template <typename VT, int R, int NS, int NB>
 __global__ void __launch_bounds__(kWarps * 32, 2)
     bwd_kernel(const __grid_constant__ BwdParams p)
 {
-    static_assert(R <= 8, "fast path needs at least four pairs per instruction");
-    constexpr int kVec = Chunk<VT>::kVec;  // value elements per 16-byte chunk
-    constexpr int kSlots = 32 / R;         // pairs per warp instruction
-    constexpr int kSG = kSlots / 4;        // samples per warp instruction
-    // instructions per batch: 16 samples, or fewer if the loaded chunks would
-    // exceed 64 registers (bf16 with 128-byte rows: 8 samples)
-    constexpr int kB = (2 * R < 64 / kVec) ? 2 * R : 64 / kVec;
-    constexpr int kBS = kB * kSG;          // samples per batch
-    constexpr int kItems = 32 / P;
-    static_assert(kB % R == 0, "a batch must split evenly over the chunk lanes");
-    static_assert(kBS <= P && P % kBS == 0, "a batch must stay inside the P sample slots");
-    constexpr int kKeep = kB / R;          // finished <v_c, g> per lane after stage A
-
-    // Per corner: (row offset, A*w) for the gather/scatter loop and
-    // (w, dw/dfx, dw/dfy) for the reduction; corner-major with row stride
-    // P + 2 (= 2 mod 8) so that both phases are free of bank conflicts.
-    constexpr int kStride = P + 2;
-    __shared__ CornerG cOff[kWarps][kItems][4 * kStride];
-    __shared__ float4 cDer[kWarps][kItems][4 * kStride];
-    __shared__ float sA[kWarps][kItems][P];
-    __shared__ int sH[kMaxLevels], sW[kMaxLevels], sStart[kMaxLevels];
-
-    const int tid = threadIdx.x;
-    if (tid < p.L) {
-        sH[tid] = p.lv.H[tid];
-        sW[tid] = p.lv.W[tid];
-        sStart[tid] = p.lv.start[tid];
-    }
-    __syncthreads();
-
-    const int warp = tid >> 5;
-    const int lane = tid & 31;
+    static_assert(R <= 8 && NS * (32 / R) <= 32, "fast path shape");
+    constexpr int G = 32 / R;
+    constexpr int kVec = Chunk<VT>::kVec;
+    constexpr int kQ = 3 * NS;                           // partial sums per lane
+    constexpr int kCnt = (kQ + R - 1) / R * R;           // padded to the chunk lanes
+    constexpr int kPer = kCnt / R;                       // finished sums per lane
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = lane / R;
+    const int chunk = lane % R;
     const int M = p.M, D = p.D, K = p.K;
     const int LK = p.L * K;
     const int MD = M * D;
-    const int slot = lane / R;
-    const int chunk = lane % R;
-    const int corner = slot & 3;
-    const int sg = slot >> 2;
+    const int nsl = (LK + G - 1) / G;
     const bool chunk_ok = chunk < p.nchunks;
+    const int lane_off = chunk_ok ? chunk * 16 : 0;
+    const char *zrow = reinterpret_cast<const char *>(kZeroRowB) + lane_off;
+    const int64_t rowbytes = (int64_t)MD * (int64_t)sizeof(VT);
+
+    int lvW[NS], lvH[NS], lvS[NS];
+#pragma unroll
+    for (int i = 0; i < NS; ++i) {
+        const int s = g + G * i;
+        const int l = s < LK ? s / K : 0;
+        lvW[i] = p.lv.W[l];
+        lvH[i] = p.lv.H[l];
+        lvS[i] = p.lv.start[l];
+    }
 
     const int64_t begin = (int64_t)blockIdx.x * p.chunk;
     const int64_t end = begin + p.chunk < p.items ? begin + p.chunk : p.items;
+    for (int64_t item = begin + warp; item < end; item += kWarps) {
+        const int m = (int)(item % M);
+        const int64_t nq = item / M;
+        const int64_t n = nq / p.Lq;
+        const int64_t sbase = item * LK;
+        const int64_t mapoff = (n * p.S * M + m) * (int64_t)D;  // element offset of the (n, m) map
+        const char *mapb = static_cast<const char *>(p.value) + mapoff * (int64_t)sizeof(VT) +
+                           lane_off;
+        float *gmap = p.grad_value + mapoff + chunk * kVec;
 
-    for (int64_t item0 = begin + warp * kItems; item0 < end; item0 += kWarps * kItems) {
-        // ---- phase 1: cell and corner derivatives, one sample per lane ----
-        {
-            const int seg = lane / P;
-            const int j = lane % P;
-            const int64_t item = item0 + seg;
-            const bool act = j < LK && item < end;
-            {  // every sample slot up to P gets entries; unused ones read zeros
-                const int l = j < LK ? j / K : 0;
-                const int H = sH[l], W = sW[l], start = sStart[l];
-                const int m = (int)(item % M);
-                const int64_t n = item / M / p.Lq;
-                const char *mapb = static_cast<const char *>(p.value) +
-                                   ((n * p.S * M + m) * (int64_t)D) * (int64_t)sizeof(VT);
-                int off[4] = {-1, -1, -1, -1};
-                float w[4] = {0.f, 0.f, 0.f, 0.f};
-                float dwx[4] = {0.f, 0.f, 0.f, 0.f};
-                float dwy[4] = {0.f, 0.f, 0.f, 0.f};
-                float a = 0.f;
-                if (act) {
-                    const int64_t si = item * LK + j;
-                    const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
-                    a = __ldcs(p.attn + si);
-                    float x, y, fx, fy;
-                    int x0, y0;
-                    if (msda_cell(t.x, t.y, H, W, x, y, x0, y0, fx, fy)) {
-                        const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
-                        w[0] = hy * hx;
-                        w[1] = hy * fx;
-                        w[2] = fy * hx;
-                        w[3] = fy * fx;
-                        dwx[0] = -hy;
-                        dwx[1] = hy;
-                        dwx[2] = -fy;
-                        dwx[3] = fy;
-                        dwy[0] = -hx;
-                        dwy[1] = -fx;
-                        dwy[2] = hx;
-                        dwy[3] = fx;
+        float gv[kVec];
+        if (chunk_ok) {
+            const float4 *gp = reinterpret_cast<const float4 *>(
+                p.grad_out + nq * (int64_t)MD + m * D + chunk * kVec);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const int r = msda_row(start, H, W, y0 + (q >> 1), x0 + (q & 1));
-                            off[q] = r < 0 ? -1 : r * MD;
+            for (int i = 0; i < kVec / 4; ++i) {
+                const float4 t = __ldcs(gp + i);
+                gv[4 * i] = t.x;
+                gv[4 * i + 1] = t.y;
+                gv[4 * i + 2] = t.z;
+                gv[4 * i + 3] = t.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < kVec; ++i) gv[i] = 0.f;
+        }
+
+        float q[kCnt];  // [quantity * NS + slot]: dA, dfx, dfy partial sums
+        float aS[NS];   // attention weight of each slot's sample
+#pragma unroll
+        for (int i = 0; i < kCnt; ++i) q[i] = 0.f;
+#pragma unroll
+        for (int i = 0; i < NS; ++i) aS[i] = 0.f;
+
+#pragma unroll
+        for (int i0 = 0; i0 < NS; i0 += NB) {
+            if (i0 >= nsl) break;  // uniform
+            const char *ptr[NB][4];
+            int goff[NB][4];
+            float w[NB][4], dwx[NB][4], dwy[NB][4];
+#pragma unroll
+            for (int u = 0; u < NB; ++u) {
+                const int i = i0 + u;
+                const int s = g + G * i;
+                float lx = 0.f, ly = 0.f, a = 0.f;
+                if (s < LK) {
+                    const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + sbase + s);
+                    lx = t.x;
+                    ly = t.y;
+                    a = __ldcs(p.attn + sbase + s);
+                }
+                aS[i] = a;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    ptr[u][c] = zrow;
+                    goff[u][c] = -1;
+                    w[u][c] = dwx[u][c] = dwy[u][c] = 0.f;
+                }
+                float x, y, fx, fy;
+                int x0, y0;
+                if (s < LK && msda_cell(lx, ly, lvH[i], lvW[i], x, y, x0, y0, fx, fy)) {
+                    const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+                    w[u][0] = hy * hx;
+                    w[u][1] = hy * fx;
+                    w[u][2] = fy * hx;
+                    w[u][3] = fy * fx;
+                    dwx[u][0] = -hy;
+                    dwx[u][1] = hy;
+                    dwx[u][2] = -fy;
+                    dwx[u][3] = fy;
+                    dwy[u][0] = -hx;
+                    dwy[u][1] = -fx;
+                    dwy[u][2] = hx;
+                    dwy[u][3] = fx;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int r = msda_row(lvS[i], lvH[i], lvW[i], y0 + (c >> 1), x0 + (c & 1));
+                        if (r >= 0) {
+                            ptr[u][c] = mapb + (int64_t)r * rowbytes;
+                            goff[u][c] = r * MD;
                         }
                     }
                 }
-                sA[warp][seg][j] = a;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    CornerG g;
-                    g.row = off[q] >= 0 ? mapb + (int64_t)off[q] * (int64_t)sizeof(VT)
-                                        : reinterpret_cast<const char *>(kZeroRowB);
-                    g.aw = a * w[q];
-                    g.goff = off[q];
-                    cOff[warp][seg][q * kStride + j] = g;
-                    cDer[warp][seg][q * kStride + j] = make_float4(w[q], dwx[q], dwy[q], 0.f);
-                }
             }
-        }
-        __syncwarp();
-
-        // ---- phase 2: per item, 16 samples at a time ----------------------
-#pragma unroll 1
-        for (int it = 0; it < kItems; ++it) {
-            const int64_t item = item0 + it;
-            if (item >= end) break;  // uniform
-            const int m = (int)(item % M);
-            const int64_t nq = item / M;
-            const int64_t n = nq / p.Lq;
-            const int64_t sbase = item * LK;
-            float g[kVec];
-            if (chunk_ok) {
-                const float4 *gp = reinterpret_cast<const float4 *>(
-                    p.grad_out + nq * (int64_t)MD + m * D + chunk * kVec);
+            uint4 raw[NB][4];
 #pragma unroll
-                for (int i = 0; i < kVec / 4; ++i) {
-                    const float4 t = __ldcs(gp + i);
-                    g[4 * i] = t.x;
-                    g[4 * i + 1] = t.y;
-                    g[4 * i + 2] = t.z;
-                    g[4 * i + 3] = t.w;
-                }
-            } else {
+            for (int u = 0; u < NB; ++u)
 #pragma unroll
-                for (int i = 0; i < kVec; ++i) g[i] = 0.f;
-            }
-            const int64_t rowbase = (n * p.S * M + m) * (int64_t)D + chunk * kVec;
-            float *gvb = p.grad_value + rowbase;
-            // lanes past the last chunk re-read chunk 0 (their g is zero)
-            const int lane_off = chunk_ok ? chunk * 16 : 0;
-
-            for (int s0 = 0; s0 < LK; s0 += kBS) {
-                // loads: instruction b covers samples s0 + b*kSG + (0..kSG-1)
-                uint4 raw[kB];
-                float aw[kB];
-                int goff[kB];
+                for (int c = 0; c < 4; ++c) raw[u][c] = __ldg(reinterpret_cast<const uint4 *>(ptr[u][c]));
 #pragma unroll
-                for (int b = 0; b < kB; ++b) {
-                    const int s = s0 + b * kSG + sg;  // < P: every slot has an entry
-                    const CornerG e = cOff[warp][it][corner * kStride + s];
-                    raw[b] = __ldg(reinterpret_cast<const uint4 *>(e.row + lane_off));
-                    aw[b] = e.aw;
-                    goff[b] = e.goff;
-                }
-                float t[kB];
+            for (int u = 0; u < NB; ++u) {
+                const int i = i0 + u;
 #pragma unroll
-                for (int b = 0; b < kB; ++b) {
+                for (int c = 0; c < 4; ++c) {
                     float v[kVec];
-                    widen<VT>(raw[b], v);
-                    t[b] = 0.f;
+                    widen<VT>(raw[u][c], v);
+                    float t = 0.f;
 #pragma unroll
-                    for (int i = 0; i < kVec; ++i) t[b] = fmaf(v[i], g[i], t[b]);
-                    if (goff[b] >= 0 && chunk_ok) {
-                        float *dst = gvb + goff[b];
+                    for (int e = 0; e < kVec; ++e) t = fmaf(v[e], gv[e], t);
+                    q[i] = fmaf(w[u][c], t, q[i]);
+                    q[NS + i] = fmaf(dwx[u][c], t, q[NS + i]);
+                    q[2 * NS + i] = fmaf(dwy[u][c], t, q[2 * NS + i]);
+                    if (goff[u][c] >= 0 && chunk_ok) {
+                        const float aw = aS[i] * w[u][c];
+                        float *dst = gmap + goff[u][c];
 #pragma unroll
-                        for (int i = 0; i < kVec; i += 4)
-                            red_add_v4(dst + i, aw[b] * g[i], aw[b] * g[i + 1], aw[b] * g[i + 2],
-                                       aw[b] * g[i + 3]);
-                    }
-                }
-                // stage A: reduce t over the R chunk lanes (lane bits below R)
-                reduce_scatter_n<R, kB, kB>(t, lane);
-                // lane now holds <v_corner, g> of instructions b = chunk*kKeep + k
-                float q[3][kKeep];
-#pragma unroll
-                for (int k = 0; k < kKeep; ++k) {
-                    const int b = chunk * kKeep + k;
-                    const int s = s0 + b * kSG + sg;
-                    float4 e = make_float4(0.f, 0.f, 0.f, 0.f);  // (w, dw/dfx, dw/dfy, -)
-                    if (s < LK) e = cDer[warp][it][corner * kStride + s];
-                    q[0][k] = e.x * t[k];
-                    q[1][k] = e.y * t[k];
-                    q[2][k] = e.z * t[k];
-                }
-                // stage B: sum over the four corner lanes of each sample
-#pragma unroll
-                for (int o = R; o < 4 * R; o <<= 1)
-#pragma unroll
-                    for (int k = 0; k < kKeep; ++k) {
-                        q[0][k] += __shfl_xor_sync(kFull, q[0][k], o);
-                        q[1][k] += __shfl_xor_sync(kFull, q[1][k], o);
-                        q[2][k] += __shfl_xor_sync(kFull, q[2][k], o);
-                    }
-                if (corner == 0) {
-#pragma unroll
-                    for (int k = 0; k < kKeep; ++k) {
-                        const int b = chunk * kKeep + k;
-                        const int s = s0 + b * kSG + sg;
-                        if (s < LK) {
-                            const int64_t si = sbase + s;
-                            if (p.grad_attn) __stcs(p.grad_attn + si, q[0][k]);
-                            if (p.grad_loc) {
-                                const int l = s / K;
-                                const float a = sA[warp][it][s];
-                                __stcs(reinterpret_cast<float2 *>(p.grad_loc) + si,
-                                       make_float2(a * ((float)sW[l] * q[1][k]),
-                                                   a * ((float)sH[l] * q[2][k])));
-                            }
-                        }
+                        for (int e = 0; e < kVec; e += 4)
+                            red_add_v4(dst + e, aw * gv[e], aw * gv[e + 1], aw * gv[e + 2],
+                                       aw * gv[e + 3]);
                     }
                 }
             }
         }
-        __syncwarp();
+
+        // combine the R chunk lanes of each group: lane `chunk` ends with the
+        // totals of partial sums chunk*kPer ... chunk*kPer + kPer - 1
+        reduce_scatter_n<R, kCnt, kCnt>(q, lane);
+#pragma unroll
+        for (int k = 0; k < kPer; ++k) {
+            const int idx = chunk * kPer + k;
+            const int qty = idx / NS;
+            const int i = idx % NS;
+            const int s = g + G * i;
+            if (qty < 3 && s < LK) {
+                const int64_t si = sbase + s;
+                if (qty == 0) {
+                    if (p.grad_attn) __stcs(p.grad_attn + si, q[k]);
+                } else if (p.grad_loc) {
+                    // the slot's level: every lane holds lvW/lvH for all its slots
+                    float scale = 0.f, a = 0.f;
+#pragma unroll
+                    for (int jj = 0; jj < NS; ++jj)
+                        if (jj == i) {
+                            scale = (qty == 1) ? (float)lvW[jj] : (float)lvH[jj];
+                            a = aS[jj];
+                        }
+                    __stcs(p.grad_loc + 2 * si + (qty - 1), a * (scale * q[k]));
+                }
+            }
+        }
     }
 }
 
-template <typename VT, int R, int P>
+template <typename VT, int R, int NS>
 cudaError_t launch_fast(BwdParams p, cudaStream_t stream)
 {
-    constexpr int kRound = kWarps * (32 / P);
-    auto kern = bwd_kernel<VT, R, P>;
-    const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kRound);
+    constexpr int NB = NS < 2 ? NS : 2;
+    auto kern = bwd_kernel<VT, R, NS, NB>;
+    const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kWarps);
     p.chunk = (p.items + ctas - 1) / ctas;
-    p.chunk = (p.chunk + kRound - 1) / kRound * kRound;
+    p.chunk = (p.chunk + kWarps - 1) / kWarps * kWarps;
     const dim3 grid((unsigned)((p.items + p.chunk - 1) / p.chunk));
     kern<<<grid, kWarps * 32, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
-// Samples per batch of the fast path (compile-time, per value type and R).
-template <typename VT, int R>
-constexpr int batch_samples()
-{
-    constexpr int kVec = Chunk<VT>::kVec;
-    constexpr int kB = (2 * R < 64 / kVec) ? 2 * R : 64 / kVec;
-    return kB * (8 / R);
-}
-
 template <typename VT, int R>
 cudaError_t launch_fast_r(const BwdParams &p, cudaStream_t stream)
 {
-    // P: a power of two >= L*K and >= the samples of one batch
-    constexpr int kBS = batch_samples<VT, R>();
+    constexpr int G = 32 / R;
     const int LK = p.L * p.K;
-    const int need = LK > kBS ? LK : kBS;
-    if constexpr (kBS <= 8) {
-        if (need <= 8) return launch_fast<VT, R, 8>(p, stream);
+    const int nsl = (LK + G - 1) / G;
+    if (nsl <= 1) return launch_fast<VT, R, 1>(p, stream);
+    if constexpr (G <= 16) {
+        if (nsl <= 2) return launch_fast<VT, R, 2>(p, stream);
     }
-    if (need <= 16) return launch_fast<VT, R, 16>(p, stream);
-    return launch_fast<VT, R, 32>(p, stream);
+    if constexpr (G <= 8) {
+        if (nsl <= 4) return launch_fast<VT, R, 4>(p, stream);
+    }
+    if constexpr (G <= 4) {
+        return launch_fast<VT, R, 8>(p, stream);
+    }
+    return cudaErrorInvalidValue;  // not reached: L*K <= 32
 }
 
 template <typename VT>

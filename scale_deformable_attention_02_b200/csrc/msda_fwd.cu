@@ -4,24 +4,21 @@
 // page, "Multi-scale deformable attention" equation):
 //   out[n,q,m,:] = sum_{l,k} A[n,q,m,l,k] * bilinear(value[n, level l, m, :], loc)
 //
-// Work decomposition.  An "item" is one (n, q, m); it has L*K samples.  A warp
-// owns 32/P consecutive items, where P = max(4, next power of two >= L*K) is
-// the number of lanes given to one item in phase 1.
-//   1. Every lane owns one sample (lane j of an item's P-lane segment owns
-//      sample j).  It reads the sample's location and weight -- or, fused,
-//      forms them: the joint softmax over the item's L*K logits runs inside
-//      the P-lane segment with xor shuffles, and the location map is an IEEE
-//      divide and add -- finds the cell and writes four corner entries
-//      (row offset, attention weight x bilinear weight) to shared memory.
-//   2. The warp walks the 4*L*K (sample, corner) pairs of its items together.
-//      A (pixel, head) row of D elements is split into 16-byte chunks; R lanes
-//      cover one row and 32/R rows are gathered per warp instruction, so every
-//      corner read is a coalesced 16-byte-per-lane load of whole rows (fp32,
-//      D = 32: 8 lanes x 16 B, the four corners of a sample in one
-//      instruction; bf16, D = 32: 4 lanes, two samples per instruction).
-//      Lanes accumulate their chunk in fp32 with packed FMA (`__ffma2_rn`).
-//   3. Xor shuffles combine the 32/R partial sums of a chunk, and lanes
-//      0..R-1 store each item's D outputs.
+// An "item" is one (n, q, m); it has L*K samples, each with four corner rows of
+// D elements.  A (pixel, head) row is split into 16-byte chunks and R lanes
+// cover one row, so a warp instruction gathers 32/R whole rows with 16 bytes
+// per lane (fp32, D = 32: R = 8; bf16, D = 32: R = 4); lanes accumulate their
+// chunk in fp32 with packed FMA (`__ffma2_rn`).  Two kernels:
+//   * fwd_kernel (rows of at most 128 bytes): a group of R lanes owns whole
+//     samples; every lane forms its corner addresses and weights in registers
+//     (see its comment).
+//   * fwd_kernel_wide (wider rows): lane j of an item's P-lane segment forms
+//     sample j's cell and writes four (row address, weight) entries to shared
+//     memory; the warp then walks the (sample, corner) pairs.
+// Both run persistent CTAs that sweep contiguous item ranges (neighbouring
+// queries sample neighbouring pixels, so rows are reused from L1), issue a
+// batch of gathers before consuming any, and send corners outside the level
+// to a zero row instead of branching.
 // Single-use data (locations, weights, logits, offsets, outputs) is read and
 // written with evict-first hints so that the value map, which every sample
 // gathers from, keeps the L2.  The gather is the whole cost ("Deformable
@@ -94,7 +91,7 @@ struct Pairs<__nv_bfloat16> {
 
 template <typename VT, int R, int P, bool kFused, bool kExact>
 __global__ void __launch_bounds__(kWarps * 32, 3)
-    fwd_kernel(const __grid_constant__ FwdParams p)
+    fwd_kernel_wide(const __grid_constant__ FwdParams p)
 {
     constexpr int kNP = Pairs<VT>::kN;  // float pairs per 16-byte chunk
     constexpr int kSlots = 32 / R;      // (sample, corner) pairs per warp instruction
@@ -263,11 +260,209 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Fast path for value rows of at most 128 bytes (R <= 8 lanes per row).
+//
+// Lane layout: G = 32/R groups of R lanes; group g owns samples g, g+G, g+2G,
+// ... of the item (all four corners of each), lane `chunk` of the group owns
+// 16 bytes of every row.  So every lane forms the row addresses and weights
+// it gathers with in its own registers -- no shared-memory entries -- and a
+// warp instruction still gathers G whole rows, 16 bytes per lane.  The
+// per-level metadata of a lane's sample slots is the same for every item and
+// is read once.  Fused: lane j first forms sample j's location and attention
+// weight (one IEEE divide per coordinate, one softmax per item), and the
+// group lanes fetch them with three shuffles.
+// ---------------------------------------------------------------------------
+template <typename VT, int R, int NS, int NB, bool kFused>
+__global__ void __launch_bounds__(kWarps * 32, 3)
+    fwd_kernel(const __grid_constant__ FwdParams p)
+{
+    static_assert(R <= 8 && NS * (32 / R) <= 32, "fast path shape");
+    constexpr int G = 32 / R;           // samples gathered per warp instruction
+    constexpr int kNP = Pairs<VT>::kN;  // float pairs per 16-byte chunk
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = lane / R;
+    const int chunk = lane % R;
+    const int M = p.M, D = p.D, K = p.K;
+    const int LK = p.L * K;
+    const int MD = M * D;
+    const int nsl = (LK + G - 1) / G;  // sample slots in use, <= NS
+    const bool chunk_ok = chunk < p.nchunks;
+    // lanes past the last chunk of a row re-read chunk 0; their sums are discarded
+    const int lane_off = chunk_ok ? chunk * 16 : 0;
+    const char *zrow = reinterpret_cast<const char *>(kZeroRow) + lane_off;
+    const int64_t rowbytes = (int64_t)MD * (int64_t)sizeof(VT);
+
+    int lvW[NS], lvH[NS], lvS[NS];  // level of sample slot i (sample g + G*i)
+#pragma unroll
+    for (int i = 0; i < NS; ++i) {
+        const int s = g + G * i;
+        const int l = s < LK ? s / K : 0;
+        lvW[i] = p.lv.W[l];
+        lvH[i] = p.lv.H[l];
+        lvS[i] = p.lv.start[l];
+    }
+
+    const int64_t begin = (int64_t)blockIdx.x * p.chunk;
+    const int64_t end = begin + p.chunk < p.items ? begin + p.chunk : p.items;
+    for (int64_t item = begin + warp; item < end; item += kWarps) {
+        const int m = (int)(item % M);
+        const int64_t nq = item / M;
+        const int64_t n = nq / p.Lq;
+        const int64_t sbase = item * LK;
+        const char *mapb = static_cast<const char *>(p.value) +
+                           (n * p.S * M + m) * (int64_t)D * (int64_t)sizeof(VT) + lane_off;
+
+        float ax = 0.f, ay = 0.f, aa = 0.f;  // fused: sample `lane`'s location and weight
+        if constexpr (kFused) {
+            const bool act = lane < LK;
+            const float z = act ? __ldcs(p.logits + sbase + lane) : -INFINITY;
+            const float mx = warp_max(z);
+            const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
+            const float sum = warp_sum(e);
+            aa = __fdiv_rn(e, sum);
+            if (act) {
+                const int l = lane / K;
+                const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sbase + lane);
+                if (p.ref_dim == 2) {
+                    // point reference: offsets are level-l pixels
+                    const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
+                    ax = __fadd_rn(r.x, __fdiv_rn(o.x, (float)p.lv.W[l]));
+                    ay = __fadd_rn(r.y, __fdiv_rn(o.y, (float)p.lv.H[l]));
+                } else {
+                    // box reference (cx, cy, w, h): offsets are in box units
+                    const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
+                    const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
+                    ax = __fadd_rn(c.x, __fmul_rn(o.x, s2.x));
+                    ay = __fadd_rn(c.y, __fmul_rn(o.y, s2.y));
+                }
+                if (p.loc_out)
+                    __stcs(reinterpret_cast<float2 *>(p.loc_out) + sbase + lane,
+                           make_float2(ax, ay));
+                if (p.attn_out) __stcs(p.attn_out + sbase + lane, aa);
+            }
+        }
+
+        float2 acc[kNP];
+#pragma unroll
+        for (int i = 0; i < kNP; ++i) acc[i] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int i0 = 0; i0 < NS; i0 += NB) {
+            if (i0 >= nsl) break;  // uniform across the warp
+            const char *ptr[NB][4];
+            float wt[NB][4];
+#pragma unroll
+            for (int u = 0; u < NB; ++u) {
+                const int i = i0 + u;
+                const int s = g + G * i;  // < 32
+                const bool have = s < LK;
+                float lx = 0.f, ly = 0.f, a = 0.f;
+                if constexpr (kFused) {
+                    lx = __shfl_sync(kFull, ax, s);
+                    ly = __shfl_sync(kFull, ay, s);
+                    a = __shfl_sync(kFull, aa, s);
+                } else if (have) {
+                    const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + sbase + s);
+                    lx = t.x;
+                    ly = t.y;
+                    a = __ldcs(p.attn + sbase + s);
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    ptr[u][c] = zrow;
+                    wt[u][c] = 0.f;
+                }
+                float x, y, fx, fy;
+                int x0, y0;
+                if (have && msda_cell(lx, ly, lvH[i], lvW[i], x, y, x0, y0, fx, fy)) {
+                    const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+                    const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int r = msda_row(lvS[i], lvH[i], lvW[i], y0 + (c >> 1), x0 + (c & 1));
+                        if (r >= 0) {
+                            ptr[u][c] = mapb + (int64_t)r * rowbytes;
+                            wt[u][c] = w[c] * a;
+                        }
+                    }
+                }
+            }
+            uint4 raw[NB][4];
+#pragma unroll
+            for (int u = 0; u < NB; ++u)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) raw[u][c] = __ldg(reinterpret_cast<const uint4 *>(ptr[u][c]));
+#pragma unroll
+            for (int u = 0; u < NB; ++u)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    float2 v[kNP];
+                    Pairs<VT>::widen(raw[u][c], v);
+                    const float2 wb = make_float2(wt[u][c], wt[u][c]);
+#pragma unroll
+                    for (int i = 0; i < kNP; ++i) acc[i] = __ffma2_rn(wb, v[i], acc[i]);
+                }
+        }
+
+        // sum over the G groups, then lanes 0..R-1 store the item's D outputs
+#pragma unroll
+        for (int o = R; o < 32; o <<= 1)
+#pragma unroll
+            for (int i = 0; i < kNP; ++i) {
+                acc[i].x += __shfl_xor_sync(kFull, acc[i].x, o);
+                acc[i].y += __shfl_xor_sync(kFull, acc[i].y, o);
+            }
+        if (g == 0 && chunk_ok) {
+            float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D +
+                                                     chunk * (2 * kNP));
+#pragma unroll
+            for (int i = 0; i < kNP / 2; ++i)
+                __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
+                                            acc[2 * i + 1].y));
+        }
+    }
+}
+
+template <typename VT, int R, int NS, bool kFused>
+cudaError_t launch_fast(FwdParams p, cudaStream_t stream)
+{
+    constexpr int NB = NS < 2 ? NS : 2;  // sample slots gathered per batch (4 rows each)
+    auto kern = fwd_kernel<VT, R, NS, NB, kFused>;
+    const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kWarps);
+    p.chunk = (p.items + ctas - 1) / ctas;
+    p.chunk = (p.chunk + kWarps - 1) / kWarps * kWarps;
+    const dim3 grid((unsigned)((p.items + p.chunk - 1) / p.chunk));
+    kern<<<grid, kWarps * 32, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+template <typename VT, int R, bool kFused>
+cudaError_t launch_fast_r(const FwdParams &p, cudaStream_t stream)
+{
+    constexpr int G = 32 / R;
+    const int LK = p.L * p.K;
+    const int nsl = (LK + G - 1) / G;  // sample slots per lane
+    if (nsl <= 1) return launch_fast<VT, R, 1, kFused>(p, stream);
+    if constexpr (G <= 16) {
+        if (nsl <= 2) return launch_fast<VT, R, 2, kFused>(p, stream);
+    }
+    if constexpr (G <= 8) {
+        if (nsl <= 4) return launch_fast<VT, R, 4, kFused>(p, stream);
+    }
+    if constexpr (G <= 4) {
+        return launch_fast<VT, R, 8, kFused>(p, stream);
+    }
+    return cudaErrorInvalidValue;  // not reached: L*K <= 32
+}
+
+
 template <typename VT, int R, int P, bool kFused>
 cudaError_t launch_p(FwdParams p, bool exact, cudaStream_t stream)
 {
     constexpr int kRound = kWarps * (32 / P);  // items per CTA round
-    auto kern = exact ? fwd_kernel<VT, R, P, kFused, true> : fwd_kernel<VT, R, P, kFused, false>;
+    auto kern = exact ? fwd_kernel_wide<VT, R, P, kFused, true>
+                      : fwd_kernel_wide<VT, R, P, kFused, false>;
     const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kRound);
     p.chunk = (p.items + ctas - 1) / ctas;
     p.chunk = (p.chunk + kRound - 1) / kRound * kRound;
@@ -296,10 +491,10 @@ cudaError_t launch_fwd_vt(const FwdParams &p, int R, cudaStream_t stream)
 {
     const bool exact = p.nchunks == R;
     switch (R) {
-    case 1: return launch_r<VT, 1, kFused>(p, exact, stream);
-    case 2: return launch_r<VT, 2, kFused>(p, exact, stream);
-    case 4: return launch_r<VT, 4, kFused>(p, exact, stream);
-    case 8: return launch_r<VT, 8, kFused>(p, exact, stream);
+    case 1: return launch_fast_r<VT, 1, kFused>(p, stream);
+    case 2: return launch_fast_r<VT, 2, kFused>(p, stream);
+    case 4: return launch_fast_r<VT, 4, kFused>(p, stream);
+    case 8: return launch_fast_r<VT, 8, kFused>(p, stream);
     case 16: return launch_r<VT, 16, kFused>(p, exact, stream);
     case 32: return launch_r<VT, 32, kFused>(p, exact, stream);
     default: return cudaErrorInvalidValue;
