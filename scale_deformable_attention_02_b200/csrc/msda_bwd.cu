@@ -253,237 +253,274 @@ __global__ void __launch_bounds__(kWarps * 32)
     }
 }
 
-// Fast path for value rows of at most 128 bytes (R <= 8 lanes per row).
+// Four consecutive value elements of one lane, widened to fp32: a 16-byte
+// load for fp32, an 8-byte load for bf16.  The backward's fast path gives
+// every lane four elements so that R = D/4 lanes cover a row of the fp32
+// gradient and one vector reduction instruction updates whole 128-byte
+// gradient rows, whatever the value dtype.
+template <typename VT>
+struct Lane4;
+
+template <>
+struct Lane4<float> {
+    using Raw = uint4;
+    __device__ __forceinline__ static Raw load(const float *p)
+    {
+        return __ldg(reinterpret_cast<const uint4 *>(p));
+    }
+    __device__ __forceinline__ static void widen(const Raw &r, float (&v)[4])
+    {
+        v[0] = __uint_as_float(r.x);
+        v[1] = __uint_as_float(r.y);
+        v[2] = __uint_as_float(r.z);
+        v[3] = __uint_as_float(r.w);
+    }
+};
+
+template <>
+struct Lane4<__nv_bfloat16> {
+    using Raw = uint2;
+    __device__ __forceinline__ static Raw load(const __nv_bfloat16 *p)
+    {
+        return __ldg(reinterpret_cast<const uint2 *>(p));
+    }
+    __device__ __forceinline__ static void widen(const Raw &r, float (&v)[4])
+    {
+        v[0] = __uint_as_float(r.x << 16);
+        v[1] = __uint_as_float(r.x & 0xffff0000u);
+        v[2] = __uint_as_float(r.y << 16);
+        v[3] = __uint_as_float(r.y & 0xffff0000u);
+    }
+};
+
+// Fast path for D <= 32 (R = D/4 <= 8 lanes per row, four elements per lane).
 //
-// Lane layout as in the forward fast path: G = 32/R groups of R lanes, group g
-// owns samples g, g+G, ... of the item with all four corners, lane `chunk` owns
-// 16 bytes of every row.  Per sample a lane gathers the four corner chunks,
-// forms t_c = <v_c, g_chunk>, scatters A*w_c*g_chunk with a vector reduction
-// (corners inside the level only; outside corners read a zero row), and adds
-// w_c t_c, dw_c/dfx t_c, dw_c/dfy t_c into three per-sample partial sums.
-// The four corners are summed inside the lane, so only the R chunk lanes of a
-// group have to be combined: one butterfly reduce-scatter of all the item's
-// partial sums at the end.
-template <typename VT, int R, int NS, int NB>
-__global__ void __launch_bounds__(kWarps * 32, 2)
+// The scatter into grad_value is bound by the L2's atomic throughput (a flat
+// cost per 128-byte row), the gathers by how many rows the L2 returns per
+// second; both want many warps per SM, so the footprint stays small:
+//   * a warp loops over rounds of 32/P items; lane j of an item's P-lane
+//     segment owns sample j (level metadata in registers for the whole
+//     kernel) and loads the next round's location and weight while the
+//     current round gathers;
+//   * phase 1 stores, per corner, an 8-byte (row offset | -1, A*w) entry
+//     (corner-major, stride P + 2: no bank conflicts) and, per sample,
+//     (fx, fy, A*W, A*H);
+//   * phase 2 takes R instructions at a time (each gathers 32/R corner rows,
+//     16 bytes per lane), forms t = <v_chunk, g_chunk>, scatters A*w*g_chunk
+//     with a vector reduction, reduces t over the R chunk lanes with a
+//     butterfly reduce-scatter, weights it with (w, dw/dfx, dw/dfy) of its
+//     corner and sums the four corner lanes with two xor steps.
+#ifndef MSDA_BWD_MIN_CTAS
+#define MSDA_BWD_MIN_CTAS 3
+#endif
+
+template <typename VT, int R, int P>
+__global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
     bwd_kernel(const __grid_constant__ BwdParams p)
 {
-    static_assert(R <= 8 && NS * (32 / R) <= 32, "fast path shape");
-    constexpr int G = 32 / R;
-    constexpr int kVec = Chunk<VT>::kVec;
-    constexpr int kQ = 3 * NS;                           // partial sums per lane
-    constexpr int kCnt = (kQ + R - 1) / R * R;           // padded to the chunk lanes
-    constexpr int kPer = kCnt / R;                       // finished sums per lane
+    static_assert(R <= 8, "fast path: at least four pairs per warp instruction");
+    constexpr int kVec = 4;                // value elements per lane
+    using Raw = typename Lane4<VT>::Raw;
+    constexpr int kSlots = 32 / R;         // pairs per warp instruction
+    constexpr int kSG = kSlots / 4;        // samples per warp instruction
+    constexpr int kB = R;                  // instructions per batch: one t per lane after stage A
+    constexpr int kBS = kB * kSG;          // samples per batch (= 8)
+    constexpr int kItems = 32 / P;
+    constexpr int kStride = P + 2;
+    static_assert(kBS <= P && P % kBS == 0, "a batch must stay inside the P sample slots");
+    __shared__ int2 ent[kWarps][kItems][4 * kStride];  // (row element offset | -1, A*w)
+    __shared__ float4 smp[kWarps][kItems][P];          // (fx, fy, A*W, A*H)
+
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int g = lane / R;
-    const int chunk = lane % R;
     const int M = p.M, D = p.D, K = p.K;
     const int LK = p.L * K;
     const int MD = M * D;
-    const int nsl = (LK + G - 1) / G;
+
+    const int seg = lane / P;
+    const int j = lane % P;
+    const bool jact = j < LK;
+    const int lvl = jact ? j / K : 0;
+    const int H = p.lv.H[lvl], W = p.lv.W[lvl], start = p.lv.start[lvl];
+
+    const int slot = lane / R;
+    const int chunk = lane % R;
+    const int corner = slot & 3;
+    const int sg = slot >> 2;
     const bool chunk_ok = chunk < p.nchunks;
-    const int lane_off = chunk_ok ? chunk * 16 : 0;
-    const char *zrow = reinterpret_cast<const char *>(kZeroRowB) + lane_off;
-    const int64_t rowbytes = (int64_t)MD * (int64_t)sizeof(VT);
+    const int lane_elem = (chunk_ok ? chunk : 0) * kVec;
+    const bool cx = corner & 1, cy = corner >> 1;
 
-    int lvW[NS], lvH[NS], lvS[NS];
-#pragma unroll
-    for (int i = 0; i < NS; ++i) {
-        const int s = g + G * i;
-        const int l = s < LK ? s / K : 0;
-        lvW[i] = p.lv.W[l];
-        lvH[i] = p.lv.H[l];
-        lvS[i] = p.lv.start[l];
-    }
+    const int64_t stride = (int64_t)gridDim.x * kWarps * kItems;
+    int64_t item0 = ((int64_t)blockIdx.x * kWarps + warp) * kItems;
 
-    const int64_t begin = (int64_t)blockIdx.x * p.chunk;
-    const int64_t end = begin + p.chunk < p.items ? begin + p.chunk : p.items;
-    for (int64_t item = begin + warp; item < end; item += kWarps) {
-        const int m = (int)(item % M);
-        const int64_t nq = item / M;
-        const int64_t n = nq / p.Lq;
-        const int64_t sbase = item * LK;
-        const int64_t mapoff = (n * p.S * M + m) * (int64_t)D;  // element offset of the (n, m) map
-        const char *mapb = static_cast<const char *>(p.value) + mapoff * (int64_t)sizeof(VT) +
-                           lane_off;
-        float *gmap = p.grad_value + mapoff + chunk * kVec;
-
-        float gv[kVec];
-        if (chunk_ok) {
-            const float4 *gp = reinterpret_cast<const float4 *>(
-                p.grad_out + nq * (int64_t)MD + m * D + chunk * kVec);
-#pragma unroll
-            for (int i = 0; i < kVec / 4; ++i) {
-                const float4 t = __ldcs(gp + i);
-                gv[4 * i] = t.x;
-                gv[4 * i + 1] = t.y;
-                gv[4 * i + 2] = t.z;
-                gv[4 * i + 3] = t.w;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < kVec; ++i) gv[i] = 0.f;
+    float pl_x = 0.f, pl_y = 0.f, pa = 0.f;
+    auto fetch = [&](int64_t i0) {
+        const int64_t item = i0 + seg;
+        pl_x = pl_y = pa = 0.f;
+        if (jact && item < p.items) {
+            const int64_t si = item * LK + j;
+            const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
+            pl_x = t.x;
+            pl_y = t.y;
+            pa = __ldcs(p.attn + si);
         }
+    };
+    fetch(item0);
 
-        float q[kCnt];  // [quantity * NS + slot]: dA, dfx, dfy partial sums
-        float aS[NS];   // attention weight of each slot's sample
-#pragma unroll
-        for (int i = 0; i < kCnt; ++i) q[i] = 0.f;
-#pragma unroll
-        for (int i = 0; i < NS; ++i) aS[i] = 0.f;
-
-#pragma unroll
-        for (int i0 = 0; i0 < NS; i0 += NB) {
-            if (i0 >= nsl) break;  // uniform
-            const char *ptr[NB][4];
-            int goff[NB][4];
-            float w[NB][4], dwx[NB][4], dwy[NB][4];
-#pragma unroll
-            for (int u = 0; u < NB; ++u) {
-                const int i = i0 + u;
-                const int s = g + G * i;
-                float lx = 0.f, ly = 0.f, a = 0.f;
-                if (s < LK) {
-                    const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + sbase + s);
-                    lx = t.x;
-                    ly = t.y;
-                    a = __ldcs(p.attn + sbase + s);
-                }
-                aS[i] = a;
+    for (; item0 < p.items; item0 += stride) {
+        // ---- phase 1 -------------------------------------------------------
+        {
+            const int64_t item = item0 + seg;
+            const bool act = jact && item < p.items;
+            const float lx = pl_x, ly = pl_y, a = pa;
+            fetch(item0 + stride);
+            int2 e[4] = {{-1, 0}, {-1, 0}, {-1, 0}, {-1, 0}};
+            float4 rec = make_float4(0.f, 0.f, 0.f, 0.f);
+            float x, y, fx, fy;
+            int x0, y0;
+            if (act && msda_cell(lx, ly, H, W, x, y, x0, y0, fx, fy)) {
+                const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+                const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    ptr[u][c] = zrow;
-                    goff[u][c] = -1;
-                    w[u][c] = dwx[u][c] = dwy[u][c] = 0.f;
+                    const int r = msda_row(start, H, W, y0 + (c >> 1), x0 + (c & 1));
+                    if (r >= 0) e[c] = make_int2(r * MD, __float_as_int(a * w[c]));
                 }
-                float x, y, fx, fy;
-                int x0, y0;
-                if (s < LK && msda_cell(lx, ly, lvH[i], lvW[i], x, y, x0, y0, fx, fy)) {
-                    const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
-                    w[u][0] = hy * hx;
-                    w[u][1] = hy * fx;
-                    w[u][2] = fy * hx;
-                    w[u][3] = fy * fx;
-                    dwx[u][0] = -hy;
-                    dwx[u][1] = hy;
-                    dwx[u][2] = -fy;
-                    dwx[u][3] = fy;
-                    dwy[u][0] = -hx;
-                    dwy[u][1] = -fx;
-                    dwy[u][2] = hx;
-                    dwy[u][3] = fx;
+                rec = make_float4(fx, fy, a * (float)W, a * (float)H);
+            }
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int r = msda_row(lvS[i], lvH[i], lvW[i], y0 + (c >> 1), x0 + (c & 1));
-                        if (r >= 0) {
-                            ptr[u][c] = mapb + (int64_t)r * rowbytes;
-                            goff[u][c] = r * MD;
+            for (int c = 0; c < 4; ++c) ent[warp][seg][c * kStride + j] = e[c];
+            smp[warp][seg][j] = rec;
+        }
+        __syncwarp();
+
+        // ---- phase 2 -------------------------------------------------------
+#pragma unroll 1
+        for (int it = 0; it < kItems; ++it) {
+            const int64_t itm = item0 + it;
+            if (itm >= p.items) break;  // uniform
+            const int m = (int)(itm % M);
+            const int64_t nq = itm / M;
+            const int64_t n = nq / p.Lq;
+            const int64_t sbase = itm * LK;
+            const int64_t mapoff = (n * p.S * M + m) * (int64_t)D;
+            const VT *vb = static_cast<const VT *>(p.value) + mapoff + lane_elem;
+            float *gvb = p.grad_value + mapoff + chunk * kVec;
+            float gv[kVec];
+            if (chunk_ok) {
+                const float4 *gp = reinterpret_cast<const float4 *>(
+                    p.grad_out + nq * (int64_t)MD + m * D + chunk * kVec);
+#pragma unroll
+                for (int i = 0; i < kVec / 4; ++i) {
+                    const float4 t = __ldcs(gp + i);
+                    gv[4 * i] = t.x;
+                    gv[4 * i + 1] = t.y;
+                    gv[4 * i + 2] = t.z;
+                    gv[4 * i + 3] = t.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < kVec; ++i) gv[i] = 0.f;
+            }
+            const int2 *en = ent[warp][it] + corner * kStride + sg;
+            for (int s0 = 0; s0 < LK; s0 += kBS) {
+                int2 e[kB];
+                Raw raw[kB];
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    e[b] = en[s0 + b * kSG];  // sample s0 + b*kSG + sg, this lane's corner
+                    if (e[b].x >= 0) raw[b] = Lane4<VT>::load(vb + e[b].x);
+                }
+                float t[kB];
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    t[b] = 0.f;
+                    if (e[b].x >= 0) {
+                        float v[kVec];
+                        Lane4<VT>::widen(raw[b], v);
+#pragma unroll
+                        for (int i = 0; i < kVec; ++i) t[b] = fmaf(v[i], gv[i], t[b]);
+                        if (chunk_ok) {
+                            const float aw = __int_as_float(e[b].y);
+                            float *dst = gvb + e[b].x;
+#pragma unroll
+                            for (int i = 0; i < kVec; i += 4)
+                                red_add_v4(dst + i, aw * gv[i], aw * gv[i + 1], aw * gv[i + 2],
+                                           aw * gv[i + 3]);
                         }
                     }
                 }
-            }
-            uint4 raw[NB][4];
+                // stage A: sum t over the R chunk lanes; this lane keeps instruction b = chunk
+                reduce_scatter_n<R, kB, kB>(t, lane);
+                const int s = s0 + chunk * kSG + sg;
+                const float4 rec = smp[warp][it][s < P ? s : 0];
+                const float fx = rec.x, fy = rec.y;
+                const float wxc = cx ? fx : __fsub_rn(1.f, fx);
+                const float wyc = cy ? fy : __fsub_rn(1.f, fy);
+                float q0 = (wyc * wxc) * t[0];                 // w t
+                float q1 = (cx ? wyc : -wyc) * t[0];           // dw/dfx t
+                float q2 = (cy ? wxc : -wxc) * t[0];           // dw/dfy t
+                // stage B: sum over the four corner lanes of the sample
 #pragma unroll
-            for (int u = 0; u < NB; ++u)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) raw[u][c] = __ldg(reinterpret_cast<const uint4 *>(ptr[u][c]));
-#pragma unroll
-            for (int u = 0; u < NB; ++u) {
-                const int i = i0 + u;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float v[kVec];
-                    widen<VT>(raw[u][c], v);
-                    float t = 0.f;
-#pragma unroll
-                    for (int e = 0; e < kVec; ++e) t = fmaf(v[e], gv[e], t);
-                    q[i] = fmaf(w[u][c], t, q[i]);
-                    q[NS + i] = fmaf(dwx[u][c], t, q[NS + i]);
-                    q[2 * NS + i] = fmaf(dwy[u][c], t, q[2 * NS + i]);
-                    if (goff[u][c] >= 0 && chunk_ok) {
-                        const float aw = aS[i] * w[u][c];
-                        float *dst = gmap + goff[u][c];
-#pragma unroll
-                        for (int e = 0; e < kVec; e += 4)
-                            red_add_v4(dst + e, aw * gv[e], aw * gv[e + 1], aw * gv[e + 2],
-                                       aw * gv[e + 3]);
-                    }
+                for (int o = R; o < 4 * R; o <<= 1) {
+                    q0 += __shfl_xor_sync(kFull, q0, o);
+                    q1 += __shfl_xor_sync(kFull, q1, o);
+                    q2 += __shfl_xor_sync(kFull, q2, o);
+                }
+                if (corner == 0 && s < LK) {
+                    const int64_t si = sbase + s;
+                    if (p.grad_attn) __stcs(p.grad_attn + si, q0);
+                    if (p.grad_loc)
+                        __stcs(reinterpret_cast<float2 *>(p.grad_loc) + si,
+                               make_float2(rec.z * q1, rec.w * q2));
                 }
             }
         }
-
-        // combine the R chunk lanes of each group: lane `chunk` ends with the
-        // totals of partial sums chunk*kPer ... chunk*kPer + kPer - 1
-        reduce_scatter_n<R, kCnt, kCnt>(q, lane);
-#pragma unroll
-        for (int k = 0; k < kPer; ++k) {
-            const int idx = chunk * kPer + k;
-            const int qty = idx / NS;
-            const int i = idx % NS;
-            const int s = g + G * i;
-            if (qty < 3 && s < LK) {
-                const int64_t si = sbase + s;
-                if (qty == 0) {
-                    if (p.grad_attn) __stcs(p.grad_attn + si, q[k]);
-                } else if (p.grad_loc) {
-                    // the slot's level: every lane holds lvW/lvH for all its slots
-                    float scale = 0.f, a = 0.f;
-#pragma unroll
-                    for (int jj = 0; jj < NS; ++jj)
-                        if (jj == i) {
-                            scale = (qty == 1) ? (float)lvW[jj] : (float)lvH[jj];
-                            a = aS[jj];
-                        }
-                    __stcs(p.grad_loc + 2 * si + (qty - 1), a * (scale * q[k]));
-                }
-            }
-        }
+        __syncwarp();
     }
 }
 
-template <typename VT, int R, int NS>
-cudaError_t launch_fast(BwdParams p, cudaStream_t stream)
+template <typename VT, int R, int P>
+cudaError_t launch_fast(const BwdParams &p, cudaStream_t stream)
 {
-    constexpr int NB = NS < 2 ? NS : 2;
-    auto kern = bwd_kernel<VT, R, NS, NB>;
-    const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kWarps);
-    p.chunk = (p.items + ctas - 1) / ctas;
-    p.chunk = (p.chunk + kWarps - 1) / kWarps * kWarps;
-    const dim3 grid((unsigned)((p.items + p.chunk - 1) / p.chunk));
-    kern<<<grid, kWarps * 32, 0, stream>>>(p);
+    constexpr int kRound = kWarps * (32 / P);
+    auto kern = bwd_kernel<VT, R, P>;
+    const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kRound);
+    bwd_kernel<VT, R, P><<<(unsigned)ctas, kWarps * 32, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
 template <typename VT, int R>
 cudaError_t launch_fast_r(const BwdParams &p, cudaStream_t stream)
 {
-    constexpr int G = 32 / R;
+    // P: a power of two >= L*K and >= the 8 samples of one batch
     const int LK = p.L * p.K;
-    const int nsl = (LK + G - 1) / G;
-    if (nsl <= 1) return launch_fast<VT, R, 1>(p, stream);
-    if constexpr (G <= 16) {
-        if (nsl <= 2) return launch_fast<VT, R, 2>(p, stream);
-    }
-    if constexpr (G <= 8) {
-        if (nsl <= 4) return launch_fast<VT, R, 4>(p, stream);
-    }
-    if constexpr (G <= 4) {
-        return launch_fast<VT, R, 8>(p, stream);
-    }
-    return cudaErrorInvalidValue;  // not reached: L*K <= 32
+    if (LK <= 8) return launch_fast<VT, R, 8>(p, stream);
+    if (LK <= 16) return launch_fast<VT, R, 16>(p, stream);
+    return launch_fast<VT, R, 32>(p, stream);
 }
 
 template <typename VT>
 cudaError_t launch_bwd_vt(const BwdParams &p, int R, cudaStream_t stream)
 {
+    // fast path: four elements per lane, R4 = D/4 lanes per (fp32) gradient row
+    const int r4 = p.D / 4;
+    if (p.D % 4 == 0 && r4 <= 8) {
+        BwdParams q = p;
+        q.nchunks = r4;
+        if (r4 <= 1) return launch_fast_r<VT, 1>(q, stream);
+        if (r4 <= 2) return launch_fast_r<VT, 2>(q, stream);
+        if (r4 <= 4) return launch_fast_r<VT, 4>(q, stream);
+        return launch_fast_r<VT, 8>(q, stream);
+    }
     const dim3 block(kWarps * 32);
     const dim3 grid((unsigned)((p.items + kWarps - 1) / kWarps));
     switch (R) {
-    case 1: return launch_fast_r<VT, 1>(p, stream);
-    case 2: return launch_fast_r<VT, 2>(p, stream);
-    case 4: return launch_fast_r<VT, 4>(p, stream);
-    case 8: return launch_fast_r<VT, 8>(p, stream);
+    case 1: bwd_kernel_wide<VT, 1><<<grid, block, 0, stream>>>(p); break;
+    case 2: bwd_kernel_wide<VT, 2><<<grid, block, 0, stream>>>(p); break;
+    case 4: bwd_kernel_wide<VT, 4><<<grid, block, 0, stream>>>(p); break;
+    case 8: bwd_kernel_wide<VT, 8><<<grid, block, 0, stream>>>(p); break;
     case 16: bwd_kernel_wide<VT, 16><<<grid, block, 0, stream>>>(p); break;
     case 32: bwd_kernel_wide<VT, 32><<<grid, block, 0, stream>>>(p); break;
     default: return cudaErrorInvalidValue;

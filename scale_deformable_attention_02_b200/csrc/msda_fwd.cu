@@ -260,202 +260,280 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
     }
 }
 
+// EPL consecutive value elements of one lane (16 or 8 bytes), widened to
+// float pairs when consumed.
+template <typename VT, int EPL>
+struct LaneLoad;
+
+template <>
+struct LaneLoad<float, 4> {
+    using Raw = uint4;
+    __device__ __forceinline__ static Raw load(const float *p)
+    {
+        return __ldg(reinterpret_cast<const uint4 *>(p));
+    }
+    __device__ __forceinline__ static void widen(const Raw &r, float2 (&v)[2])
+    {
+        v[0] = make_float2(__uint_as_float(r.x), __uint_as_float(r.y));
+        v[1] = make_float2(__uint_as_float(r.z), __uint_as_float(r.w));
+    }
+};
+
+template <>
+struct LaneLoad<__nv_bfloat16, 8> {
+    using Raw = uint4;
+    __device__ __forceinline__ static Raw load(const __nv_bfloat16 *p)
+    {
+        return __ldg(reinterpret_cast<const uint4 *>(p));
+    }
+    __device__ __forceinline__ static void widen(const Raw &r, float2 (&v)[4])
+    {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)  // exact widening: bf16 bits become the high half
+            v[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
+    }
+};
+
+template <>
+struct LaneLoad<__nv_bfloat16, 4> {
+    using Raw = uint2;
+    __device__ __forceinline__ static Raw load(const __nv_bfloat16 *p)
+    {
+        return __ldg(reinterpret_cast<const uint2 *>(p));
+    }
+    __device__ __forceinline__ static void widen(const Raw &r, float2 (&v)[2])
+    {
+        v[0] = make_float2(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xffff0000u));
+        v[1] = make_float2(__uint_as_float(r.y << 16), __uint_as_float(r.y & 0xffff0000u));
+    }
+};
+
 // ---------------------------------------------------------------------------
 // Fast path for value rows of at most 128 bytes (R <= 8 lanes per row).
 //
-// Lane layout: G = 32/R groups of R lanes; group g owns samples g, g+G, g+2G,
-// ... of the item (all four corners of each), lane `chunk` of the group owns
-// 16 bytes of every row.  So every lane forms the row addresses and weights
-// it gathers with in its own registers -- no shared-memory entries -- and a
-// warp instruction still gathers G whole rows, 16 bytes per lane.  The
-// per-level metadata of a lane's sample slots is the same for every item and
-// is read once.  Fused: lane j first forms sample j's location and attention
-// weight (one IEEE divide per coordinate, one softmax per item), and the
-// group lanes fetch them with three shuffles.
+// The gather is bound by how many rows the L2 can return per second, which
+// needs many warps per SM more than deep per-warp queues, so this kernel keeps
+// its register footprint small (FWD_MIN_CTAS CTAs of 8 warps per SM):
+//   * a warp loops over rounds of 32/P items (P = lanes per item); lane j of
+//     an item's P-lane segment owns sample j, whose level metadata it keeps in
+//     registers for the whole kernel;
+//   * the inputs of the next round (logits and offsets, or locations and
+//     weights) are loaded while the current round gathers;
+//   * phase 1 forms the location, weight and cell of each sample and stores
+//     its four corners as 8-byte (row offset, weight) entries, corner-major
+//     with stride P + 2 so stores and loads are free of bank conflicts;
+//   * phase 2 gathers FWD_BATCH corner-row groups before consuming them; a
+//     corner outside the level predicates its load and its FMA off.
 // ---------------------------------------------------------------------------
-template <typename VT, int R, int NS, int NB, bool kFused>
-__global__ void __launch_bounds__(kWarps * 32, 3)
+#ifndef MSDA_FWD_BATCH
+#define MSDA_FWD_BATCH 4
+#endif
+#ifndef MSDA_FWD_MIN_CTAS
+#define MSDA_FWD_MIN_CTAS 4
+#endif
+#ifndef MSDA_FWD_PREFETCH
+#define MSDA_FWD_PREFETCH 1  // load the next round's inputs during this round's gathers
+#endif
+
+template <typename VT, int EPL, int R, int P, bool kFused>
+__global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
     fwd_kernel(const __grid_constant__ FwdParams p)
 {
-    static_assert(R <= 8 && NS * (32 / R) <= 32, "fast path shape");
-    constexpr int G = 32 / R;           // samples gathered per warp instruction
-    constexpr int kNP = Pairs<VT>::kN;  // float pairs per 16-byte chunk
+    using LL = LaneLoad<VT, EPL>;
+    constexpr int kSlots = 32 / R;      // (sample, corner) pairs per warp instruction
+    constexpr int kItems = 32 / P;      // items per round
+    constexpr int kStride = P + 2;      // = 2 mod 8 for P >= 8: conflict-free entries
+    constexpr int kNP = EPL / 2;        // float pairs per lane
+    constexpr int kB0 = MSDA_FWD_BATCH;
+    constexpr int kB = kB0 * kSlots <= 4 * P ? kB0 : (4 * P) / kSlots;
+    static_assert(kB >= 1 && (4 * P) % (kB * kSlots) == 0, "a batch must tile the entries");
+    __shared__ int2 ent[kWarps][kItems][4 * kStride];  // (row element offset | -1, weight)
+
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int g = lane / R;
-    const int chunk = lane % R;
     const int M = p.M, D = p.D, K = p.K;
     const int LK = p.L * K;
     const int MD = M * D;
-    const int nsl = (LK + G - 1) / G;  // sample slots in use, <= NS
+    const int npairs = 4 * LK;
+
+    // phase-1 role: sample j of the round's item `seg`
+    const int seg = lane / P;
+    const int j = lane % P;
+    const bool jact = j < LK;
+    const int lvl = jact ? j / K : 0;
+    const int H = p.lv.H[lvl], W = p.lv.W[lvl], start = p.lv.start[lvl];
+
+    // phase-2 role: 16-byte chunk `chunk` of the rows in slot `slot`
+    const int slot = lane / R;
+    const int chunk = lane % R;
     const bool chunk_ok = chunk < p.nchunks;
     // lanes past the last chunk of a row re-read chunk 0; their sums are discarded
-    const int lane_off = chunk_ok ? chunk * 16 : 0;
-    const char *zrow = reinterpret_cast<const char *>(kZeroRow) + lane_off;
-    const int64_t rowbytes = (int64_t)MD * (int64_t)sizeof(VT);
+    const int lane_elem = (chunk_ok ? chunk : 0) * EPL;
 
-    int lvW[NS], lvH[NS], lvS[NS];  // level of sample slot i (sample g + G*i)
-#pragma unroll
-    for (int i = 0; i < NS; ++i) {
-        const int s = g + G * i;
-        const int l = s < LK ? s / K : 0;
-        lvW[i] = p.lv.W[l];
-        lvH[i] = p.lv.H[l];
-        lvS[i] = p.lv.start[l];
-    }
+    const int64_t stride = (int64_t)gridDim.x * kWarps * kItems;
+    int64_t item0 = ((int64_t)blockIdx.x * kWarps + warp) * kItems;
 
-    const int64_t begin = (int64_t)blockIdx.x * p.chunk;
-    const int64_t end = begin + p.chunk < p.items ? begin + p.chunk : p.items;
-    for (int64_t item = begin + warp; item < end; item += kWarps) {
-        const int m = (int)(item % M);
-        const int64_t nq = item / M;
-        const int64_t n = nq / p.Lq;
-        const int64_t sbase = item * LK;
-        const char *mapb = static_cast<const char *>(p.value) +
-                           (n * p.S * M + m) * (int64_t)D * (int64_t)sizeof(VT) + lane_off;
+    // inputs of this lane's sample in the round starting at item0
+    float pa = 0.f, pb = 0.f, pc = 0.f;
+    auto fetch = [&](int64_t i0) {
+        const int64_t item = i0 + seg;
+        pa = pb = pc = 0.f;
+        if (jact && item < p.items) {
+            const int64_t si = item * LK + j;
+            if constexpr (kFused) {
+                pa = __ldcs(p.logits + si);
+                const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + si);
+                pb = o.x;
+                pc = o.y;
+            } else {
+                const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
+                pb = t.x;
+                pc = t.y;
+                pa = __ldcs(p.attn + si);
+            }
+        }
+    };
+    if (MSDA_FWD_PREFETCH) fetch(item0);
 
-        float ax = 0.f, ay = 0.f, aa = 0.f;  // fused: sample `lane`'s location and weight
+    for (; item0 < p.items; item0 += stride) {
+        if (!MSDA_FWD_PREFETCH) fetch(item0);
+        // ---- phase 1 -------------------------------------------------------
+        const int64_t item = item0 + seg;
+        const bool act = jact && item < p.items;
+        const int64_t si = item * LK + j;
+        float lx, ly, a;
         if constexpr (kFused) {
-            const bool act = lane < LK;
-            const float z = act ? __ldcs(p.logits + sbase + lane) : -INFINITY;
-            const float mx = warp_max(z);
+            // joint softmax over the item's L*K logits, max-subtracted
+            const float z = act ? pa : -INFINITY;
+            const float mx = seg_max<P>(z);
             const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
-            const float sum = warp_sum(e);
-            aa = __fdiv_rn(e, sum);
+            const float sum = seg_sum<P>(e);
+            a = __fdiv_rn(e, sum);
+            lx = ly = 0.f;
             if (act) {
-                const int l = lane / K;
-                const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sbase + lane);
+                const int64_t nq = item / M;
                 if (p.ref_dim == 2) {
                     // point reference: offsets are level-l pixels
                     const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
-                    ax = __fadd_rn(r.x, __fdiv_rn(o.x, (float)p.lv.W[l]));
-                    ay = __fadd_rn(r.y, __fdiv_rn(o.y, (float)p.lv.H[l]));
+                    lx = __fadd_rn(r.x, __fdiv_rn(pb, (float)W));
+                    ly = __fadd_rn(r.y, __fdiv_rn(pc, (float)H));
                 } else {
                     // box reference (cx, cy, w, h): offsets are in box units
                     const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
                     const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
-                    ax = __fadd_rn(c.x, __fmul_rn(o.x, s2.x));
-                    ay = __fadd_rn(c.y, __fmul_rn(o.y, s2.y));
+                    lx = __fadd_rn(c.x, __fmul_rn(pb, s2.x));
+                    ly = __fadd_rn(c.y, __fmul_rn(pc, s2.y));
                 }
                 if (p.loc_out)
-                    __stcs(reinterpret_cast<float2 *>(p.loc_out) + sbase + lane,
-                           make_float2(ax, ay));
-                if (p.attn_out) __stcs(p.attn_out + sbase + lane, aa);
+                    __stcs(reinterpret_cast<float2 *>(p.loc_out) + si, make_float2(lx, ly));
+                if (p.attn_out) __stcs(p.attn_out + si, a);
             }
+        } else {
+            lx = pb;
+            ly = pc;
+            a = pa;
         }
-
-        float2 acc[kNP];
-#pragma unroll
-        for (int i = 0; i < kNP; ++i) acc[i] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int i0 = 0; i0 < NS; i0 += NB) {
-            if (i0 >= nsl) break;  // uniform across the warp
-            const char *ptr[NB][4];
-            float wt[NB][4];
-#pragma unroll
-            for (int u = 0; u < NB; ++u) {
-                const int i = i0 + u;
-                const int s = g + G * i;  // < 32
-                const bool have = s < LK;
-                float lx = 0.f, ly = 0.f, a = 0.f;
-                if constexpr (kFused) {
-                    lx = __shfl_sync(kFull, ax, s);
-                    ly = __shfl_sync(kFull, ay, s);
-                    a = __shfl_sync(kFull, aa, s);
-                } else if (have) {
-                    const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + sbase + s);
-                    lx = t.x;
-                    ly = t.y;
-                    a = __ldcs(p.attn + sbase + s);
-                }
+        if (MSDA_FWD_PREFETCH) fetch(item0 + stride);  // loads while this round gathers
+        {
+            int2 e[4] = {{-1, 0}, {-1, 0}, {-1, 0}, {-1, 0}};
+            float x, y, fx, fy;
+            int x0, y0;
+            if (act && msda_cell(lx, ly, H, W, x, y, x0, y0, fx, fy)) {
+                const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+                const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
-                    ptr[u][c] = zrow;
-                    wt[u][c] = 0.f;
+                    const int r = msda_row(start, H, W, y0 + (c >> 1), x0 + (c & 1));
+                    if (r >= 0) e[c] = make_int2(r * MD, __float_as_int(w[c] * a));
                 }
-                float x, y, fx, fy;
-                int x0, y0;
-                if (have && msda_cell(lx, ly, lvH[i], lvW[i], x, y, x0, y0, fx, fy)) {
-                    const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
-                    const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
+            }
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int r = msda_row(lvS[i], lvH[i], lvW[i], y0 + (c >> 1), x0 + (c & 1));
-                        if (r >= 0) {
-                            ptr[u][c] = mapb + (int64_t)r * rowbytes;
-                            wt[u][c] = w[c] * a;
-                        }
+            for (int c = 0; c < 4; ++c) ent[warp][seg][c * kStride + j] = e[c];
+        }
+        __syncwarp();
+
+        // ---- phase 2: gather, item by item --------------------------------
+#pragma unroll 1
+        for (int it = 0; it < kItems; ++it) {
+            const int64_t itm = item0 + it;
+            if (itm >= p.items) break;  // uniform
+            const int m = (int)(itm % M);
+            const int64_t nq = itm / M;
+            const int64_t n = nq / p.Lq;
+            const VT *vb = static_cast<const VT *>(p.value) + (n * p.S * M + m) * (int64_t)D +
+                           lane_elem;
+            const int2 *en = ent[warp][it];
+            float2 acc[kNP];
+#pragma unroll
+            for (int i = 0; i < kNP; ++i) acc[i] = make_float2(0.f, 0.f);
+            for (int t0 = 0; t0 < npairs; t0 += kB * kSlots) {
+                int2 e[kB];
+                typename LL::Raw raw[kB];
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    const int t = t0 + b * kSlots + slot;  // pair (sample t/4, corner t%4)
+                    e[b] = en[(t & 3) * kStride + (t >> 2)];
+                    if (e[b].x >= 0) raw[b] = LL::load(vb + e[b].x);
+                }
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    if (e[b].x >= 0) {
+                        float2 v[kNP];
+                        LL::widen(raw[b], v);
+                        const float wb = __int_as_float(e[b].y);
+                        const float2 w2 = make_float2(wb, wb);
+#pragma unroll
+                        for (int i = 0; i < kNP; ++i) acc[i] = __ffma2_rn(w2, v[i], acc[i]);
                     }
                 }
             }
-            uint4 raw[NB][4];
 #pragma unroll
-            for (int u = 0; u < NB; ++u)
+            for (int o = R; o < 32; o <<= 1)
 #pragma unroll
-                for (int c = 0; c < 4; ++c) raw[u][c] = __ldg(reinterpret_cast<const uint4 *>(ptr[u][c]));
-#pragma unroll
-            for (int u = 0; u < NB; ++u)
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    float2 v[kNP];
-                    Pairs<VT>::widen(raw[u][c], v);
-                    const float2 wb = make_float2(wt[u][c], wt[u][c]);
-#pragma unroll
-                    for (int i = 0; i < kNP; ++i) acc[i] = __ffma2_rn(wb, v[i], acc[i]);
+                for (int i = 0; i < kNP; ++i) {
+                    acc[i].x += __shfl_xor_sync(kFull, acc[i].x, o);
+                    acc[i].y += __shfl_xor_sync(kFull, acc[i].y, o);
                 }
-        }
-
-        // sum over the G groups, then lanes 0..R-1 store the item's D outputs
+            if (slot == 0 && chunk_ok) {
+                float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D +
+                                                         chunk * EPL);
 #pragma unroll
-        for (int o = R; o < 32; o <<= 1)
-#pragma unroll
-            for (int i = 0; i < kNP; ++i) {
-                acc[i].x += __shfl_xor_sync(kFull, acc[i].x, o);
-                acc[i].y += __shfl_xor_sync(kFull, acc[i].y, o);
+                for (int i = 0; i < kNP / 2; ++i)
+                    __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
+                                                acc[2 * i + 1].y));
             }
-        if (g == 0 && chunk_ok) {
-            float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D +
-                                                     chunk * (2 * kNP));
-#pragma unroll
-            for (int i = 0; i < kNP / 2; ++i)
-                __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
-                                            acc[2 * i + 1].y));
         }
+        __syncwarp();  // the next round overwrites this warp's entries
     }
 }
 
-template <typename VT, int R, int NS, bool kFused>
+template <typename VT, int EPL, int R, int P, bool kFused>
 cudaError_t launch_fast(FwdParams p, cudaStream_t stream)
 {
-    constexpr int NB = NS < 2 ? NS : 2;  // sample slots gathered per batch (4 rows each)
-    auto kern = fwd_kernel<VT, R, NS, NB, kFused>;
-    const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kWarps);
-    p.chunk = (p.items + ctas - 1) / ctas;
-    p.chunk = (p.chunk + kWarps - 1) / kWarps * kWarps;
-    const dim3 grid((unsigned)((p.items + p.chunk - 1) / p.chunk));
-    kern<<<grid, kWarps * 32, 0, stream>>>(p);
+    constexpr int kRound = kWarps * (32 / P);  // items per CTA round
+    auto kern = fwd_kernel<VT, EPL, R, P, kFused>;
+    const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kRound);
+    fwd_kernel<VT, EPL, R, P, kFused><<<(unsigned)ctas, kWarps * 32, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
-template <typename VT, int R, bool kFused>
+template <typename VT, int EPL, int R, bool kFused>
 cudaError_t launch_fast_r(const FwdParams &p, cudaStream_t stream)
 {
-    constexpr int G = 32 / R;
+    // P: a power of two >= L*K, >= 8 (conflict-free entry stride) and >= the
+    // 8/R samples one warp instruction gathers
     const int LK = p.L * p.K;
-    const int nsl = (LK + G - 1) / G;  // sample slots per lane
-    if (nsl <= 1) return launch_fast<VT, R, 1, kFused>(p, stream);
-    if constexpr (G <= 16) {
-        if (nsl <= 2) return launch_fast<VT, R, 2, kFused>(p, stream);
-    }
-    if constexpr (G <= 8) {
-        if (nsl <= 4) return launch_fast<VT, R, 4, kFused>(p, stream);
-    }
-    if constexpr (G <= 4) {
-        return launch_fast<VT, R, 8, kFused>(p, stream);
-    }
-    return cudaErrorInvalidValue;  // not reached: L*K <= 32
+    if (LK <= 8) return launch_fast<VT, EPL, R, 8, kFused>(p, stream);
+    if (LK <= 16) return launch_fast<VT, EPL, R, 16, kFused>(p, stream);
+    return launch_fast<VT, EPL, R, 32, kFused>(p, stream);
 }
 
+// Elements per lane for bf16 values: 8 (16-byte loads, 2x the rows per
+// instruction) or 4 (8-byte loads, the fp32 lane layout).
+#ifndef MSDA_FWD_BF16_EPL
+#define MSDA_FWD_BF16_EPL 8
+#endif
 
 template <typename VT, int R, int P, bool kFused>
 cudaError_t launch_p(FwdParams p, bool exact, cudaStream_t stream)
@@ -489,12 +567,23 @@ cudaError_t launch_r(const FwdParams &p, bool exact, cudaStream_t stream)
 template <typename VT, bool kFused>
 cudaError_t launch_fwd_vt(const FwdParams &p, int R, cudaStream_t stream)
 {
+    constexpr int EPL = sizeof(VT) == 4 ? 4 : MSDA_FWD_BF16_EPL;
+    // fast path: rows of at most 8 lanes of EPL elements
+    const int lanes = (p.D + EPL - 1) / EPL;
+    if (p.D % EPL == 0 && lanes <= 8) {
+        FwdParams q = p;
+        q.nchunks = lanes;
+        if (lanes <= 1) return launch_fast_r<VT, EPL, 1, kFused>(q, stream);
+        if (lanes <= 2) return launch_fast_r<VT, EPL, 2, kFused>(q, stream);
+        if (lanes <= 4) return launch_fast_r<VT, EPL, 4, kFused>(q, stream);
+        return launch_fast_r<VT, EPL, 8, kFused>(q, stream);
+    }
     const bool exact = p.nchunks == R;
     switch (R) {
-    case 1: return launch_fast_r<VT, 1, kFused>(p, stream);
-    case 2: return launch_fast_r<VT, 2, kFused>(p, stream);
-    case 4: return launch_fast_r<VT, 4, kFused>(p, stream);
-    case 8: return launch_fast_r<VT, 8, kFused>(p, stream);
+    case 1: return launch_r<VT, 1, kFused>(p, exact, stream);
+    case 2: return launch_r<VT, 2, kFused>(p, exact, stream);
+    case 4: return launch_r<VT, 4, kFused>(p, exact, stream);
+    case 8: return launch_r<VT, 8, kFused>(p, exact, stream);
     case 16: return launch_r<VT, 16, kFused>(p, exact, stream);
     case 32: return launch_r<VT, 32, kFused>(p, exact, stream);
     default: return cudaErrorInvalidValue;
