@@ -63,6 +63,11 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle leg")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--step", choices=["split", "fused"], default="split",
+                    help="split: fused forward writing locations and weights, then "
+                         "msda_backward (grad value, locations, weights); fused: fused "
+                         "forward writing only out, then msda_backward_fused (grad value, "
+                         "reference points, offsets, logits)")
     return ap.parse_args(argv)
 
 
@@ -92,19 +97,26 @@ def max_over_ranks(vals, world: int, device):
 # ---------------------------------------------------------------------------
 # algorithmic (unique) bytes per launch
 # ---------------------------------------------------------------------------
-def algorithmic_bytes(w: wl.Workload) -> dict:
+def algorithmic_bytes(w: wl.Workload, step: str = "split") -> dict:
     """Minimum HBM traffic of each launch: every input read once, every
     output written once (the value map counted once although its rows are
     gathered many times; the backward's zero-fill of grad_value is not
-    counted)."""
+    counted).  split: the forward also writes locations and weights, which
+    the backward reads; fused: neither pass stores them."""
     N, Lq, S, M, D, L, K = (w.N, w.queries, w.S, w.M, w.D, w.L, w.K)
     esz = 2 if w.value_dtype == "bf16" else 4
     samples = N * Lq * M * L * K
     value = N * S * M * D * esz
+    gvalue = N * S * M * D * 4
     ref = N * Lq * 2 * 4
     outb = N * Lq * M * D * 4
-    fwd = value + ref + samples * 8 + samples * 4 + outb + samples * 8 + samples * 4
-    bwd = value + samples * 8 + samples * 4 + outb + N * S * M * D * 4 + samples * 8 + samples * 4
+    per = samples * 12  # (x, y) and one weight/logit per sample, fp32
+    if step == "fused":
+        fwd = value + ref + per + outb
+        bwd = value + ref + per + outb + gvalue + ref + per
+    else:
+        fwd = value + ref + per + outb + per
+        bwd = value + per + outb + gvalue + per
     return {"fwd": fwd, "bwd": bwd, "samples": samples}
 
 
@@ -220,7 +232,8 @@ def run_ours(args):
     import torch
     import torch.distributed as dist
 
-    from scale_deformable_attention_02_b200 import msda_backward, msda_forward_fused
+    from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fused,
+                                                    msda_forward_fused)
 
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -252,15 +265,26 @@ def run_ours(args):
     starts, _ = __import__("scale_deformable_attention_02_b200").msda_level_start_index(sh)
     stream = torch.cuda.current_stream(device)
 
+    gref = torch.empty_like(ref)
+    fused = args.step == "fused"
+
     def step():
-        msda_forward_fused(value, sh, starts, ref, off, logits, out=out,
-                           sampling_locations_out=loc, attention_weights_out=attn,
-                           stream=stream)
+        if fused:
+            msda_forward_fused(value, sh, starts, ref, off, logits, out=out, stream=stream)
+        else:
+            msda_forward_fused(value, sh, starts, ref, off, logits, out=out,
+                               sampling_locations_out=loc, attention_weights_out=attn,
+                               stream=stream)
 
     def step_bwd():
-        msda_backward(value, sh, starts, loc, attn, gout, grad_value=gval,
-                      grad_sampling_locations=gloc, grad_attention_weights=gattn,
-                      stream=stream)
+        if fused:
+            msda_backward_fused(value, sh, starts, ref, off, logits, gout, grad_value=gval,
+                                grad_reference_points=gref, grad_offsets=gloc,
+                                grad_logits=gattn, stream=stream)
+        else:
+            msda_backward(value, sh, starts, loc, attn, gout, grad_value=gval,
+                          grad_sampling_locations=gloc, grad_attention_weights=gattn,
+                          stream=stream)
 
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush = torch.empty(max(2 * l2, 64 << 20), dtype=torch.uint8, device=device)
@@ -306,15 +330,17 @@ def run_ours(args):
 
     # ---- roofline of the dominant launch ----------------------------------
     peak, peak_kind = read_peaks()
-    ab = algorithmic_bytes(w)
+    ab = algorithmic_bytes(w, args.step)
     dom = "bwd" if ms_bwd >= ms_fwd else "fwd"
     dom_ms = ms_bwd if dom == "bwd" else ms_fwd
     achieved = ab[dom] / (dom_ms / 1e3) / 1e9
+    bwd_name = ("memset + bwd_kernel (msda_backward_fused)" if args.step == "fused"
+                else "memset + bwd_kernel (msda_backward)")
     kernels = {
         "fwd": {"kernel": "fwd_kernel (msda_forward_fused)", "ms": ms_fwd,
                 "algorithmic_bytes": ab["fwd"],
                 "GB_s": ab["fwd"] / (ms_fwd / 1e3) / 1e9},
-        "bwd": {"kernel": "memset + bwd_kernel (msda_backward)", "ms": ms_bwd,
+        "bwd": {"kernel": bwd_name, "ms": ms_bwd,
                 "algorithmic_bytes": ab["bwd"],
                 "GB_s": ab["bwd"] / (ms_bwd / 1e3) / 1e9},
     }
@@ -324,7 +350,9 @@ def run_ours(args):
         "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
         "frac": achieved / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
         if peak_kind == "measured" else "fallback 6.65 TB/s",
-        "traffic": read_traffic(args.workload, dom), "kernel": kernels[dom]["kernel"],
+        "traffic": read_traffic(args.workload if args.step == "split" else
+                                args.workload + "/fused", dom),
+        "kernel": kernels[dom]["kernel"],
         "algorithmic_bytes_per_launch": ab[dom],
     }
 
@@ -349,6 +377,10 @@ def run_ours(args):
                     "encoder/decoder, no dataset or trained weights)",
             "config": {
                 "workload": WORKLOAD_TEXT[args.workload],
+                "step": ("fused forward (out only) + fused backward (grad value, reference "
+                         "points, offsets, logits)" if args.step == "fused" else
+                         "fused forward (out, locations, weights) + backward (grad value, "
+                         "locations, weights)"),
                 "value_dtype": w.value_dtype,
                 "global_batch": w.N * world,
                 "queries_per_step": queries * world,
@@ -391,7 +423,9 @@ def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_
     buffers: H2D of the step's inputs, fused forward, backward, D2H of the
     step's results (out, grad_value, grad_sampling_locations,
     grad_attention_weights), all inside the timed events."""
-    from scale_deformable_attention_02_b200 import msda_backward, msda_forward_fused
+    from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fused,
+                                                    msda_forward_fused)
+    fused = args.step == "fused"
 
     def pinned(a):
         a = np.ascontiguousarray(a)
@@ -403,6 +437,8 @@ def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_
     d_in = {k: torch.empty(h_in[k].shape, dtype=h_in[k].dtype, device=device) for k in names}
     res_shapes = {"out": (w.N, w.queries, w.M * w.D), "grad_value": (w.N, w.S, w.M, w.D),
                   "grad_loc": tuple(inp["offsets"].shape), "grad_attn": tuple(inp["logits"].shape)}
+    if fused:
+        res_shapes["grad_ref"] = tuple(inp["reference_points"].shape)
     h_out = {k: torch.empty(s, dtype=torch.float32).pin_memory() for k, s in res_shapes.items()}
     d_out = {k: torch.empty(s, dtype=torch.float32, device=device) for k, s in res_shapes.items()}
     loc = torch.empty(tuple(inp["offsets"].shape), device=device)
@@ -413,12 +449,21 @@ def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_
         for k in names:
             d_in[k].copy_(h_in[k], non_blocking=True)
         v = d_in["value"].view(torch.bfloat16) if bf16 else d_in["value"]
-        msda_forward_fused(v, sh, starts, d_in["reference_points"], d_in["offsets"],
-                           d_in["logits"], out=d_out["out"], sampling_locations_out=loc,
-                           attention_weights_out=attn, stream=stream)
-        msda_backward(v, sh, starts, loc, attn, d_in["grad_out"],
-                      grad_value=d_out["grad_value"], grad_sampling_locations=d_out["grad_loc"],
-                      grad_attention_weights=d_out["grad_attn"], stream=stream)
+        if fused:
+            msda_forward_fused(v, sh, starts, d_in["reference_points"], d_in["offsets"],
+                               d_in["logits"], out=d_out["out"], stream=stream)
+            msda_backward_fused(v, sh, starts, d_in["reference_points"], d_in["offsets"],
+                                d_in["logits"], d_in["grad_out"], grad_value=d_out["grad_value"],
+                                grad_reference_points=d_out["grad_ref"],
+                                grad_offsets=d_out["grad_loc"], grad_logits=d_out["grad_attn"],
+                                stream=stream)
+        else:
+            msda_forward_fused(v, sh, starts, d_in["reference_points"], d_in["offsets"],
+                               d_in["logits"], out=d_out["out"], sampling_locations_out=loc,
+                               attention_weights_out=attn, stream=stream)
+            msda_backward(v, sh, starts, loc, attn, d_in["grad_out"],
+                          grad_value=d_out["grad_value"], grad_sampling_locations=d_out["grad_loc"],
+                          grad_attention_weights=d_out["grad_attn"], stream=stream)
         for k in res_shapes:
             h_out[k].copy_(d_out[k], non_blocking=True)
 

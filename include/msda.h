@@ -212,6 +212,44 @@ MSDA_API msda_status msda_backward(const void *value, msda_dtype value_dtype,
                           float *grad_attention_weights, msda_dims dims,
                           msda_stream_t stream);
 
+/*
+ * Backward of msda_forward_fused, chained to the raw projection outputs.
+ * The attention weights and sampling locations are recomputed from the
+ * inputs exactly as msda_forward_fused forms them (bit for bit), the
+ * gradients through the interpolation are formed as in msda_backward, and
+ * the chain rule is applied inside the kernel ("Deformable DETR" wiki page,
+ * "Multi-scale deformable attention" and "Variants"; the gradients reach the
+ * 3MK projection through the offsets and the softmax):
+ *   point reference (loc = ref + off / W_l):
+ *     grad_offsets = grad_loc / W_l (per level),  grad_reference = sum of grad_loc
+ *   box reference (loc = (cx, cy) + off * (w, h)):
+ *     grad_offsets = grad_loc * (w, h),
+ *     grad_reference = (sum grad_loc_x, sum grad_loc_y,
+ *                       sum grad_loc_x * off_x, sum grad_loc_y * off_y)
+ *   grad_logits = A * (grad_A - sum_j A_j grad_A_j)     (per head, over L*K)
+ * where the sums run over the heads, levels and points of the query.
+ *
+ *   reference_points, reference_dim, offsets, logits  as msda_forward_fused
+ *   grad_out                device [N,Lq,M*D] fp32, 16-byte aligned
+ *   grad_value              device [N,S,M,D] fp32; zeroed, then accumulated
+ *   grad_reference_points   NULL or device [N,Lq,reference_dim] fp32;
+ *                           zeroed, then accumulated over heads (atomics)
+ *   grad_offsets            NULL or device [N,Lq,M,L,K,2] fp32 (written)
+ *   grad_logits             NULL or device [N,Lq,M,L,K] fp32 (written)
+ *
+ * Limits: D <= 32 (MSDA_ERR_UNSUPPORTED otherwise).  Errors: as
+ * msda_forward_fused; every gradient buffer is an output for the alias check.
+ */
+MSDA_API msda_status msda_backward_fused(const void *value, msda_dtype value_dtype,
+                                         const int64_t *spatial_shapes,
+                                         const int64_t *level_start_index,
+                                         const float *reference_points, int reference_dim,
+                                         const float *offsets, const float *logits,
+                                         const float *grad_out, float *grad_value,
+                                         float *grad_reference_points, float *grad_offsets,
+                                         float *grad_logits, msda_dims dims,
+                                         msda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

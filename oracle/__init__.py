@@ -75,6 +75,10 @@ def lib():
             _lib.ora_backward.argtypes = [P, I, P, P, P, I, P, P, P, P, P, P, P, Dims]
             _lib.ora_fused_chain.restype = None
             _lib.ora_fused_chain.argtypes = [P, P, P, P, Dims, P, P, P]
+            _lib.ora_fused_chain_box.restype = None
+            _lib.ora_fused_chain_box.argtypes = [P, P, P, P, P, Dims, P, P, P]
+            _lib.ora_locations_box_f64.restype = None
+            _lib.ora_locations_box_f64.argtypes = [P, P, Dims, P]
             _lib.ora_sample_points_f32.restype = None
             _lib.ora_sample_points_f32.argtypes = [P, P, P, Dims, P, P, P, P, P, P]
             _lib.ora_set_threads.restype = None
@@ -224,6 +228,31 @@ def fused_chain(grad_loc, grad_attn, attn, shapes):
     lib().ora_fused_chain(_ptr(gl), _ptr(ga), _ptr(a), _ptr(shapes),
                           Dims(N, Lq, 0, M, 0, L, K), _ptr(g_ref), _ptr(g_off), _ptr(g_z))
     return g_ref, g_off, g_z
+
+
+def fused_chain_box(grad_loc, grad_attn, attn, box, off):
+    """Chain for box references: returns (grad_box [N,Lq,4], grad_off, grad_logits)."""
+    gl = np.ascontiguousarray(grad_loc, dtype=np.float64)
+    ga = np.ascontiguousarray(grad_attn, dtype=np.float64)
+    a = np.ascontiguousarray(attn, dtype=np.float64)
+    bx = np.ascontiguousarray(box, dtype=np.float64)
+    of = np.ascontiguousarray(off, dtype=np.float64)
+    N, Lq, M, L, K = a.shape
+    g_box = np.empty((N, Lq, 4), dtype=np.float64)
+    g_off = np.empty(gl.shape, dtype=np.float64)
+    g_z = np.empty(a.shape, dtype=np.float64)
+    lib().ora_fused_chain_box(_ptr(gl), _ptr(ga), _ptr(a), _ptr(bx), _ptr(of),
+                              Dims(N, Lq, 0, M, 0, L, K), _ptr(g_box), _ptr(g_off), _ptr(g_z))
+    return g_box, g_off, g_z
+
+
+def locations_box_f64(box: np.ndarray, off: np.ndarray) -> np.ndarray:
+    box = np.ascontiguousarray(box, dtype=np.float64)
+    off = np.ascontiguousarray(off, dtype=np.float64)
+    N, Lq, M, L, K, _ = off.shape
+    loc = np.empty_like(off)
+    lib().ora_locations_box_f64(_ptr(box), _ptr(off), Dims(N, Lq, 0, M, 0, L, K), _ptr(loc))
+    return loc
 
 
 def sample_points(loc: np.ndarray, shapes: np.ndarray) -> dict:

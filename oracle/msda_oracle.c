@@ -441,6 +441,63 @@ void ora_fused_chain(const double *grad_loc, const double *grad_attn, const doub
 }
 
 /*
+ * The same chain for box references (cx, cy, w, h) with loc = (cx, cy) +
+ * off * (w, h) (iterative box refinement, "Deformable DETR" wiki page,
+ * "Variants"):
+ *   grad_off_x = grad_loc_x * w,  grad_off_y = grad_loc_y * h
+ *   grad_box   = (sum grad_loc_x, sum grad_loc_y,
+ *                 sum grad_loc_x * off_x, sum grad_loc_y * off_y)
+ *   grad_z     = A * (grad_A - sum_j A_j grad_A_j)
+ * box [N,Lq,4], off like grad_loc, grad_box [N,Lq,4].  fp64.
+ */
+void ora_fused_chain_box(const double *grad_loc, const double *grad_attn, const double *attn,
+                         const double *box, const double *off, ora_dims d, double *grad_box,
+                         double *grad_off, double *grad_logits)
+{
+    const int64_t N = d.N, Lq = d.Lq, M = d.M, L = d.L, K = d.K;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t q = 0; q < Lq; ++q) {
+            const double *b = box + 4 * (n * Lq + q);
+            double gcx = 0.0, gcy = 0.0, gw = 0.0, gh = 0.0;
+            for (int64_t m = 0; m < M; ++m) {
+                const int64_t base = ((n * Lq + q) * M + m) * L * K;
+                double dot = 0.0;
+                for (int64_t j = 0; j < L * K; ++j)
+                    dot += attn[base + j] * grad_attn[base + j];
+                for (int64_t j = 0; j < L * K; ++j) {
+                    const int64_t i = base + j;
+                    grad_logits[i] = attn[i] * (grad_attn[i] - dot);
+                    grad_off[2 * i] = grad_loc[2 * i] * b[2];
+                    grad_off[2 * i + 1] = grad_loc[2 * i + 1] * b[3];
+                    gcx += grad_loc[2 * i];
+                    gcy += grad_loc[2 * i + 1];
+                    gw += grad_loc[2 * i] * off[2 * i];
+                    gh += grad_loc[2 * i + 1] * off[2 * i + 1];
+                }
+            }
+            double *gb = grad_box + 4 * (n * Lq + q);
+            gb[0] = gcx;
+            gb[1] = gcy;
+            gb[2] = gw;
+            gb[3] = gh;
+        }
+}
+
+/* fp64 box location map (finite-difference checks). */
+void ora_locations_box_f64(const double *box, const double *off, ora_dims d, double *loc)
+{
+    const int64_t N = d.N, Lq = d.Lq, M = d.M, L = d.L, K = d.K;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t q = 0; q < Lq; ++q)
+            for (int64_t j = 0; j < M * L * K; ++j) {
+                const int64_t i = (n * Lq + q) * M * L * K + j;
+                const double *b = box + 4 * (n * Lq + q);
+                loc[2 * i] = b[0] + off[2 * i] * b[2];
+                loc[2 * i + 1] = b[1] + off[2 * i + 1] * b[3];
+            }
+}
+
+/*
  * Per-sample index record, for bit-exact comparison of the cell arithmetic:
  * valid flag, the fp32 pixel coordinates (x, y) = (loc_x*W - 0.5,
  * loc_y*H - 0.5), the cell (x0, y0), and the flattened row of each of the

@@ -37,6 +37,7 @@ SIGNATURES = {
     "msda_forward": (INT, [P, INT, P, P, P, P, P, Dims, P]),
     "msda_forward_fused": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, Dims, P]),
     "msda_backward": (INT, [P, INT, P, P, P, P, P, P, P, P, Dims, P]),
+    "msda_backward_fused": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, P, P, Dims, P]),
     "msda_debug_sample_points": (INT, [P, P, P, Dims, P, P, P, P, P, P, P]),
 }
 

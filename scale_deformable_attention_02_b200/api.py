@@ -220,6 +220,53 @@ def msda_backward(value: torch.Tensor, spatial_shapes, level_start_index,
     return grad_value, grad_sampling_locations, grad_attention_weights
 
 
+def msda_backward_fused(value: torch.Tensor, spatial_shapes, level_start_index,
+                        reference_points: torch.Tensor, offsets: torch.Tensor,
+                        logits: torch.Tensor, grad_out: torch.Tensor,
+                        grad_value: torch.Tensor | None = None,
+                        grad_reference_points: torch.Tensor | None = None,
+                        grad_offsets: torch.Tensor | None = None,
+                        grad_logits: torch.Tensor | None = None,
+                        need_reference_grad: bool = True, need_offset_grad: bool = True,
+                        need_logit_grad: bool = True, stream=None):
+    """Gradients of msda_forward_fused with respect to the value map, the
+    reference points, the offsets and the logits.  Returns (grad_value,
+    grad_reference_points or None, grad_offsets or None, grad_logits or None)."""
+    dev = value.device
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    d = _value_dims(value, shapes, tuple(offsets.shape))
+    rdim = reference_points.shape[-1] if reference_points.dim() == 3 else -1
+    if rdim not in (2, 4):
+        raise ValueError("reference_points must be [N, Lq, 2] or [N, Lq, 4]")
+    _need(reference_points, "reference_points", (d.N, d.Lq, rdim), dev)
+    _need(offsets, "offsets", (d.N, d.Lq, d.M, d.L, d.K, 2), dev)
+    _need(logits, "logits", (d.N, d.Lq, d.M, d.L, d.K), dev)
+    _need(grad_out, "grad_out", (d.N, d.Lq, d.M * d.D), dev)
+    if not value.is_contiguous():
+        raise ValueError("value must be contiguous")
+    if grad_value is None:
+        grad_value = torch.empty(tuple(value.shape), device=dev, dtype=torch.float32)
+    _need(grad_value, "grad_value", tuple(value.shape), dev)
+    if grad_reference_points is None and need_reference_grad:
+        grad_reference_points = torch.empty_like(reference_points)
+    if grad_offsets is None and need_offset_grad:
+        grad_offsets = torch.empty_like(offsets)
+    if grad_logits is None and need_logit_grad:
+        grad_logits = torch.empty_like(logits)
+    if grad_reference_points is not None:
+        _need(grad_reference_points, "grad_reference_points", tuple(reference_points.shape), dev)
+    if grad_offsets is not None:
+        _need(grad_offsets, "grad_offsets", tuple(offsets.shape), dev)
+    if grad_logits is not None:
+        _need(grad_logits, "grad_logits", tuple(logits.shape), dev)
+    _check(_lib.load().msda_backward_fused(
+        _dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
+        _dptr(reference_points), int(rdim), _dptr(offsets), _dptr(logits), _dptr(grad_out),
+        _dptr(grad_value), _dptr(grad_reference_points), _dptr(grad_offsets),
+        _dptr(grad_logits), d, _stream_handle(dev, stream)), "msda_backward_fused")
+    return grad_value, grad_reference_points, grad_offsets, grad_logits
+
+
 def msda_debug_sample_points(spatial_shapes, level_start_index,
                              sampling_locations: torch.Tensor, stream=None) -> dict:
     """Per-sample cell record computed by the kernels' own cell arithmetic."""

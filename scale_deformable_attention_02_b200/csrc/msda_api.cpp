@@ -312,6 +312,77 @@ msda_status msda_backward(const void *value, msda_dtype value_dtype,
         msda::launch_backward(p, value_dtype == MSDA_BF16, pr.lanes, s));
 }
 
+msda_status msda_backward_fused(const void *value, msda_dtype value_dtype,
+                                const int64_t *spatial_shapes,
+                                const int64_t *level_start_index,
+                                const float *reference_points, int reference_dim,
+                                const float *offsets, const float *logits,
+                                const float *grad_out, float *grad_value,
+                                float *grad_reference_points, float *grad_offsets,
+                                float *grad_logits, msda_dims d, msda_stream_t stream)
+{
+    Problem pr;
+    msda_status st = check_dims(value_dtype, spatial_shapes, level_start_index, d, &pr);
+    if (st != MSDA_OK) return st;
+    if (reference_dim != 2 && reference_dim != 4) return MSDA_ERR_SHAPE;
+    if (d.D > 32) return MSDA_ERR_UNSUPPORTED;
+    if (pr.n_value > 0 && !grad_value) return MSDA_ERR_NULL;
+    if (pr.n_out > 0 && (!reference_points || !offsets || !logits || !grad_out))
+        return MSDA_ERR_NULL;
+    if (pr.n_out > 0 && pr.n_value > 0 && !value) return MSDA_ERR_NULL;
+    if (!aligned(value, 16) || !aligned(grad_out, 16) || !aligned(grad_value, 16) ||
+        !aligned(reference_points, 8) || !aligned(offsets, 8) || !aligned(logits, 4) ||
+        !aligned(grad_reference_points, 8) || !aligned(grad_offsets, 8) ||
+        !aligned(grad_logits, 4))
+        return MSDA_ERR_ALIGN;
+    const int64_t nq = pr.items / d.M;
+    const Span outs[] = {{grad_value, pr.n_value * 4},
+                         {grad_reference_points, nq * reference_dim * 4},
+                         {grad_offsets, pr.samples * 8},
+                         {grad_logits, pr.samples * 4}};
+    const Span ins[] = {{value, pr.n_value * pr.esz},
+                        {reference_points, nq * reference_dim * 4},
+                        {offsets, pr.samples * 8},
+                        {logits, pr.samples * 4},
+                        {grad_out, pr.n_out * 4}};
+    if (any_alias(outs, 4, ins, 5)) return MSDA_ERR_ALIAS;
+
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (pr.n_value > 0) {
+        st = cuda_status(cudaMemsetAsync(grad_value, 0, (size_t)pr.n_value * 4, s));
+        if (st != MSDA_OK) return st;
+    }
+    if (grad_reference_points && nq > 0) {
+        st = cuda_status(
+            cudaMemsetAsync(grad_reference_points, 0, (size_t)(nq * reference_dim) * 4, s));
+        if (st != MSDA_OK) return st;
+    }
+    if (pr.n_out == 0) return MSDA_OK;
+
+    msda::BwdParams p;
+    memset(&p, 0, sizeof p);
+    p.value = value;
+    p.ref = reference_points;
+    p.ref_dim = reference_dim;
+    p.off = offsets;
+    p.logits = logits;
+    p.grad_out = grad_out;
+    p.grad_value = grad_value;
+    p.grad_ref = grad_reference_points;
+    p.grad_off = grad_offsets;
+    p.grad_logits = grad_logits;
+    p.items = pr.items;
+    p.Lq = (int)d.Lq;
+    p.S = (int)d.S;
+    p.M = (int)d.M;
+    p.D = (int)d.D;
+    p.L = (int)d.L;
+    p.K = (int)d.K;
+    p.nchunks = pr.nchunks;
+    p.lv = pr.lv;
+    return cuda_status(msda::launch_backward_fused(p, value_dtype == MSDA_BF16, s));
+}
+
 msda_status msda_debug_sample_points(const int64_t *spatial_shapes,
                                      const int64_t *level_start_index,
                                      const float *sampling_locations, msda_dims d,

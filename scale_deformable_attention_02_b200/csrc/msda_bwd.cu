@@ -314,7 +314,7 @@ struct Lane4<__nv_bfloat16> {
 #define MSDA_BWD_MIN_CTAS 3
 #endif
 
-template <typename VT, int R, int P>
+template <typename VT, int R, int P, bool kFused>
 __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
     bwd_kernel(const __grid_constant__ BwdParams p)
 {
@@ -328,8 +328,10 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
     constexpr int kItems = 32 / P;
     constexpr int kStride = P + 2;
     static_assert(kBS <= P && P % kBS == 0, "a batch must stay inside the P sample slots");
+    constexpr int kNB = P / kBS;           // batches per item, at most
     __shared__ int2 ent[kWarps][kItems][4 * kStride];  // (row element offset | -1, A*w)
     __shared__ float4 smp[kWarps][kItems][P];          // (fx, fy, A*W, A*H)
+    __shared__ float4 smq[kWarps][kItems][kFused ? P : 1];  // fused: (A, off_x, off_y, -)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -354,16 +356,24 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
     const int64_t stride = (int64_t)gridDim.x * kWarps * kItems;
     int64_t item0 = ((int64_t)blockIdx.x * kWarps + warp) * kItems;
 
+    // this lane's sample inputs: (loc.x, loc.y, A), or fused (off.x, off.y, logit)
     float pl_x = 0.f, pl_y = 0.f, pa = 0.f;
     auto fetch = [&](int64_t i0) {
         const int64_t item = i0 + seg;
         pl_x = pl_y = pa = 0.f;
         if (jact && item < p.items) {
             const int64_t si = item * LK + j;
-            const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
-            pl_x = t.x;
-            pl_y = t.y;
-            pa = __ldcs(p.attn + si);
+            if constexpr (kFused) {
+                const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + si);
+                pl_x = o.x;
+                pl_y = o.y;
+                pa = __ldcs(p.logits + si);
+            } else {
+                const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
+                pl_x = t.x;
+                pl_y = t.y;
+                pa = __ldcs(p.attn + si);
+            }
         }
     };
     fetch(item0);
@@ -373,7 +383,31 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
         {
             const int64_t item = item0 + seg;
             const bool act = jact && item < p.items;
-            const float lx = pl_x, ly = pl_y, a = pa;
+            float lx = pl_x, ly = pl_y, a = pa;
+            if constexpr (kFused) {
+                // the fused forward's softmax and location map, bit for bit
+                const float ox = pl_x, oy = pl_y;
+                const float z = act ? pa : -INFINITY;
+                const float mx = seg_max<P>(z);
+                const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
+                const float sum = seg_sum<P>(e);
+                a = __fdiv_rn(e, sum);
+                lx = ly = 0.f;
+                if (act) {
+                    const int64_t nq = item / M;
+                    if (p.ref_dim == 2) {
+                        const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
+                        lx = __fadd_rn(r.x, __fdiv_rn(ox, (float)W));
+                        ly = __fadd_rn(r.y, __fdiv_rn(oy, (float)H));
+                    } else {
+                        const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
+                        const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
+                        lx = __fadd_rn(c.x, __fmul_rn(ox, s2.x));
+                        ly = __fadd_rn(c.y, __fmul_rn(oy, s2.y));
+                    }
+                }
+                smq[warp][seg][j] = make_float4(act ? a : 0.f, ox, oy, 0.f);
+            }
             fetch(item0 + stride);
             int2 e[4] = {{-1, 0}, {-1, 0}, {-1, 0}, {-1, 0}};
             float4 rec = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -424,7 +458,18 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
                 for (int i = 0; i < kVec; ++i) gv[i] = 0.f;
             }
             const int2 *en = ent[warp][it] + corner * kStride + sg;
-            for (int s0 = 0; s0 < LK; s0 += kBS) {
+            // fused: chain accumulators of this lane's (writer) samples
+            float ckA[kNB], ckdA[kNB];
+            float dpart = 0.f, rx = 0.f, ry = 0.f, rw = 0.f, rh = 0.f;
+            float2 bwh = make_float2(0.f, 0.f);
+            if constexpr (kFused) {
+                if (p.ref_dim == 4) bwh = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
+            }
+#pragma unroll
+            for (int bi = 0; bi < kNB; ++bi) {
+                ckA[bi] = ckdA[bi] = 0.f;
+                const int s0 = bi * kBS;
+                if (s0 >= LK) break;  // uniform
                 int2 e[kB];
                 Raw raw[kB];
 #pragma unroll
@@ -470,10 +515,57 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
                 }
                 if (corner == 0 && s < LK) {
                     const int64_t si = sbase + s;
-                    if (p.grad_attn) __stcs(p.grad_attn + si, q0);
-                    if (p.grad_loc)
-                        __stcs(reinterpret_cast<float2 *>(p.grad_loc) + si,
-                               make_float2(rec.z * q1, rec.w * q2));
+                    const float dlx = rec.z * q1, dly = rec.w * q2;  // d loc
+                    if constexpr (!kFused) {
+                        if (p.grad_attn) __stcs(p.grad_attn + si, q0);
+                        if (p.grad_loc)
+                            __stcs(reinterpret_cast<float2 *>(p.grad_loc) + si,
+                                   make_float2(dlx, dly));
+                    } else {
+                        const float4 r2 = smq[warp][it][s];  // (A, off_x, off_y, -)
+                        float2 goff;
+                        if (p.ref_dim == 2) {
+                            // loc = ref + off / W_l: d off = d loc / W_l = A * (sum dw t)
+                            goff = make_float2(r2.x * q1, r2.x * q2);
+                        } else {
+                            // loc = c + off * (w, h)
+                            goff = make_float2(dlx * bwh.x, dly * bwh.y);
+                            rw = fmaf(dlx, r2.y, rw);
+                            rh = fmaf(dly, r2.z, rh);
+                        }
+                        if (p.grad_off) __stcs(reinterpret_cast<float2 *>(p.grad_off) + si, goff);
+                        rx += dlx;
+                        ry += dly;
+                        dpart = fmaf(r2.x, q0, dpart);
+                        ckA[bi] = r2.x;
+                        ckdA[bi] = q0;
+                    }
+                }
+            }
+            if constexpr (kFused) {
+                // softmax Jacobian: d z_s = A_s (d A_s - sum_j A_j d A_j)
+                const float dot = warp_sum(dpart);
+#pragma unroll
+                for (int bi = 0; bi < kNB; ++bi) {
+                    const int s = bi * kBS + chunk * kSG + sg;
+                    if (corner == 0 && s < LK && p.grad_logits)
+                        __stcs(p.grad_logits + sbase + s, ckA[bi] * (ckdA[bi] - dot));
+                }
+                // reference gradient: sum over this head's samples, then over heads
+                rx = warp_sum(rx);
+                ry = warp_sum(ry);
+                if (p.ref_dim == 4) {
+                    rw = warp_sum(rw);
+                    rh = warp_sum(rh);
+                }
+                if (lane == 0 && p.grad_ref) {
+                    float *gr = p.grad_ref + nq * p.ref_dim;
+                    atomicAdd(gr, rx);
+                    atomicAdd(gr + 1, ry);
+                    if (p.ref_dim == 4) {
+                        atomicAdd(gr + 2, rw);
+                        atomicAdd(gr + 3, rh);
+                    }
                 }
             }
         }
@@ -481,24 +573,37 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
     }
 }
 
-template <typename VT, int R, int P>
+template <typename VT, int R, int P, bool kFused>
 cudaError_t launch_fast(const BwdParams &p, cudaStream_t stream)
 {
     constexpr int kRound = kWarps * (32 / P);
-    auto kern = bwd_kernel<VT, R, P>;
+    auto kern = bwd_kernel<VT, R, P, kFused>;
     const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kRound);
-    bwd_kernel<VT, R, P><<<(unsigned)ctas, kWarps * 32, 0, stream>>>(p);
+    bwd_kernel<VT, R, P, kFused><<<(unsigned)ctas, kWarps * 32, 0, stream>>>(p);
     return cudaGetLastError();
 }
 
-template <typename VT, int R>
+template <typename VT, int R, bool kFused = false>
 cudaError_t launch_fast_r(const BwdParams &p, cudaStream_t stream)
 {
     // P: a power of two >= L*K and >= the 8 samples of one batch
     const int LK = p.L * p.K;
-    if (LK <= 8) return launch_fast<VT, R, 8>(p, stream);
-    if (LK <= 16) return launch_fast<VT, R, 16>(p, stream);
-    return launch_fast<VT, R, 32>(p, stream);
+    if (LK <= 8) return launch_fast<VT, R, 8, kFused>(p, stream);
+    if (LK <= 16) return launch_fast<VT, R, 16, kFused>(p, stream);
+    return launch_fast<VT, R, 32, kFused>(p, stream);
+}
+
+template <typename VT>
+cudaError_t launch_bwd_fused_vt(const BwdParams &p, cudaStream_t stream)
+{
+    const int r4 = p.D / 4;
+    if (p.D % 4 != 0 || r4 > 8) return cudaErrorInvalidValue;
+    BwdParams q = p;
+    q.nchunks = r4;
+    if (r4 <= 1) return launch_fast_r<VT, 1, true>(q, stream);
+    if (r4 <= 2) return launch_fast_r<VT, 2, true>(q, stream);
+    if (r4 <= 4) return launch_fast_r<VT, 4, true>(q, stream);
+    return launch_fast_r<VT, 8, true>(q, stream);
 }
 
 template <typename VT>
@@ -529,6 +634,13 @@ cudaError_t launch_bwd_vt(const BwdParams &p, int R, cudaStream_t stream)
 }
 
 }  // namespace
+
+cudaError_t launch_backward_fused(const BwdParams &p, bool bf16, cudaStream_t stream)
+{
+    if (p.items == 0) return cudaSuccess;
+    return bf16 ? launch_bwd_fused_vt<__nv_bfloat16>(p, stream)
+                : launch_bwd_fused_vt<float>(p, stream);
+}
 
 cudaError_t launch_backward(const BwdParams &p, bool bf16, int lanes_per_row,
                             cudaStream_t stream)

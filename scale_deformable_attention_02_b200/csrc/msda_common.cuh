@@ -103,4 +103,21 @@ __device__ __forceinline__ float warp_sum(float v)
     return v;
 }
 
+// Max / sum over aligned segments of P lanes (P a power of two <= 32).
+template <int P>
+__device__ __forceinline__ float seg_max(float v)
+{
+#pragma unroll
+    for (int o = P / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
+    return v;
+}
+
+template <int P>
+__device__ __forceinline__ float seg_sum(float v)
+{
+#pragma unroll
+    for (int o = P / 2; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+    return v;
+}
+
 }  // namespace msda

@@ -45,22 +45,6 @@ struct __align__(16) Corner {
 // 512 bytes of zeros: the row that corners outside the level read.
 __device__ __align__(128) float4 kZeroRow[32] = {};
 
-template <int P>
-__device__ __forceinline__ float seg_max(float v)
-{
-#pragma unroll
-    for (int o = P / 2; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(kFull, v, o));
-    return v;
-}
-
-template <int P>
-__device__ __forceinline__ float seg_sum(float v)
-{
-#pragma unroll
-    for (int o = P / 2; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
-    return v;
-}
-
 // One 16-byte chunk of a value row: loaded raw (4 registers), widened to
 // float pairs only when it is consumed, so a batch of loads in flight costs
 // the same registers for fp32 and bf16.

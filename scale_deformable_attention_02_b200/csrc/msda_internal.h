@@ -34,12 +34,19 @@ struct FwdParams {
 
 struct BwdParams {
     const void *value;
-    const float *loc;
+    const float *loc;   // unfused inputs
     const float *attn;
+    const float *ref;     // fused inputs: [N,Lq,ref_dim]
+    const float *off;     // [N,Lq,M,L,K,2]
+    const float *logits;  // [N,Lq,M,L,K]
+    int ref_dim;
     const float *grad_out;
     float *grad_value;
-    float *grad_loc;   // nullable
-    float *grad_attn;  // nullable
+    float *grad_loc;     // nullable (unfused)
+    float *grad_attn;    // nullable (unfused)
+    float *grad_ref;     // nullable (fused; zeroed by the host, accumulated over heads)
+    float *grad_off;     // nullable (fused)
+    float *grad_logits;  // nullable (fused)
     int64_t items;
     int64_t chunk;  // items per CTA (set by the launcher)
     int Lq, S, M, D, L, K;
@@ -66,6 +73,9 @@ cudaError_t launch_forward(const FwdParams &p, bool bf16, bool fused, int lanes_
                            cudaStream_t stream);
 cudaError_t launch_backward(const BwdParams &p, bool bf16, int lanes_per_row,
                             cudaStream_t stream);
+// Backward of the fused forward (chained to ref, offsets and logits); needs
+// D <= 32 (returns cudaErrorInvalidValue otherwise, caught by the host checks).
+cudaError_t launch_backward_fused(const BwdParams &p, bool bf16, cudaStream_t stream);
 cudaError_t launch_sample_points(const PointsParams &p, cudaStream_t stream);
 
 }  // namespace msda

@@ -210,3 +210,25 @@ def test_binding_rejects_mismatched_tensors():
     attn = torch.zeros(1, 4, 2, 2, 3)  # K mismatch
     with pytest.raises(ValueError):
         msda_forward(value, wl.TINY_SHAPES, None, loc, attn)
+
+
+def test_backward_fused_argument_errors(lib):
+    pr = Prob()
+
+    def call(rdim=2, gv=None, gr=None, go=None, gz=None, ref=None, dims=None):
+        return lib.msda_backward_fused(fake(0), 0, pr.sp(), pr.st(), ref or fake(1), rdim,
+                                       fake(2), fake(3), fake(4), gv or fake(5), gr, go, gz,
+                                       dims or pr.dims, None)
+
+    assert call(rdim=3) == SHAPE
+    assert call(gv=fake(5, 8)) == ALIGN
+    assert call(gr=fake(6, 4)) == ALIGN
+    assert call(go=fake(2)) == ALIAS           # grad_offsets over the offsets
+    assert call(gz=fake(5, 64)) == ALIAS       # grad_logits inside grad_value
+    assert call(gr=fake(6), go=fake(6, 8)) == ALIAS
+    wide = Prob(D=64)
+    assert lib.msda_backward_fused(fake(0), 0, wide.sp(), wide.st(), fake(1), 2, fake(2),
+                                   fake(3), fake(4), fake(5), None, None, None, wide.dims,
+                                   None) == UNSUP
+    assert lib.msda_backward_fused(fake(0), 0, pr.sp(), pr.st(), None, 2, fake(2), fake(3),
+                                   fake(4), fake(5), None, None, None, pr.dims, None) == NULL

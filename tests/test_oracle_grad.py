@@ -146,13 +146,15 @@ def test_finite_differences_fused_chain():
         m[ii] -= h
         fd = (F(ref, off, p) - F(ref, off, m)) / (2 * h)
         assert abs(fd - g_z[ii]) <= 1e-6 * (1 + abs(fd))
-    if not skip.any():
-        for ii in np.ndindex(*ref.shape):
-            p, m = ref.copy(), ref.copy()
-            p[ii] += h
-            m[ii] -= h
-            fd = (F(p, off, z) - F(m, off, z)) / (2 * h)
-            assert abs(fd - g_ref[ii]) <= 1e-6 * (1 + abs(fd))
+    # moving the reference moves every sample by ~1e-5 px: only samples within
+    # 1e-4 px of a cell boundary could cross a kink
+    assert not _kink_mask(loc, shapes, 1e-4).any()
+    for ii in np.ndindex(*ref.shape):
+        p, m = ref.copy(), ref.copy()
+        p[ii] += h
+        m[ii] -= h
+        fd = (F(p, off, z) - F(m, off, z)) / (2 * h)
+        assert abs(fd - g_ref[ii]) <= 1e-6 * (1 + abs(fd))
 
 
 def test_backward_mass_bounds_the_sums():
@@ -168,3 +170,51 @@ def test_backward_mass_bounds_the_sums():
     g = np.abs(d["grad_out"])
     _, _, ga2, _, mga2 = oracle.backward(v, sh, loc, A, g, with_mass=True)
     np.testing.assert_allclose(ga2, mga2, rtol=1e-13, atol=0)
+
+
+def test_finite_differences_fused_chain_box():
+    """Box references (cx, cy, w, h): central differences of <g, F(box, off,
+    logits)> through loc = (cx, cy) + off * (w, h) match the chained
+    gradients, including those of the box itself."""
+    d = wl.make_random_problem(13, N=1, Lq=3, M=2, D=3, K=2,
+                               shapes=((6, 7), (3, 4)), offset_std=0.3)
+    shapes, value = d["spatial_shapes"], d["value"]
+    rng = np.random.default_rng(14)
+    box = np.concatenate([rng.uniform(0.3, 0.7, (1, 3, 2)), rng.uniform(0.1, 0.4, (1, 3, 2))],
+                         axis=-1)
+    off = d["offsets"].astype(np.float64)
+    z = d["logits"].astype(np.float64)
+    g = d["grad_out"].astype(np.float64)
+
+    def F(box_, off_, z_):
+        loc = oracle.locations_box_f64(box_, off_)
+        return np.sum(g * oracle.forward(value, shapes, loc, oracle.softmax(z_), loc_f32=False))
+
+    loc = oracle.locations_box_f64(box, off)
+    A = oracle.softmax(z)
+    _, gl, ga = oracle.backward(value, shapes, loc, A, g, loc_f32=False)
+    g_box, g_off, g_z = oracle.fused_chain_box(gl, ga, A, box, off)
+    skip = _kink_mask(loc, shapes, 1e-3)
+    h = 1e-6
+    for ii in np.ndindex(*off.shape[:-1]):
+        if skip[ii]:
+            continue
+        for c in range(2):
+            p_, m_ = off.copy(), off.copy()
+            p_[ii + (c,)] += h
+            m_[ii + (c,)] -= h
+            fd = (F(box, p_, z) - F(box, m_, z)) / (2 * h)
+            assert abs(fd - g_off[ii + (c,)]) <= 1e-6 * (1 + abs(fd))
+    for ii in np.ndindex(*z.shape):
+        p_, m_ = z.copy(), z.copy()
+        p_[ii] += h
+        m_[ii] -= h
+        fd = (F(box, off, p_) - F(box, off, m_)) / (2 * h)
+        assert abs(fd - g_z[ii]) <= 1e-6 * (1 + abs(fd))
+    assert not _kink_mask(loc, shapes, 1e-4).any()
+    for ii in np.ndindex(*box.shape):
+        p_, m_ = box.copy(), box.copy()
+        p_[ii] += h
+        m_[ii] -= h
+        fd = (F(p_, off, z) - F(m_, off, z)) / (2 * h)
+        assert abs(fd - g_box[ii]) <= 1e-6 * (1 + abs(fd))
