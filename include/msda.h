@@ -75,7 +75,10 @@ typedef enum {
     MSDA_ERR_ALIGN = 5,       /* a pointer or row size breaks the alignment rule */
     MSDA_ERR_ALIAS = 6,       /* an output overlaps an input or another output   */
     MSDA_ERR_UNSUPPORTED = 7, /* valid problem outside this build's limits       */
-    MSDA_ERR_CUDA = 8         /* the CUDA runtime reported an error at launch    */
+    MSDA_ERR_CUDA = 8,        /* the CUDA runtime reported an error at launch    */
+    MSDA_ERR_DEVICE_CHECK = 9 /* bounds-checked build only (msda_checked.h): a
+                                 gather or scatter fell outside the value map
+                                 and was skipped                                 */
 } msda_status;
 
 typedef enum {

@@ -4,12 +4,13 @@ The compute path is libmsda.so (hand-written sm_100a CUDA kernels behind the
 C ABI in include/msda.h); this package is its thin Python binding, plus the
 seeded synthetic workloads used by the tests and the benchmark.
 """
-from ._lib import LIB_PATH, MSDA_BF16, MSDA_F32
-from .api import (MsdaError, msda_backward, msda_backward_fused, msda_debug_sample_points,
-                  msda_forward, msda_forward_fused, msda_level_start_index)
+from ._lib import LIB_CHECKED_PATH, LIB_PATH, MSDA_BF16, MSDA_F32
+from .api import (MsdaError, checked_library, last_violation, msda_backward,
+                  msda_backward_fused, msda_debug_sample_points, msda_forward,
+                  msda_forward_fused, msda_level_start_index)
 
 __all__ = [
-    "LIB_PATH", "MSDA_BF16", "MSDA_F32", "MsdaError", "msda_backward", "msda_backward_fused",
-    "msda_debug_sample_points", "msda_forward", "msda_forward_fused",
-    "msda_level_start_index",
+    "LIB_CHECKED_PATH", "LIB_PATH", "MSDA_BF16", "MSDA_F32", "MsdaError", "checked_library",
+    "last_violation", "msda_backward", "msda_backward_fused", "msda_debug_sample_points",
+    "msda_forward", "msda_forward_fused", "msda_level_start_index",
 ]

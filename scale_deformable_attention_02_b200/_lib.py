@@ -1,6 +1,7 @@
 """ctypes view of libmsda.so (the C ABI in include/msda.h and
-include/msda_debug.h).  No fallback: if the library is missing or does not
-load, every call raises."""
+include/msda_debug.h) and of its bounds-checked build libmsda_checked.so
+(plus include/msda_checked.h).  No fallback: if a library is missing or does
+not load, every call raises."""
 from __future__ import annotations
 
 import ctypes
@@ -9,6 +10,7 @@ import threading
 
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmsda.so")
+LIB_CHECKED_PATH = os.path.join(PKG, "libmsda_checked.so")
 
 MSDA_F32 = 0
 MSDA_BF16 = 1
@@ -16,7 +18,7 @@ MSDA_BF16 = 1
 STATUS_NAMES = {
     0: "MSDA_OK", 1: "MSDA_ERR_NULL", 2: "MSDA_ERR_SHAPE", 3: "MSDA_ERR_LEVELS",
     4: "MSDA_ERR_DTYPE", 5: "MSDA_ERR_ALIGN", 6: "MSDA_ERR_ALIAS",
-    7: "MSDA_ERR_UNSUPPORTED", 8: "MSDA_ERR_CUDA",
+    7: "MSDA_ERR_UNSUPPORTED", 8: "MSDA_ERR_CUDA", 9: "MSDA_ERR_DEVICE_CHECK",
 }
 
 # Every function declared in include/*.h, with its ctypes signature.
@@ -41,26 +43,42 @@ SIGNATURES = {
     "msda_debug_sample_points": (INT, [P, P, P, Dims, P, P, P, P, P, P, P]),
 }
 
+# Only in libmsda_checked.so (include/msda_checked.h).
+CHECKED_SIGNATURES = {
+    "msda_checked_set_limit": (INT, [I64]),
+    "msda_checked_last_violation": (INT, [P, P]),
+}
+
 _lock = threading.Lock()
-_lib = None
+_libs: dict = {}
+_route = threading.local()  # .checked: this thread's binding calls use the checked build
 
 
-def load() -> ctypes.CDLL:
-    """Load libmsda.so (built in-tree by scale_deformable_attention_02_b200.build)."""
-    global _lib
+def _open(path: str, signatures: dict) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is not built; run `python -m "
+            "scale_deformable_attention_02_b200.build` (needs nvcc)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in signatures.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+def load(checked: bool | None = None) -> ctypes.CDLL:
+    """Load libmsda.so, or libmsda_checked.so when `checked` is true (None: the
+    library the calling thread routes to, see api.checked_library)."""
+    if checked is None:
+        checked = getattr(_route, "checked", False)
     with _lock:
-        if _lib is None:
-            if not os.path.exists(LIB_PATH):
-                raise RuntimeError(
-                    f"{LIB_PATH} is not built; run `python -m "
-                    "scale_deformable_attention_02_b200.build` (needs nvcc)")
-            lib = ctypes.CDLL(LIB_PATH)
-            for name, (res, args) in SIGNATURES.items():
-                fn = getattr(lib, name)
-                fn.restype = res
-                fn.argtypes = args
-            _lib = lib
-        return _lib
+        if checked not in _libs:
+            if checked:
+                _libs[True] = _open(LIB_CHECKED_PATH, {**SIGNATURES, **CHECKED_SIGNATURES})
+            else:
+                _libs[False] = _open(LIB_PATH, SIGNATURES)
+        return _libs[checked]
 
 
 def status_string(code: int) -> str:

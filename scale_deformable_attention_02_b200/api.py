@@ -4,7 +4,9 @@ Each function takes torch CUDA tensors, checks that their dtypes, devices,
 shapes and contiguity agree, allocates missing outputs with torch, and calls
 the C entry point of the same name on the current (or given) CUDA stream.
 Every step of the computation runs in libmsda.so's kernels; there is no
-other code path.
+other code path.  Inside `with checked_library():` the calls of the current
+thread go to libmsda_checked.so instead (the bounds-checked build of the same
+sources, include/msda_checked.h).
 
 Layouts (see include/msda.h):
   value [N,S,M,D] float32 | bfloat16, sampling_locations [N,Lq,M,L,K,2],
@@ -14,6 +16,7 @@ Layouts (see include/msda.h):
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 
 import numpy as np
@@ -23,14 +26,48 @@ from . import _lib
 
 
 class MsdaError(RuntimeError):
-    """A non-OK status from libmsda.so."""
+    """A non-OK status from libmsda.so.  For MSDA_ERR_DEVICE_CHECK (checked
+    build), `violations` and `first_element` say what the kernel skipped."""
 
     def __init__(self, status: int, where: str):
         self.status = int(status)
+        self.violations = 0
+        self.first_element = -1
         msg = f"{where}: {_lib.status_string(status)}"
         if self.status == 8:
             msg += f" (cudaError {_lib.load().msda_last_cuda_error()})"
+        if self.status == 9:
+            self.violations, self.first_element = last_violation()
+            msg += (f" ({self.violations} accesses skipped, first at value element "
+                    f"{self.first_element})")
         super().__init__(msg)
+
+
+@contextlib.contextmanager
+def checked_library(limit: int | None = None):
+    """Route this thread's calls to libmsda_checked.so, where every value-map
+    gather and grad_value scatter is bounds-checked on the device and a call
+    that skipped one raises MsdaError(MSDA_ERR_DEVICE_CHECK).  `limit` lowers
+    the bound to that many value elements (a test of the checks themselves)."""
+    lib = _lib.load(checked=True)
+    prev = getattr(_lib._route, "checked", False)
+    _lib._route.checked = True
+    if limit is not None:
+        lib.msda_checked_set_limit(int(limit))
+    try:
+        yield lib
+    finally:
+        if limit is not None:
+            lib.msda_checked_set_limit(-1)
+        _lib._route.checked = prev
+
+
+def last_violation() -> tuple[int, int]:
+    """(accesses skipped, first element index) of this thread's last
+    MSDA_ERR_DEVICE_CHECK in the checked build."""
+    cnt, first = ctypes.c_int64(0), ctypes.c_int64(-1)
+    _lib.load(checked=True).msda_checked_last_violation(ctypes.byref(cnt), ctypes.byref(first))
+    return cnt.value, first.value
 
 
 def _check(status: int, where: str) -> None:

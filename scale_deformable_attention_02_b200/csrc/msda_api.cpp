@@ -6,16 +6,21 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "msda.h"
 #include "msda_debug.h"
 #include "msda_internal.h"
+#ifdef MSDA_CHECKED
+#include "msda_checked.h"
+#endif
 
 namespace {
 
 using msda::Levels;
 using msda::kMaxLK;
 
-constexpr int kAbiVersion = 10000;  // 1.0.0
+constexpr int kAbiVersion = 10100;  // 1.1.0: MSDA_ERR_DEVICE_CHECK, msda_backward_fused
 constexpr int64_t kI32Max = 2147483647LL;
 constexpr int64_t kGuard = (int64_t)1 << 62;
 
@@ -120,6 +125,54 @@ msda_status cuda_status(cudaError_t e)
     return MSDA_ERR_CUDA;
 }
 
+#ifdef MSDA_CHECKED
+std::atomic<int64_t> g_check_limit{-1};
+thread_local int64_t g_violation_count = 0;
+thread_local int64_t g_violation_first = -1;
+#endif
+
+// The bounds-check fields of a launch: the value map's element count (or the
+// lowered test limit) and the device word.  Nothing in the default build.
+template <class Params>
+msda_status set_checks(Params *p, const Problem &pr)
+{
+    p->check_limit = pr.n_value;
+    p->check = nullptr;
+#ifdef MSDA_CHECKED
+    const int64_t lim = g_check_limit.load();
+    if (lim >= 0 && lim < p->check_limit) p->check_limit = lim;
+    p->check = msda::check_word();
+    if (!p->check) {
+        const cudaError_t e = cudaGetLastError();
+        return cuda_status(e != cudaSuccess ? e : cudaErrorUnknown);
+    }
+#endif
+    return MSDA_OK;
+}
+
+// Status of a launch.  The bounds-checked build also waits for the stream,
+// reads the device word, and clears it if the kernel recorded a violation.
+msda_status launched(cudaError_t e, cudaStream_t s)
+{
+    msda_status st = cuda_status(e);
+#ifdef MSDA_CHECKED
+    if (st != MSDA_OK) return st;
+    unsigned long long *dw = msda::check_word();
+    unsigned long long h[2] = {0, 0};
+    st = cuda_status(cudaMemcpyAsync(h, dw, sizeof h, cudaMemcpyDeviceToHost, s));
+    if (st == MSDA_OK) st = cuda_status(cudaStreamSynchronize(s));
+    if (st != MSDA_OK || h[0] == 0) return st;
+    g_violation_count = (int64_t)h[0];
+    g_violation_first = (int64_t)h[1];
+    st = cuda_status(cudaMemsetAsync(dw, 0, sizeof h, s));
+    if (st == MSDA_OK) st = cuda_status(cudaStreamSynchronize(s));
+    return st == MSDA_OK ? MSDA_ERR_DEVICE_CHECK : st;
+#else
+    (void)s;
+    return st;
+#endif
+}
+
 }  // namespace
 
 extern "C" {
@@ -137,6 +190,8 @@ const char *msda_status_string(msda_status status)
     case MSDA_ERR_ALIAS: return "MSDA_ERR_ALIAS: an output overlaps an input or another output";
     case MSDA_ERR_UNSUPPORTED: return "MSDA_ERR_UNSUPPORTED: outside this build's limits";
     case MSDA_ERR_CUDA: return "MSDA_ERR_CUDA: the CUDA runtime reported an error";
+    case MSDA_ERR_DEVICE_CHECK:
+        return "MSDA_ERR_DEVICE_CHECK: a bounds check skipped a value-map access";
     }
     return "MSDA_ERR_UNKNOWN";
 }
@@ -199,8 +254,9 @@ msda_status msda_forward(const void *value, msda_dtype value_dtype,
     p.K = (int)d.K;
     p.nchunks = pr.nchunks;
     p.lv = pr.lv;
-    return cuda_status(msda::launch_forward(p, value_dtype == MSDA_BF16, false, pr.lanes,
-                                            static_cast<cudaStream_t>(stream)));
+    if ((st = set_checks(&p, pr)) != MSDA_OK) return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return launched(msda::launch_forward(p, value_dtype == MSDA_BF16, false, pr.lanes, s), s);
 }
 
 msda_status msda_forward_fused(const void *value, msda_dtype value_dtype,
@@ -252,8 +308,9 @@ msda_status msda_forward_fused(const void *value, msda_dtype value_dtype,
     p.K = (int)d.K;
     p.nchunks = pr.nchunks;
     p.lv = pr.lv;
-    return cuda_status(msda::launch_forward(p, value_dtype == MSDA_BF16, true, pr.lanes,
-                                            static_cast<cudaStream_t>(stream)));
+    if ((st = set_checks(&p, pr)) != MSDA_OK) return st;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    return launched(msda::launch_forward(p, value_dtype == MSDA_BF16, true, pr.lanes, s), s);
 }
 
 msda_status msda_backward(const void *value, msda_dtype value_dtype,
@@ -308,8 +365,8 @@ msda_status msda_backward(const void *value, msda_dtype value_dtype,
     p.K = (int)d.K;
     p.nchunks = pr.nchunks;
     p.lv = pr.lv;
-    return cuda_status(
-        msda::launch_backward(p, value_dtype == MSDA_BF16, pr.lanes, s));
+    if ((st = set_checks(&p, pr)) != MSDA_OK) return st;
+    return launched(msda::launch_backward(p, value_dtype == MSDA_BF16, pr.lanes, s), s);
 }
 
 msda_status msda_backward_fused(const void *value, msda_dtype value_dtype,
@@ -380,7 +437,8 @@ msda_status msda_backward_fused(const void *value, msda_dtype value_dtype,
     p.K = (int)d.K;
     p.nchunks = pr.nchunks;
     p.lv = pr.lv;
-    return cuda_status(msda::launch_backward_fused(p, value_dtype == MSDA_BF16, s));
+    if ((st = set_checks(&p, pr)) != MSDA_OK) return st;
+    return launched(msda::launch_backward_fused(p, value_dtype == MSDA_BF16, s), s);
 }
 
 msda_status msda_debug_sample_points(const int64_t *spatial_shapes,
@@ -418,5 +476,20 @@ msda_status msda_debug_sample_points(const int64_t *spatial_shapes,
     p.lv = pr.lv;
     return cuda_status(msda::launch_sample_points(p, static_cast<cudaStream_t>(stream)));
 }
+
+#ifdef MSDA_CHECKED
+msda_status msda_checked_set_limit(int64_t value_elements)
+{
+    g_check_limit.store(value_elements < 0 ? -1 : value_elements);
+    return MSDA_OK;
+}
+
+msda_status msda_checked_last_violation(int64_t *count, int64_t *first_element)
+{
+    if (count) *count = g_violation_count;
+    if (first_element) *first_element = g_violation_first;
+    return MSDA_OK;
+}
+#endif
 
 }  // extern "C"

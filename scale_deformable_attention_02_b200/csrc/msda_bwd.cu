@@ -214,7 +214,8 @@ __global__ void __launch_bounds__(kWarps * 32)
                 for (int ci = 0; ci < kCpl; ++ci) {
                     const CornerB e = corners[warp][s * 4 + cslot * kCpl + ci];
                     float t = 0.f;
-                    if (e.off >= 0 && chunk_ok) {
+                    if (e.off >= 0 && chunk_ok &&
+                        msda_in_map(p.check, p.check_limit, rowbase + e.off, kVec)) {
                         float x[kVec];
                         Chunk<VT>::load(vbase + e.off, x);
 #pragma unroll
@@ -439,7 +440,8 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
             const int64_t n = nq / p.Lq;
             const int64_t sbase = itm * LK;
             const int64_t mapoff = (n * p.S * M + m) * (int64_t)D;
-            const VT *vb = static_cast<const VT *>(p.value) + mapoff + lane_elem;
+            const int64_t vbe = mapoff + lane_elem;
+            const VT *vb = static_cast<const VT *>(p.value) + vbe;
             float *gvb = p.grad_value + mapoff + chunk * kVec;
             float gv[kVec];
             if (chunk_ok) {
@@ -475,6 +477,9 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
 #pragma unroll
                 for (int b = 0; b < kB; ++b) {
                     e[b] = en[s0 + b * kSG];  // sample s0 + b*kSG + sg, this lane's corner
+                    // bounds-checked build: a skipped corner reads zeros and scatters nothing
+                    if (e[b].x >= 0 && !msda_in_map(p.check, p.check_limit, vbe + e[b].x, kVec))
+                        e[b].x = -1;
                     if (e[b].x >= 0) raw[b] = Lane4<VT>::load(vb + e[b].x);
                 }
                 float t[kB];

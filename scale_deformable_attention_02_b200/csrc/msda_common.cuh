@@ -39,6 +39,29 @@ __device__ __forceinline__ bool msda_cell(float lx, float ly, int H, int W, floa
     return true;
 }
 
+// Bounds check of one access to the value map (or to grad_value, which has
+// the same layout): value elements [first, first + count) against [0, limit).
+// Only the bounds-checked build (-DMSDA_CHECKED) tests anything: there an
+// access outside the range is to be skipped by the caller, and it is counted
+// in check[0] with the first one's element index in check[1].  In the default
+// build every index is in range by construction (cells come from msda_cell
+// and msda_row, dims are validated on the host) and this is the constant true.
+__device__ __forceinline__ bool msda_in_map(unsigned long long *check, int64_t limit,
+                                            int64_t first, int count)
+{
+#ifdef MSDA_CHECKED
+    if (first >= 0 && first + count <= limit) return true;
+    if (check && atomicAdd(check, 1ull) == 0ull) check[1] = (unsigned long long)first;
+    return false;
+#else
+    (void)check;
+    (void)limit;
+    (void)first;
+    (void)count;
+    return true;
+#endif
+}
+
 // Value row of pixel (yy, xx) on a level, or -1 outside the level (zero
 // padding: such a corner contributes nothing).
 __device__ __forceinline__ int msda_row(int start, int H, int W, int yy, int xx)

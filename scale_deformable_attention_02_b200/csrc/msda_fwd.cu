@@ -211,8 +211,17 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
                 for (int b = 0; b < kB; ++b) {
                     const int t = t0 + b * kSlots + slot;  // pair t = (sample t/4, corner t%4)
                     const Corner e = ent[(t & 3) * kStride + (t >> 2)];
+                    const char *row = e.row;
                     w[b] = e.w.x;
-                    raw[b] = __ldg(reinterpret_cast<const uint4 *>(e.row + lane_off));
+                    if (row != reinterpret_cast<const char *>(kZeroRow) &&
+                        !msda_in_map(p.check, p.check_limit,
+                                     (row - static_cast<const char *>(p.value) + lane_off) /
+                                         (int64_t)sizeof(VT),
+                                     16 / (int)sizeof(VT))) {
+                        row = reinterpret_cast<const char *>(kZeroRow);  // skipped: reads zeros
+                        w[b] = 0.f;
+                    }
+                    raw[b] = __ldg(reinterpret_cast<const uint4 *>(row + lane_off));
                 }
 #pragma unroll
                 for (int b = 0; b < kB; ++b) {
@@ -445,8 +454,8 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
             const int m = (int)(itm % M);
             const int64_t nq = itm / M;
             const int64_t n = nq / p.Lq;
-            const VT *vb = static_cast<const VT *>(p.value) + (n * p.S * M + m) * (int64_t)D +
-                           lane_elem;
+            const int64_t vbe = (n * p.S * M + m) * (int64_t)D + lane_elem;
+            const VT *vb = static_cast<const VT *>(p.value) + vbe;
             const int2 *en = ent[warp][it];
             float2 acc[kNP];
 #pragma unroll
@@ -458,6 +467,8 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
                 for (int b = 0; b < kB; ++b) {
                     const int t = t0 + b * kSlots + slot;  // pair (sample t/4, corner t%4)
                     e[b] = en[(t & 3) * kStride + (t >> 2)];
+                    if (e[b].x >= 0 && !msda_in_map(p.check, p.check_limit, vbe + e[b].x, EPL))
+                        e[b].x = -1;  // bounds-checked build: skipped, reads as zero
                     if (e[b].x >= 0) raw[b] = LL::load(vb + e[b].x);
                 }
 #pragma unroll

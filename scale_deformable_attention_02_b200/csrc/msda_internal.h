@@ -30,6 +30,11 @@ struct FwdParams {
     int Lq, S, M, D, L, K;
     int nchunks;  // 16-byte chunks per value row
     Levels lv;
+    // bounds-checked build only (-DMSDA_CHECKED): value elements an access
+    // may touch, and the device word counting skipped accesses
+    // ([0] = count, [1] = first element index)
+    int64_t check_limit;
+    unsigned long long *check;
 };
 
 struct BwdParams {
@@ -52,6 +57,11 @@ struct BwdParams {
     int Lq, S, M, D, L, K;
     int nchunks;
     Levels lv;
+    // bounds-checked build only (-DMSDA_CHECKED): value elements an access
+    // may touch, and the device word counting skipped accesses
+    // ([0] = count, [1] = first element index)
+    int64_t check_limit;
+    unsigned long long *check;
 };
 
 struct PointsParams {
@@ -77,5 +87,12 @@ cudaError_t launch_backward(const BwdParams &p, bool bf16, int lanes_per_row,
 // D <= 32 (returns cudaErrorInvalidValue otherwise, caught by the host checks).
 cudaError_t launch_backward_fused(const BwdParams &p, bool bf16, cudaStream_t stream);
 cudaError_t launch_sample_points(const PointsParams &p, cudaStream_t stream);
+
+#ifdef MSDA_CHECKED
+// The current device's check word (two zero-initialised 64-bit counters in a
+// file-scope __device__ array), or nullptr if the runtime cannot give its
+// address.
+unsigned long long *check_word();
+#endif
 
 }  // namespace msda

@@ -1,7 +1,8 @@
-"""The C ABI on the host: the library loads, exports every symbol the headers
-declare, computes the level metadata, and rejects bad arguments with the
-documented status codes before any device work.  CPU only: every call here
-returns before touching CUDA (pointers are fake and never dereferenced)."""
+"""The C ABI on the host: both builds of the library (libmsda.so and the
+bounds-checked libmsda_checked.so) load, export exactly the symbols their
+headers declare, compute the level metadata, and reject bad arguments with
+the documented status codes before any device work.  CPU only: every call
+here returns before touching CUDA (pointers are fake and never dereferenced)."""
 import ctypes
 import glob
 import os
@@ -19,26 +20,36 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 OK, NULL, SHAPE, LEVELS, DTYPE, ALIGN, ALIAS, UNSUP = range(8)
 
+PRODUCT_HEADERS = ("msda.h", "msda_debug.h")
+CHECKED_HEADERS = PRODUCT_HEADERS + ("msda_checked.h",)
 
-@pytest.fixture(scope="module")
-def lib():
+
+@pytest.fixture(scope="module", params=[False, True], ids=["libmsda", "libmsda_checked"])
+def lib(request):
     msda_build.build()
-    return _lib.load()
+    return _lib.load(checked=request.param)
 
 
-def declared_functions():
+def declared_functions(headers=PRODUCT_HEADERS):
     names = []
-    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
-        text = open(h).read()
+    for h in headers:
+        text = open(os.path.join(ROOT, "include", h)).read()
         names += re.findall(r"^MSDA_API\s+[\w\s\*]*?\b(msda_\w+)\s*\(", text, flags=re.M)
     return sorted(set(names))
 
 
+def test_every_header_is_covered():
+    assert sorted(os.path.basename(h) for h in glob.glob(os.path.join(ROOT, "include", "*.h"))) \
+        == sorted(CHECKED_HEADERS)
+
+
 def test_headers_declare_the_entry_points():
     names = declared_functions()
-    for must in ("msda_forward", "msda_forward_fused", "msda_backward",
+    for must in ("msda_forward", "msda_forward_fused", "msda_backward", "msda_backward_fused",
                  "msda_level_start_index", "msda_status_string", "msda_debug_sample_points"):
         assert must in names
+    assert set(declared_functions(CHECKED_HEADERS)) - set(names) == {
+        "msda_checked_set_limit", "msda_checked_last_violation"}
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -47,18 +58,45 @@ def test_library_exports_every_declared_symbol(lib):
         assert name in _lib.SIGNATURES, f"binding lacks {name}"
 
 
-def test_library_exports_nothing_else():
+@pytest.mark.parametrize("path,headers", [(_lib.LIB_PATH, PRODUCT_HEADERS),
+                                          (_lib.LIB_CHECKED_PATH, CHECKED_HEADERS)])
+def test_library_exports_nothing_else(path, headers):
     import subprocess
-    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True,
+    msda_build.build()
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True,
                          text=True, check=True).stdout
     exported = sorted({ln.split()[-1] for ln in out.splitlines() if " T " in ln})
-    assert exported == declared_functions()
+    assert exported == declared_functions(headers)
+    for name in exported:
+        assert name in _lib.SIGNATURES or name in _lib.CHECKED_SIGNATURES
 
 
 def test_status_strings_and_version(lib):
     for code, name in _lib.STATUS_NAMES.items():
         assert lib.msda_status_string(code).decode().startswith(name)
-    assert lib.msda_abi_version() == 10000
+    assert lib.msda_abi_version() == 10100
+
+
+def test_checked_build_host_calls():
+    """The checked build's own entry points: a fresh thread has seen no
+    violation; setting and restoring the limit needs no device."""
+    import threading
+    msda_build.build()
+    lib = _lib.load(checked=True)
+    out = {}
+
+    def fresh():
+        cnt, first = ctypes.c_int64(7), ctypes.c_int64(7)
+        out["st"] = lib.msda_checked_last_violation(ctypes.byref(cnt), ctypes.byref(first))
+        out["v"] = (cnt.value, first.value)
+        out["null"] = lib.msda_checked_last_violation(None, None)
+
+    t = threading.Thread(target=fresh)
+    t.start()
+    t.join()
+    assert out == {"st": OK, "v": (0, -1), "null": OK}
+    assert lib.msda_checked_set_limit(1000) == OK
+    assert lib.msda_checked_set_limit(-5) == OK
 
 
 @pytest.mark.parametrize("shapes", [wl.TINY_SHAPES, wl.ENCODER_SHAPES, wl.STRESS_SHAPES,
