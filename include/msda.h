@@ -44,9 +44,10 @@
  *  - Every argument check happens before any device work: a call that
  *    returns an error has launched nothing and written nothing.
  *
- * Limits of this build: 1 <= L*K <= 32; D*sizeof(value element) a multiple
- * of 16 bytes and at most 512 bytes; S*M*D and N*Lq*M*L*K*2 below 2^31.
- * Calls beyond them return MSDA_ERR_UNSUPPORTED.  N = 0 or Lq = 0 is a valid
+ * Limits of this build: L <= 32 and 1 <= L*K <= 128; D*sizeof(value
+ * element) a multiple of 16 bytes (else MSDA_ERR_ALIGN) and at most 512
+ * bytes; H_l, W_l, S*M*D below 2^31 (row offsets inside one batch entry are
+ * 32-bit).  Other calls beyond them return MSDA_ERR_UNSUPPORTED.  N = 0 or Lq = 0 is a valid
  * empty problem (the backward then only zeroes grad_value).
  */
 #ifndef MSDA_H
@@ -240,8 +241,9 @@ MSDA_API msda_status msda_backward(const void *value, msda_dtype value_dtype,
  *   grad_offsets            NULL or device [N,Lq,M,L,K,2] fp32 (written)
  *   grad_logits             NULL or device [N,Lq,M,L,K] fp32 (written)
  *
- * Limits: D <= 32 (MSDA_ERR_UNSUPPORTED otherwise).  Errors: as
- * msda_forward_fused; every gradient buffer is an output for the alias check.
+ * Limits: D <= 32 for either value dtype (MSDA_ERR_UNSUPPORTED otherwise).
+ * Errors: as msda_forward_fused; every gradient buffer is an output for the
+ * alias check.
  */
 MSDA_API msda_status msda_backward_fused(const void *value, msda_dtype value_dtype,
                                          const int64_t *spatial_shapes,
@@ -252,6 +254,69 @@ MSDA_API msda_status msda_backward_fused(const void *value, msda_dtype value_dty
                                          float *grad_reference_points, float *grad_offsets,
                                          float *grad_logits, msda_dims dims,
                                          msda_stream_t stream);
+
+/*
+ * Deformable groups ("Deformable Attention" glossary page: heads grouped
+ * into deformable groups that share the same set of sampled keys, with
+ * different projection weights).  The M heads form `groups` groups of
+ * Hg = M/groups consecutive heads (head m is in group m / Hg); the heads of a
+ * group sample the same locations, each with its own attention weights and
+ * its own value channels.  The four calls below are msda_forward,
+ * msda_forward_fused, msda_backward and msda_backward_fused with every
+ * per-location tensor indexed by group instead of head:
+ *
+ *   sampling_locations, offsets,
+ *   sampling_locations_out, grad_sampling_locations, grad_offsets
+ *                                 [N, Lq, groups, L, K, 2]
+ *   attention_weights, logits, attention_weights_out, grad_attention_weights,
+ *   grad_logits                   [N, Lq, M, L, K]      (per head, unchanged)
+ *
+ * The fused forward writes each group's locations once.  In the backward the
+ * Hg heads of a group add into one location gradient: grad_sampling_locations
+ * and grad_offsets are then zeroed by the call and accumulated with atomics
+ * (groups < M; with groups == M they are written, as in the ungrouped calls,
+ * which these equal).
+ * Errors: as the ungrouped calls, plus MSDA_ERR_SHAPE unless
+ * 1 <= groups <= M and groups divides M.
+ */
+MSDA_API msda_status msda_forward_grouped(const void *value, msda_dtype value_dtype,
+                                          const int64_t *spatial_shapes,
+                                          const int64_t *level_start_index,
+                                          const float *sampling_locations,
+                                          const float *attention_weights, float *out,
+                                          msda_dims dims, int64_t groups, msda_stream_t stream);
+
+MSDA_API msda_status msda_forward_fused_grouped(const void *value, msda_dtype value_dtype,
+                                                const int64_t *spatial_shapes,
+                                                const int64_t *level_start_index,
+                                                const float *reference_points,
+                                                int reference_dim, const float *offsets,
+                                                const float *logits, float *out,
+                                                float *sampling_locations_out,
+                                                float *attention_weights_out, msda_dims dims,
+                                                int64_t groups, msda_stream_t stream);
+
+MSDA_API msda_status msda_backward_grouped(const void *value, msda_dtype value_dtype,
+                                           const int64_t *spatial_shapes,
+                                           const int64_t *level_start_index,
+                                           const float *sampling_locations,
+                                           const float *attention_weights,
+                                           const float *grad_out, float *grad_value,
+                                           float *grad_sampling_locations,
+                                           float *grad_attention_weights, msda_dims dims,
+                                           int64_t groups, msda_stream_t stream);
+
+MSDA_API msda_status msda_backward_fused_grouped(const void *value, msda_dtype value_dtype,
+                                                 const int64_t *spatial_shapes,
+                                                 const int64_t *level_start_index,
+                                                 const float *reference_points,
+                                                 int reference_dim, const float *offsets,
+                                                 const float *logits, const float *grad_out,
+                                                 float *grad_value,
+                                                 float *grad_reference_points,
+                                                 float *grad_offsets, float *grad_logits,
+                                                 msda_dims dims, int64_t groups,
+                                                 msda_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -40,6 +40,11 @@ SIGNATURES = {
     "msda_forward_fused": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, Dims, P]),
     "msda_backward": (INT, [P, INT, P, P, P, P, P, P, P, P, Dims, P]),
     "msda_backward_fused": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, P, P, Dims, P]),
+    "msda_forward_grouped": (INT, [P, INT, P, P, P, P, P, Dims, I64, P]),
+    "msda_forward_fused_grouped": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, Dims, I64, P]),
+    "msda_backward_grouped": (INT, [P, INT, P, P, P, P, P, P, P, P, Dims, I64, P]),
+    "msda_backward_fused_grouped": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, P, P, Dims, I64,
+                                          P]),
     "msda_debug_sample_points": (INT, [P, P, P, Dims, P, P, P, P, P, P, P]),
 }
 

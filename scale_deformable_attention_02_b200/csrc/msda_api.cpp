@@ -64,7 +64,8 @@ bool any_alias(const Span *outs, int nout, const Span *ins, int nin)
 // Validated problem: element counts and launch-side metadata.
 struct Problem {
     int64_t items;    // N*Lq*M
-    int64_t samples;  // N*Lq*M*L*K
+    int64_t samples;  // N*Lq*M*L*K: per-head tensors (weights, logits)
+    int64_t lsamples; // N*Lq*G*L*K: per-group tensors (locations, offsets)
     int64_t n_value;  // N*S*M*D
     int64_t n_out;    // N*Lq*M*D
     int esz;          // value element size
@@ -81,7 +82,8 @@ msda_status check_dims(msda_dtype dt, const int64_t *shapes, const int64_t *star
     if (dt != MSDA_F32 && dt != MSDA_BF16) return MSDA_ERR_DTYPE;
     if (d.N < 0 || d.Lq < 0 || d.S < 0 || d.M < 1 || d.D < 1 || d.L < 1 || d.K < 1)
         return MSDA_ERR_SHAPE;
-    if (d.L > kMaxLK || d.K > kMaxLK || d.L * d.K > kMaxLK) return MSDA_ERR_UNSUPPORTED;
+    if (d.L > msda::kMaxLevels || d.K > kMaxLK || d.L * d.K > kMaxLK)
+        return MSDA_ERR_UNSUPPORTED;
     memset(&pr->lv, 0, sizeof pr->lv);
     int64_t acc = 0;
     for (int64_t l = 0; l < d.L; ++l) {
@@ -116,6 +118,31 @@ msda_status check_dims(msda_dtype dt, const int64_t *shapes, const int64_t *star
     while (lanes < pr->nchunks) lanes <<= 1;
     pr->lanes = lanes;
     return MSDA_OK;
+}
+
+// Deformable groups: G groups of M/G consecutive heads share one set of
+// sampling locations (G = M: every head has its own).
+msda_status check_groups(const msda_dims &d, int64_t G, Problem *pr)
+{
+    if (G < 1 || G > d.M || d.M % G != 0) return MSDA_ERR_SHAPE;
+    pr->lsamples = pr->samples / d.M * G;
+    return MSDA_OK;
+}
+
+template <class Params>
+void set_dims(Params *p, const msda_dims &d, int64_t G, const Problem &pr)
+{
+    p->items = pr.items;
+    p->Lq = (int)d.Lq;
+    p->S = (int)d.S;
+    p->M = (int)d.M;
+    p->D = (int)d.D;
+    p->L = (int)d.L;
+    p->K = (int)d.K;
+    p->G = (int)G;
+    p->Hg = (int)(d.M / G);
+    p->nchunks = pr.nchunks;
+    p->lv = pr.lv;
 }
 
 msda_status cuda_status(cudaError_t e)
@@ -218,14 +245,19 @@ msda_status msda_level_start_index(const int64_t *spatial_shapes, int64_t L,
     return MSDA_OK;
 }
 
-msda_status msda_forward(const void *value, msda_dtype value_dtype,
-                         const int64_t *spatial_shapes, const int64_t *level_start_index,
-                         const float *sampling_locations, const float *attention_weights,
-                         float *out, msda_dims d, msda_stream_t stream)
+}  // extern "C"
+
+namespace {
+
+msda_status forward_impl(const void *value, msda_dtype value_dtype, const int64_t *spatial_shapes,
+                         const int64_t *level_start_index, const float *sampling_locations,
+                         const float *attention_weights, float *out, msda_dims d, int64_t G,
+                         msda_stream_t stream)
 {
     Problem pr;
     msda_status st = check_dims(value_dtype, spatial_shapes, level_start_index, d, &pr);
     if (st != MSDA_OK) return st;
+    if ((st = check_groups(d, G, &pr)) != MSDA_OK) return st;
     if (pr.n_out > 0 && (!sampling_locations || !attention_weights || !out))
         return MSDA_ERR_NULL;
     if (pr.n_out > 0 && pr.n_value > 0 && !value) return MSDA_ERR_NULL;
@@ -234,7 +266,7 @@ msda_status msda_forward(const void *value, msda_dtype value_dtype,
         return MSDA_ERR_ALIGN;
     const Span outs[] = {{out, pr.n_out * 4}};
     const Span ins[] = {{value, pr.n_value * pr.esz},
-                        {sampling_locations, pr.samples * 8},
+                        {sampling_locations, pr.lsamples * 8},
                         {attention_weights, pr.samples * 4}};
     if (any_alias(outs, 1, ins, 3)) return MSDA_ERR_ALIAS;
     if (pr.n_out == 0) return MSDA_OK;
@@ -245,31 +277,23 @@ msda_status msda_forward(const void *value, msda_dtype value_dtype,
     p.loc = sampling_locations;
     p.attn = attention_weights;
     p.out = out;
-    p.items = pr.items;
-    p.Lq = (int)d.Lq;
-    p.S = (int)d.S;
-    p.M = (int)d.M;
-    p.D = (int)d.D;
-    p.L = (int)d.L;
-    p.K = (int)d.K;
-    p.nchunks = pr.nchunks;
-    p.lv = pr.lv;
+    set_dims(&p, d, G, pr);
     if ((st = set_checks(&p, pr)) != MSDA_OK) return st;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     return launched(msda::launch_forward(p, value_dtype == MSDA_BF16, false, pr.lanes, s), s);
 }
 
-msda_status msda_forward_fused(const void *value, msda_dtype value_dtype,
-                               const int64_t *spatial_shapes,
-                               const int64_t *level_start_index,
+msda_status forward_fused_impl(const void *value, msda_dtype value_dtype,
+                               const int64_t *spatial_shapes, const int64_t *level_start_index,
                                const float *reference_points, int reference_dim,
                                const float *offsets, const float *logits, float *out,
                                float *sampling_locations_out, float *attention_weights_out,
-                               msda_dims d, msda_stream_t stream)
+                               msda_dims d, int64_t G, msda_stream_t stream)
 {
     Problem pr;
     msda_status st = check_dims(value_dtype, spatial_shapes, level_start_index, d, &pr);
     if (st != MSDA_OK) return st;
+    if ((st = check_groups(d, G, &pr)) != MSDA_OK) return st;
     if (reference_dim != 2 && reference_dim != 4) return MSDA_ERR_SHAPE;
     if (pr.n_out > 0 && (!reference_points || !offsets || !logits || !out))
         return MSDA_ERR_NULL;
@@ -280,11 +304,11 @@ msda_status msda_forward_fused(const void *value, msda_dtype value_dtype,
         return MSDA_ERR_ALIGN;
     const int64_t nq = pr.items / d.M;
     const Span outs[] = {{out, pr.n_out * 4},
-                         {sampling_locations_out, pr.samples * 8},
+                         {sampling_locations_out, pr.lsamples * 8},
                          {attention_weights_out, pr.samples * 4}};
     const Span ins[] = {{value, pr.n_value * pr.esz},
                         {reference_points, nq * reference_dim * 4},
-                        {offsets, pr.samples * 8},
+                        {offsets, pr.lsamples * 8},
                         {logits, pr.samples * 4}};
     if (any_alias(outs, 3, ins, 4)) return MSDA_ERR_ALIAS;
     if (pr.n_out == 0) return MSDA_OK;
@@ -299,30 +323,23 @@ msda_status msda_forward_fused(const void *value, msda_dtype value_dtype,
     p.out = out;
     p.loc_out = sampling_locations_out;
     p.attn_out = attention_weights_out;
-    p.items = pr.items;
-    p.Lq = (int)d.Lq;
-    p.S = (int)d.S;
-    p.M = (int)d.M;
-    p.D = (int)d.D;
-    p.L = (int)d.L;
-    p.K = (int)d.K;
-    p.nchunks = pr.nchunks;
-    p.lv = pr.lv;
+    set_dims(&p, d, G, pr);
     if ((st = set_checks(&p, pr)) != MSDA_OK) return st;
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     return launched(msda::launch_forward(p, value_dtype == MSDA_BF16, true, pr.lanes, s), s);
 }
 
-msda_status msda_backward(const void *value, msda_dtype value_dtype,
+msda_status backward_impl(const void *value, msda_dtype value_dtype,
                           const int64_t *spatial_shapes, const int64_t *level_start_index,
                           const float *sampling_locations, const float *attention_weights,
                           const float *grad_out, float *grad_value,
                           float *grad_sampling_locations, float *grad_attention_weights,
-                          msda_dims d, msda_stream_t stream)
+                          msda_dims d, int64_t G, msda_stream_t stream)
 {
     Problem pr;
     msda_status st = check_dims(value_dtype, spatial_shapes, level_start_index, d, &pr);
     if (st != MSDA_OK) return st;
+    if ((st = check_groups(d, G, &pr)) != MSDA_OK) return st;
     if (pr.n_value > 0 && !grad_value) return MSDA_ERR_NULL;
     if (pr.n_out > 0 && (!sampling_locations || !attention_weights || !grad_out))
         return MSDA_ERR_NULL;
@@ -332,10 +349,10 @@ msda_status msda_backward(const void *value, msda_dtype value_dtype,
         !aligned(grad_sampling_locations, 8) || !aligned(grad_attention_weights, 4))
         return MSDA_ERR_ALIGN;
     const Span outs[] = {{grad_value, pr.n_value * 4},
-                         {grad_sampling_locations, pr.samples * 8},
+                         {grad_sampling_locations, pr.lsamples * 8},
                          {grad_attention_weights, pr.samples * 4}};
     const Span ins[] = {{value, pr.n_value * pr.esz},
-                        {sampling_locations, pr.samples * 8},
+                        {sampling_locations, pr.lsamples * 8},
                         {attention_weights, pr.samples * 4},
                         {grad_out, pr.n_out * 4}};
     if (any_alias(outs, 3, ins, 4)) return MSDA_ERR_ALIAS;
@@ -343,6 +360,11 @@ msda_status msda_backward(const void *value, msda_dtype value_dtype,
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (pr.n_value > 0) {
         st = cuda_status(cudaMemsetAsync(grad_value, 0, (size_t)pr.n_value * 4, s));
+        if (st != MSDA_OK) return st;
+    }
+    if (grad_sampling_locations && G < d.M && pr.lsamples > 0) {  // heads of a group add up
+        st = cuda_status(
+            cudaMemsetAsync(grad_sampling_locations, 0, (size_t)pr.lsamples * 8, s));
         if (st != MSDA_OK) return st;
     }
     if (pr.n_out == 0) return MSDA_OK;
@@ -356,31 +378,23 @@ msda_status msda_backward(const void *value, msda_dtype value_dtype,
     p.grad_value = grad_value;
     p.grad_loc = grad_sampling_locations;
     p.grad_attn = grad_attention_weights;
-    p.items = pr.items;
-    p.Lq = (int)d.Lq;
-    p.S = (int)d.S;
-    p.M = (int)d.M;
-    p.D = (int)d.D;
-    p.L = (int)d.L;
-    p.K = (int)d.K;
-    p.nchunks = pr.nchunks;
-    p.lv = pr.lv;
+    set_dims(&p, d, G, pr);
     if ((st = set_checks(&p, pr)) != MSDA_OK) return st;
     return launched(msda::launch_backward(p, value_dtype == MSDA_BF16, pr.lanes, s), s);
 }
 
-msda_status msda_backward_fused(const void *value, msda_dtype value_dtype,
-                                const int64_t *spatial_shapes,
-                                const int64_t *level_start_index,
+msda_status backward_fused_impl(const void *value, msda_dtype value_dtype,
+                                const int64_t *spatial_shapes, const int64_t *level_start_index,
                                 const float *reference_points, int reference_dim,
                                 const float *offsets, const float *logits,
                                 const float *grad_out, float *grad_value,
                                 float *grad_reference_points, float *grad_offsets,
-                                float *grad_logits, msda_dims d, msda_stream_t stream)
+                                float *grad_logits, msda_dims d, int64_t G, msda_stream_t stream)
 {
     Problem pr;
     msda_status st = check_dims(value_dtype, spatial_shapes, level_start_index, d, &pr);
     if (st != MSDA_OK) return st;
+    if ((st = check_groups(d, G, &pr)) != MSDA_OK) return st;
     if (reference_dim != 2 && reference_dim != 4) return MSDA_ERR_SHAPE;
     if (d.D > 32) return MSDA_ERR_UNSUPPORTED;
     if (pr.n_value > 0 && !grad_value) return MSDA_ERR_NULL;
@@ -395,11 +409,11 @@ msda_status msda_backward_fused(const void *value, msda_dtype value_dtype,
     const int64_t nq = pr.items / d.M;
     const Span outs[] = {{grad_value, pr.n_value * 4},
                          {grad_reference_points, nq * reference_dim * 4},
-                         {grad_offsets, pr.samples * 8},
+                         {grad_offsets, pr.lsamples * 8},
                          {grad_logits, pr.samples * 4}};
     const Span ins[] = {{value, pr.n_value * pr.esz},
                         {reference_points, nq * reference_dim * 4},
-                        {offsets, pr.samples * 8},
+                        {offsets, pr.lsamples * 8},
                         {logits, pr.samples * 4},
                         {grad_out, pr.n_out * 4}};
     if (any_alias(outs, 4, ins, 5)) return MSDA_ERR_ALIAS;
@@ -412,6 +426,10 @@ msda_status msda_backward_fused(const void *value, msda_dtype value_dtype,
     if (grad_reference_points && nq > 0) {
         st = cuda_status(
             cudaMemsetAsync(grad_reference_points, 0, (size_t)(nq * reference_dim) * 4, s));
+        if (st != MSDA_OK) return st;
+    }
+    if (grad_offsets && G < d.M && pr.lsamples > 0) {  // heads of a group add up
+        st = cuda_status(cudaMemsetAsync(grad_offsets, 0, (size_t)pr.lsamples * 8, s));
         if (st != MSDA_OK) return st;
     }
     if (pr.n_out == 0) return MSDA_OK;
@@ -428,17 +446,117 @@ msda_status msda_backward_fused(const void *value, msda_dtype value_dtype,
     p.grad_ref = grad_reference_points;
     p.grad_off = grad_offsets;
     p.grad_logits = grad_logits;
-    p.items = pr.items;
-    p.Lq = (int)d.Lq;
-    p.S = (int)d.S;
-    p.M = (int)d.M;
-    p.D = (int)d.D;
-    p.L = (int)d.L;
-    p.K = (int)d.K;
-    p.nchunks = pr.nchunks;
-    p.lv = pr.lv;
+    set_dims(&p, d, G, pr);
     if ((st = set_checks(&p, pr)) != MSDA_OK) return st;
     return launched(msda::launch_backward_fused(p, value_dtype == MSDA_BF16, s), s);
+}
+
+}  // namespace
+
+extern "C" {
+
+msda_status msda_forward(const void *value, msda_dtype value_dtype,
+                         const int64_t *spatial_shapes, const int64_t *level_start_index,
+                         const float *sampling_locations, const float *attention_weights,
+                         float *out, msda_dims d, msda_stream_t stream)
+{
+    return forward_impl(value, value_dtype, spatial_shapes, level_start_index,
+                        sampling_locations, attention_weights, out, d, d.M, stream);
+}
+
+msda_status msda_forward_grouped(const void *value, msda_dtype value_dtype,
+                                 const int64_t *spatial_shapes,
+                                 const int64_t *level_start_index,
+                                 const float *sampling_locations,
+                                 const float *attention_weights, float *out, msda_dims d,
+                                 int64_t groups, msda_stream_t stream)
+{
+    return forward_impl(value, value_dtype, spatial_shapes, level_start_index,
+                        sampling_locations, attention_weights, out, d, groups, stream);
+}
+
+msda_status msda_forward_fused(const void *value, msda_dtype value_dtype,
+                               const int64_t *spatial_shapes,
+                               const int64_t *level_start_index,
+                               const float *reference_points, int reference_dim,
+                               const float *offsets, const float *logits, float *out,
+                               float *sampling_locations_out, float *attention_weights_out,
+                               msda_dims d, msda_stream_t stream)
+{
+    return forward_fused_impl(value, value_dtype, spatial_shapes, level_start_index,
+                              reference_points, reference_dim, offsets, logits, out,
+                              sampling_locations_out, attention_weights_out, d, d.M, stream);
+}
+
+msda_status msda_forward_fused_grouped(const void *value, msda_dtype value_dtype,
+                                       const int64_t *spatial_shapes,
+                                       const int64_t *level_start_index,
+                                       const float *reference_points, int reference_dim,
+                                       const float *offsets, const float *logits, float *out,
+                                       float *sampling_locations_out,
+                                       float *attention_weights_out, msda_dims d,
+                                       int64_t groups, msda_stream_t stream)
+{
+    return forward_fused_impl(value, value_dtype, spatial_shapes, level_start_index,
+                              reference_points, reference_dim, offsets, logits, out,
+                              sampling_locations_out, attention_weights_out, d, groups, stream);
+}
+
+msda_status msda_backward(const void *value, msda_dtype value_dtype,
+                          const int64_t *spatial_shapes, const int64_t *level_start_index,
+                          const float *sampling_locations, const float *attention_weights,
+                          const float *grad_out, float *grad_value,
+                          float *grad_sampling_locations, float *grad_attention_weights,
+                          msda_dims d, msda_stream_t stream)
+{
+    return backward_impl(value, value_dtype, spatial_shapes, level_start_index,
+                         sampling_locations, attention_weights, grad_out, grad_value,
+                         grad_sampling_locations, grad_attention_weights, d, d.M, stream);
+}
+
+msda_status msda_backward_grouped(const void *value, msda_dtype value_dtype,
+                                  const int64_t *spatial_shapes,
+                                  const int64_t *level_start_index,
+                                  const float *sampling_locations,
+                                  const float *attention_weights, const float *grad_out,
+                                  float *grad_value, float *grad_sampling_locations,
+                                  float *grad_attention_weights, msda_dims d, int64_t groups,
+                                  msda_stream_t stream)
+{
+    return backward_impl(value, value_dtype, spatial_shapes, level_start_index,
+                         sampling_locations, attention_weights, grad_out, grad_value,
+                         grad_sampling_locations, grad_attention_weights, d, groups, stream);
+}
+
+msda_status msda_backward_fused(const void *value, msda_dtype value_dtype,
+                                const int64_t *spatial_shapes,
+                                const int64_t *level_start_index,
+                                const float *reference_points, int reference_dim,
+                                const float *offsets, const float *logits,
+                                const float *grad_out, float *grad_value,
+                                float *grad_reference_points, float *grad_offsets,
+                                float *grad_logits, msda_dims d, msda_stream_t stream)
+{
+    return backward_fused_impl(value, value_dtype, spatial_shapes, level_start_index,
+                               reference_points, reference_dim, offsets, logits, grad_out,
+                               grad_value, grad_reference_points, grad_offsets, grad_logits, d,
+                               d.M, stream);
+}
+
+msda_status msda_backward_fused_grouped(const void *value, msda_dtype value_dtype,
+                                        const int64_t *spatial_shapes,
+                                        const int64_t *level_start_index,
+                                        const float *reference_points, int reference_dim,
+                                        const float *offsets, const float *logits,
+                                        const float *grad_out, float *grad_value,
+                                        float *grad_reference_points, float *grad_offsets,
+                                        float *grad_logits, msda_dims d, int64_t groups,
+                                        msda_stream_t stream)
+{
+    return backward_fused_impl(value, value_dtype, spatial_shapes, level_start_index,
+                               reference_points, reference_dim, offsets, logits, grad_out,
+                               grad_value, grad_reference_points, grad_offsets, grad_logits, d,
+                               groups, stream);
 }
 
 msda_status msda_debug_sample_points(const int64_t *spatial_shapes,

@@ -106,7 +106,9 @@ __device__ __forceinline__ void reduce_scatter_n(float (&v)[N], int lane)
 }
 
 // Generic path (any row width): one warp per item, partial sums of 32 lanes
-// reduced every 8 samples.  Used for rows wider than 128 bytes.
+// reduced every 8 samples.  Used for rows wider than 128 bytes.  The item's
+// samples are taken in blocks of 32 (one per lane in phase 1), so any L*K up
+// to kMaxLK works.
 template <typename VT, int R>
 __global__ void __launch_bounds__(kWarps * 32)
     bwd_kernel_wide(const __grid_constant__ BwdParams p)
@@ -118,8 +120,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     constexpr int kCpl = 4 / kCornerSlots;            // corners per lane
     constexpr int kPer = kNV / kSpan;                 // finished sums per lane
 
-    __shared__ CornerB corners[kWarps][kMaxLK * 4];
-    __shared__ float sA[kWarps][kMaxLK];
+    __shared__ CornerB corners[kWarps][32 * 4];
+    __shared__ float sA[kWarps][32];
     __shared__ int sH[kMaxLevels], sW[kMaxLevels], sStart[kMaxLevels];
 
     const int tid = threadIdx.x;
@@ -140,40 +142,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int m = (int)(item % M);
     const int64_t nq = item / M;
     const int64_t n = nq / p.Lq;
-    const int64_t sbase = item * LK;
 
-    // ---- phase 1: cell and corner derivatives of sample `lane` -------------
-    if (lane < LK) {
-        const int l = lane / K;
-        const int H = sH[l], W = sW[l], start = sStart[l];
-        const float2 t = __ldg(reinterpret_cast<const float2 *>(p.loc) + sbase + lane);
-        sA[warp][lane] = __ldg(p.attn + sbase + lane);
-        CornerB c[4] = {{-1, 0.f, 0.f, 0.f}, {-1, 0.f, 0.f, 0.f}, {-1, 0.f, 0.f, 0.f},
-                        {-1, 0.f, 0.f, 0.f}};
-        float x, y, fx, fy;
-        int x0, y0;
-        if (msda_cell(t.x, t.y, H, W, x, y, x0, y0, fx, fy)) {
-            const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
-            // corner j = (dy, dx) = (j >> 1, j & 1)
-            const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
-            const float dwx[4] = {-hy, hy, -fy, fy};
-            const float dwy[4] = {-hx, -fx, hx, fx};
-            const int MD = M * D;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const int r = msda_row(start, H, W, y0 + (j >> 1), x0 + (j & 1));
-                c[j].off = r < 0 ? -1 : r * MD;
-                c[j].w = w[j];
-                c[j].dwx = dwx[j];
-                c[j].dwy = dwy[j];
-            }
-        }
-#pragma unroll
-        for (int j = 0; j < 4; ++j) corners[warp][lane * 4 + j] = c[j];
-    }
-    __syncwarp();
-
-    // ---- phase 2/3 -------------------------------------------------------
     const int grp = lane / kSpan;
     const int lin = lane % kSpan;
     const int cslot = lin / R;
@@ -200,57 +169,102 @@ __global__ void __launch_bounds__(kWarps * 32)
     const VT *vbase = static_cast<const VT *>(p.value) + rowbase;
     float *gvbase = p.grad_value + rowbase;
 
-    const int per_batch = kBatch * kGroups;
-    for (int b0 = 0; b0 < LK; b0 += per_batch) {
-        float v[kNV];
+    const int64_t litem = msda_loc_item(item, M, p.G, p.Hg);
+    const bool shared_loc = p.Hg > 1;
+    for (int blk0 = 0; blk0 < LK; blk0 += 32) {
+        const int nb = LK - blk0 < 32 ? LK - blk0 : 32;  // samples in this block
+        const int64_t sbase = item * LK + blk0;   // per head
+        const int64_t lbase = litem * LK + blk0;  // per group
+        // ---- phase 1: cell and corner derivatives of sample blk0 + lane -------
+        if (lane < nb) {
+            const int l = (blk0 + lane) / K;
+            const int H = sH[l], W = sW[l], start = sStart[l];
+            const float2 t = __ldg(reinterpret_cast<const float2 *>(p.loc) + lbase + lane);
+            sA[warp][lane] = __ldg(p.attn + sbase + lane);
+            CornerB c[4] = {{-1, 0.f, 0.f, 0.f}, {-1, 0.f, 0.f, 0.f}, {-1, 0.f, 0.f, 0.f},
+                            {-1, 0.f, 0.f, 0.f}};
+            float x, y, fx, fy;
+            int x0, y0;
+            if (msda_cell(t.x, t.y, H, W, x, y, x0, y0, fx, fy)) {
+                const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+                // corner j = (dy, dx) = (j >> 1, j & 1)
+                const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
+                const float dwx[4] = {-hy, hy, -fy, fy};
+                const float dwy[4] = {-hx, -fx, hx, fx};
+                const int MD = M * D;
 #pragma unroll
-        for (int i = 0; i < kNV; ++i) v[i] = 0.f;
+                for (int j = 0; j < 4; ++j) {
+                    const int r = msda_row(start, H, W, y0 + (j >> 1), x0 + (j & 1));
+                    c[j].off = r < 0 ? -1 : r * MD;
+                    c[j].w = w[j];
+                    c[j].dwx = dwx[j];
+                    c[j].dwy = dwy[j];
+                }
+            }
 #pragma unroll
-        for (int it = 0; it < kBatch; ++it) {
-            const int s = b0 + it * kGroups + grp;
-            if (s < LK) {
-                const float a = sA[warp][s];
+            for (int j = 0; j < 4; ++j) corners[warp][lane * 4 + j] = c[j];
+        }
+        __syncwarp();
+
+        // ---- phase 2/3 ---------------------------------------------------
+        const int per_batch = kBatch * kGroups;
+        for (int b0 = 0; b0 < nb; b0 += per_batch) {
+            float v[kNV];
 #pragma unroll
-                for (int ci = 0; ci < kCpl; ++ci) {
-                    const CornerB e = corners[warp][s * 4 + cslot * kCpl + ci];
-                    float t = 0.f;
-                    if (e.off >= 0 && chunk_ok &&
-                        msda_in_map(p.check, p.check_limit, rowbase + e.off, kVec)) {
-                        float x[kVec];
-                        Chunk<VT>::load(vbase + e.off, x);
+            for (int i = 0; i < kNV; ++i) v[i] = 0.f;
 #pragma unroll
-                        for (int i = 0; i < kVec; ++i) t = fmaf(x[i], g[i], t);
-                        const float aw = a * e.w;
-                        float *dst = gvbase + e.off;
+            for (int it = 0; it < kBatch; ++it) {
+                const int s = b0 + it * kGroups + grp;
+                if (s < nb) {
+                    const float a = sA[warp][s];
 #pragma unroll
-                        for (int i = 0; i < kVec; i += 4)
-                            red_add_v4(dst + i, aw * g[i], aw * g[i + 1], aw * g[i + 2],
-                                       aw * g[i + 3]);
+                    for (int ci = 0; ci < kCpl; ++ci) {
+                        const CornerB e = corners[warp][s * 4 + cslot * kCpl + ci];
+                        float t = 0.f;
+                        if (e.off >= 0 && chunk_ok &&
+                            msda_in_map(p.check, p.check_limit, rowbase + e.off, kVec)) {
+                            float x[kVec];
+                            Chunk<VT>::load(vbase + e.off, x);
+#pragma unroll
+                            for (int i = 0; i < kVec; ++i) t = fmaf(x[i], g[i], t);
+                            const float aw = a * e.w;
+                            float *dst = gvbase + e.off;
+#pragma unroll
+                            for (int i = 0; i < kVec; i += 4)
+                                red_add_v4(dst + i, aw * g[i], aw * g[i + 1], aw * g[i + 2],
+                                           aw * g[i + 3]);
+                        }
+                        v[it] = fmaf(e.w, t, v[it]);
+                        v[kBatch + it] = fmaf(e.dwx, t, v[kBatch + it]);
+                        v[2 * kBatch + it] = fmaf(e.dwy, t, v[2 * kBatch + it]);
                     }
-                    v[it] = fmaf(e.w, t, v[it]);
-                    v[kBatch + it] = fmaf(e.dwx, t, v[kBatch + it]);
-                    v[2 * kBatch + it] = fmaf(e.dwy, t, v[2 * kBatch + it]);
                 }
             }
-        }
-        reduce_scatter<kSpan, kNV>(v, lane);
+            reduce_scatter<kSpan, kNV>(v, lane);
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-            const int idx = lin * kPer + i;
-            const int qty = idx / kBatch;
-            const int it = idx % kBatch;
-            const int s = b0 + it * kGroups + grp;
-            if (qty < 3 && s < LK) {
-                const int64_t si = sbase + s;
-                if (qty == 0) {
-                    if (p.grad_attn) p.grad_attn[si] = v[i];
-                } else if (p.grad_loc) {
-                    const int l = s / K;
-                    const float scale = (qty == 1) ? (float)sW[l] : (float)sH[l];
-                    p.grad_loc[2 * si + (qty - 1)] = sA[warp][s] * (scale * v[i]);
+            for (int i = 0; i < kPer; ++i) {
+                const int idx = lin * kPer + i;
+                const int qty = idx / kBatch;
+                const int it = idx % kBatch;
+                const int s = b0 + it * kGroups + grp;
+                if (qty < 3 && s < nb) {
+                    const int64_t si = sbase + s;
+                    if (qty == 0) {
+                        if (p.grad_attn) p.grad_attn[si] = v[i];
+                    } else if (p.grad_loc) {
+                        const int l = (blk0 + s) / K;
+                        const float scale = (qty == 1) ? (float)sW[l] : (float)sH[l];
+                        float *dst = p.grad_loc + 2 * (lbase + s) + (qty - 1);
+                        const float gl = sA[warp][s] * (scale * v[i]);
+                        if (shared_loc)
+                            atomicAdd(dst, gl);  // the group's heads add into one location
+                        else
+                            *dst = gl;
+                    }
                 }
             }
         }
+        __syncwarp();  // the next block overwrites corners and weights
     }
 }
 
@@ -363,14 +377,15 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
         const int64_t item = i0 + seg;
         pl_x = pl_y = pa = 0.f;
         if (jact && item < p.items) {
-            const int64_t si = item * LK + j;
+            const int64_t si = item * LK + j;                               // per head
+            const int64_t sl = msda_loc_item(item, M, p.G, p.Hg) * LK + j;  // per group
             if constexpr (kFused) {
-                const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + si);
+                const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sl);
                 pl_x = o.x;
                 pl_y = o.y;
                 pa = __ldcs(p.logits + si);
             } else {
-                const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
+                const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + sl);
                 pl_x = t.x;
                 pl_y = t.y;
                 pa = __ldcs(p.attn + si);
@@ -438,7 +453,8 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
             const int m = (int)(itm % M);
             const int64_t nq = itm / M;
             const int64_t n = nq / p.Lq;
-            const int64_t sbase = itm * LK;
+            const int64_t sbase = itm * LK;                                 // per head
+            const int64_t lbase = msda_loc_item(itm, M, p.G, p.Hg) * LK;    // per group
             const int64_t mapoff = (n * p.S * M + m) * (int64_t)D;
             const int64_t vbe = mapoff + lane_elem;
             const VT *vb = static_cast<const VT *>(p.value) + vbe;
@@ -523,9 +539,7 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
                     const float dlx = rec.z * q1, dly = rec.w * q2;  // d loc
                     if constexpr (!kFused) {
                         if (p.grad_attn) __stcs(p.grad_attn + si, q0);
-                        if (p.grad_loc)
-                            __stcs(reinterpret_cast<float2 *>(p.grad_loc) + si,
-                                   make_float2(dlx, dly));
+                        if (p.grad_loc) msda_put_loc_grad(p.grad_loc, lbase + s, dlx, dly, p.Hg > 1);
                     } else {
                         const float4 r2 = smq[warp][it][s];  // (A, off_x, off_y, -)
                         float2 goff;
@@ -538,7 +552,8 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
                             rw = fmaf(dlx, r2.y, rw);
                             rh = fmaf(dly, r2.z, rh);
                         }
-                        if (p.grad_off) __stcs(reinterpret_cast<float2 *>(p.grad_off) + si, goff);
+                        if (p.grad_off)
+                            msda_put_loc_grad(p.grad_off, lbase + s, goff.x, goff.y, p.Hg > 1);
                         rx += dlx;
                         ry += dly;
                         dpart = fmaf(r2.x, q0, dpart);
@@ -578,6 +593,256 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
     }
 }
 
+// Items of more than 32 samples (32 < L*K <= kMaxLK) with rows of at most
+// eight 4-element lanes.  The lane layout, entries and two-stage reduction are
+// bwd_kernel's with one item per warp and round; the item's samples are taken
+// in blocks of 32 (lane j of phase 1 owns sample blk*32 + j).  The fused
+// variant forms the joint softmax first (long_softmax, as the forward does)
+// and keeps every sample's (A, dA) in shared memory until the softmax
+// Jacobian's sum over all blocks is known.
+template <typename VT, int R, bool kFused>
+__global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
+    bwd_kernel_long(const __grid_constant__ BwdParams p)
+{
+    static_assert(R <= 8, "at least four pairs per warp instruction");
+    constexpr int kVec = 4;
+    using Raw = typename Lane4<VT>::Raw;
+    constexpr int kSlots = 32 / R;
+    constexpr int kSG = kSlots / 4;  // samples per warp instruction
+    constexpr int kB = R;            // instructions per batch
+    constexpr int kBS = kB * kSG;    // samples per batch (= 8)
+    constexpr int kStride = 34;
+    constexpr int kNBt = 32 / kBS;   // batches per block
+    constexpr int kNB = kMaxLK / 32;
+    __shared__ int2 ent[kWarps][4 * kStride];                // (row offset | -1, A*w)
+    __shared__ float4 smp[kWarps][32];                       // (fx, fy, A*W, A*H)
+    __shared__ float4 smq[kWarps][kFused ? 32 : 1];          // fused: (A, off_x, off_y, -)
+    __shared__ float2 smd[kWarps][kFused ? kMaxLK : 1];      // fused: (A, dA) per sample
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int M = p.M, D = p.D, K = p.K;
+    const int LK = p.L * K;
+    const int MD = M * D;
+    const int nblk = (LK + 31) / 32;
+
+    const int slot = lane / R;
+    const int chunk = lane % R;
+    const int corner = slot & 3;
+    const int sg = slot >> 2;
+    const bool chunk_ok = chunk < p.nchunks;
+    const int lane_elem = (chunk_ok ? chunk : 0) * kVec;
+    const bool cx = corner & 1, cy = corner >> 1;
+
+    for (int64_t item = (int64_t)blockIdx.x * kWarps + warp; item < p.items;
+         item += (int64_t)gridDim.x * kWarps) {
+        const int m = (int)(item % M);
+        const int64_t nq = item / M;
+        const int64_t n = nq / p.Lq;
+        const int64_t mapoff = (n * p.S * M + m) * (int64_t)D;
+        const int64_t vbe = mapoff + lane_elem;
+        const VT *vb = static_cast<const VT *>(p.value) + vbe;
+        float *gvb = p.grad_value + mapoff + chunk * kVec;
+        const int64_t lbase = msda_loc_item(item, M, p.G, p.Hg) * LK;  // per group
+        float gv[kVec];
+        if (chunk_ok) {
+            const float4 t = __ldcs(reinterpret_cast<const float4 *>(
+                p.grad_out + nq * (int64_t)MD + m * D + chunk * kVec));
+            gv[0] = t.x;
+            gv[1] = t.y;
+            gv[2] = t.z;
+            gv[3] = t.w;
+        } else {
+            gv[0] = gv[1] = gv[2] = gv[3] = 0.f;
+        }
+        float z[kNB];
+        float sum = 1.f;
+        float2 bwh = make_float2(0.f, 0.f);
+        if constexpr (kFused) {
+#pragma unroll
+            for (int b = 0; b < kNB; ++b) {
+                const int s = b * 32 + lane;
+                z[b] = s < LK ? __ldcs(p.logits + item * LK + s) : -INFINITY;
+            }
+            sum = long_softmax<kNB>(z);
+            if (p.ref_dim == 4) bwh = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
+        }
+        float dpart = 0.f, rx = 0.f, ry = 0.f, rw = 0.f, rh = 0.f;
+
+#pragma unroll 1
+        for (int blk = 0; blk < nblk; ++blk) {
+            // ---- phase 1: sample blk*32 + lane ---------------------------------
+            {
+                const int s = blk * 32 + lane;
+                const bool act = s < LK;
+                const int64_t si = item * LK + s;  // per head
+                const int l = act ? s / K : 0;
+                const int H = p.lv.H[l], W = p.lv.W[l], start = p.lv.start[l];
+                float lx = 0.f, ly = 0.f, a = 0.f;
+                if constexpr (kFused) {
+                    float ox = 0.f, oy = 0.f;
+                    if (act) {
+                        a = __fdiv_rn(pick<kNB>(z, blk), sum);
+                        const float2 o =
+                            __ldcs(reinterpret_cast<const float2 *>(p.off) + lbase + s);
+                        ox = o.x;
+                        oy = o.y;
+                        if (p.ref_dim == 2) {
+                            const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
+                            lx = __fadd_rn(r.x, __fdiv_rn(ox, (float)W));
+                            ly = __fadd_rn(r.y, __fdiv_rn(oy, (float)H));
+                        } else {
+                            const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
+                            lx = __fadd_rn(c.x, __fmul_rn(ox, bwh.x));
+                            ly = __fadd_rn(c.y, __fmul_rn(oy, bwh.y));
+                        }
+                    }
+                    smq[warp][lane] = make_float4(a, ox, oy, 0.f);
+                } else if (act) {
+                    const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + lbase + s);
+                    lx = t.x;
+                    ly = t.y;
+                    a = __ldcs(p.attn + si);
+                }
+                int2 e[4] = {{-1, 0}, {-1, 0}, {-1, 0}, {-1, 0}};
+                float4 rec = make_float4(0.f, 0.f, 0.f, 0.f);
+                float x, y, fx, fy;
+                int x0, y0;
+                if (act && msda_cell(lx, ly, H, W, x, y, x0, y0, fx, fy)) {
+                    const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+                    const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int r = msda_row(start, H, W, y0 + (c >> 1), x0 + (c & 1));
+                        if (r >= 0) e[c] = make_int2(r * MD, __float_as_int(a * w[c]));
+                    }
+                    rec = make_float4(fx, fy, a * (float)W, a * (float)H);
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) ent[warp][c * kStride + lane] = e[c];
+                smp[warp][lane] = rec;
+            }
+            __syncwarp();
+
+            // ---- phase 2: batches of 8 samples ----------------------------------
+            const int2 *en = ent[warp] + corner * kStride + sg;
+#pragma unroll
+            for (int bi = 0; bi < kNBt; ++bi) {
+                const int s0 = bi * kBS;
+                if (blk * 32 + s0 >= LK) break;  // uniform
+                int2 e[kB];
+                Raw raw[kB];
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    e[b] = en[s0 + b * kSG];
+                    if (e[b].x >= 0 && !msda_in_map(p.check, p.check_limit, vbe + e[b].x, kVec))
+                        e[b].x = -1;  // bounds-checked build: reads zeros, scatters nothing
+                    if (e[b].x >= 0) raw[b] = Lane4<VT>::load(vb + e[b].x);
+                }
+                float t[kB];
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    t[b] = 0.f;
+                    if (e[b].x >= 0) {
+                        float v[kVec];
+                        Lane4<VT>::widen(raw[b], v);
+#pragma unroll
+                        for (int i = 0; i < kVec; ++i) t[b] = fmaf(v[i], gv[i], t[b]);
+                        if (chunk_ok) {
+                            const float aw = __int_as_float(e[b].y);
+                            red_add_v4(gvb + e[b].x, aw * gv[0], aw * gv[1], aw * gv[2],
+                                       aw * gv[3]);
+                        }
+                    }
+                }
+                reduce_scatter_n<R, kB, kB>(t, lane);
+                const int s = s0 + chunk * kSG + sg;  // sample within the block, < 32
+                const int sgl = blk * 32 + s;
+                const float4 rec = smp[warp][s];
+                const float fx = rec.x, fy = rec.y;
+                const float wxc = cx ? fx : __fsub_rn(1.f, fx);
+                const float wyc = cy ? fy : __fsub_rn(1.f, fy);
+                float q0 = (wyc * wxc) * t[0];
+                float q1 = (cx ? wyc : -wyc) * t[0];
+                float q2 = (cy ? wxc : -wxc) * t[0];
+#pragma unroll
+                for (int o = R; o < 4 * R; o <<= 1) {
+                    q0 += __shfl_xor_sync(kFull, q0, o);
+                    q1 += __shfl_xor_sync(kFull, q1, o);
+                    q2 += __shfl_xor_sync(kFull, q2, o);
+                }
+                if (corner == 0 && sgl < LK) {
+                    const int64_t si = item * LK + sgl;
+                    const float dlx = rec.z * q1, dly = rec.w * q2;
+                    if constexpr (!kFused) {
+                        if (p.grad_attn) __stcs(p.grad_attn + si, q0);
+                        if (p.grad_loc)
+                            msda_put_loc_grad(p.grad_loc, lbase + sgl, dlx, dly, p.Hg > 1);
+                    } else {
+                        const float4 r2 = smq[warp][s];  // (A, off_x, off_y, -)
+                        float2 goff;
+                        if (p.ref_dim == 2) {
+                            goff = make_float2(r2.x * q1, r2.x * q2);
+                        } else {
+                            goff = make_float2(dlx * bwh.x, dly * bwh.y);
+                            rw = fmaf(dlx, r2.y, rw);
+                            rh = fmaf(dly, r2.z, rh);
+                        }
+                        if (p.grad_off)
+                            msda_put_loc_grad(p.grad_off, lbase + sgl, goff.x, goff.y, p.Hg > 1);
+                        rx += dlx;
+                        ry += dly;
+                        dpart = fmaf(r2.x, q0, dpart);
+                        smd[warp][sgl] = make_float2(r2.x, q0);
+                    }
+                }
+            }
+            __syncwarp();  // the next block overwrites the entries and records
+        }
+        if constexpr (kFused) {
+            // softmax Jacobian over all L*K samples: d z_s = A_s (dA_s - sum_j A_j dA_j)
+            const float dot = warp_sum(dpart);
+            for (int s = lane; s < LK; s += 32) {
+                const float2 ad = smd[warp][s];
+                if (p.grad_logits) __stcs(p.grad_logits + item * LK + s, ad.x * (ad.y - dot));
+            }
+            rx = warp_sum(rx);
+            ry = warp_sum(ry);
+            if (p.ref_dim == 4) {
+                rw = warp_sum(rw);
+                rh = warp_sum(rh);
+            }
+            if (lane == 0 && p.grad_ref) {
+                float *gr = p.grad_ref + nq * p.ref_dim;
+                atomicAdd(gr, rx);
+                atomicAdd(gr + 1, ry);
+                if (p.ref_dim == 4) {
+                    atomicAdd(gr + 2, rw);
+                    atomicAdd(gr + 3, rh);
+                }
+            }
+            __syncwarp();  // the next item overwrites smd
+        }
+    }
+}
+
+template <typename VT, bool kFused>
+cudaError_t launch_long(const BwdParams &p, cudaStream_t stream)
+{
+    const int r4 = p.D / 4;  // D % 4 == 0 and r4 <= 8 checked by the caller
+    BwdParams q = p;
+    q.nchunks = r4;
+    auto go = [&](auto kern) {
+        const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, q.items, kWarps);
+        kern<<<(unsigned)ctas, kWarps * 32, 0, stream>>>(q);
+        return cudaGetLastError();
+    };
+    if (r4 <= 1) return go(bwd_kernel_long<VT, 1, kFused>);
+    if (r4 <= 2) return go(bwd_kernel_long<VT, 2, kFused>);
+    if (r4 <= 4) return go(bwd_kernel_long<VT, 4, kFused>);
+    return go(bwd_kernel_long<VT, 8, kFused>);
+}
+
 template <typename VT, int R, int P, bool kFused>
 cudaError_t launch_fast(const BwdParams &p, cudaStream_t stream)
 {
@@ -603,6 +868,7 @@ cudaError_t launch_bwd_fused_vt(const BwdParams &p, cudaStream_t stream)
 {
     const int r4 = p.D / 4;
     if (p.D % 4 != 0 || r4 > 8) return cudaErrorInvalidValue;
+    if (p.L * p.K > kLaneLK) return launch_long<VT, true>(p, stream);
     BwdParams q = p;
     q.nchunks = r4;
     if (r4 <= 1) return launch_fast_r<VT, 1, true>(q, stream);
@@ -616,6 +882,7 @@ cudaError_t launch_bwd_vt(const BwdParams &p, int R, cudaStream_t stream)
 {
     // fast path: four elements per lane, R4 = D/4 lanes per (fp32) gradient row
     const int r4 = p.D / 4;
+    if (p.D % 4 == 0 && r4 <= 8 && p.L * p.K > kLaneLK) return launch_long<VT, false>(p, stream);
     if (p.D % 4 == 0 && r4 <= 8) {
         BwdParams q = p;
         q.nchunks = r4;

@@ -62,6 +62,35 @@ __device__ __forceinline__ bool msda_in_map(unsigned long long *check, int64_t l
 #endif
 }
 
+// Item of the per-sample location tensors (sampling locations, offsets and
+// their gradients) that item = (n*Lq + q)*M + m reads: the heads of one
+// deformable group share one set of sampling locations ("Deformable
+// Attention" glossary page, heads grouped into deformable groups that share
+// the sampled keys), so with G groups of Hg = M/G consecutive heads it is
+// (n*Lq + q)*G + m/Hg.  Hg = 1 (a group per head) gives the item itself.
+__device__ __forceinline__ int64_t msda_loc_item(int64_t item, int M, int G, int Hg)
+{
+    if (Hg == 1) return item;
+    const int64_t nq = item / M;
+    const int m = (int)(item - nq * M);
+    return nq * G + m / Hg;
+}
+
+// Writes the gradient of one shared location: a plain store when every head
+// has its own locations, else a vector reduction into the zeroed output, since
+// the Hg heads of a group add into one location (their order is unspecified).
+__device__ __forceinline__ void msda_put_loc_grad(float *base, int64_t sl, float gx, float gy,
+                                                  bool shared)
+{
+    float2 *dst = reinterpret_cast<float2 *>(base) + sl;
+    if (!shared) {
+        __stcs(dst, make_float2(gx, gy));
+        return;
+    }
+    asm volatile("red.global.add.v2.f32 [%0], {%1, %2};" ::"l"(dst), "f"(gx), "f"(gy)
+                 : "memory");
+}
+
 // Value row of pixel (yy, xx) on a level, or -1 outside the level (zero
 // padding: such a corner contributes nothing).
 __device__ __forceinline__ int msda_row(int start, int H, int W, int yy, int xx)
@@ -141,6 +170,38 @@ __device__ __forceinline__ float seg_sum(float v)
 #pragma unroll
     for (int o = P / 2; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
     return v;
+}
+
+// Joint softmax statistics of one item of more than 32 samples, held by one
+// warp: lane j holds the logits of samples j, j + 32, ... in z[] (NB = the
+// blocks of 32 there can be; entries past L*K are -inf).  On return z[b] is
+// exp(z[b] - max) and the result is the sum over all samples, so that the
+// weight of sample b*32 + j is __fdiv_rn(z[b], sum).  The forward and the
+// backward both call this, so they form bit-identical weights.
+template <int NB>
+__device__ __forceinline__ float long_softmax(float (&z)[NB])
+{
+    float mx = z[0];
+#pragma unroll
+    for (int b = 1; b < NB; ++b) mx = fmaxf(mx, z[b]);
+    mx = warp_max(mx);
+    float sum = 0.f;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        z[b] = z[b] == -INFINITY ? 0.f : expf(__fsub_rn(z[b], mx));
+        sum += z[b];
+    }
+    return warp_sum(sum);
+}
+
+// z[i] for a run-time i < NB, as a chain of selects (no local memory).
+template <int NB>
+__device__ __forceinline__ float pick(const float (&z)[NB], int i)
+{
+    float r = z[0];
+#pragma unroll
+    for (int b = 1; b < NB; ++b) r = (i == b) ? z[b] : r;
+    return r;
 }
 
 }  // namespace msda

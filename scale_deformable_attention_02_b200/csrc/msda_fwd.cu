@@ -123,7 +123,8 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
             const int j = lane % P;    // sample within the item
             const int64_t item = item0 + seg;
             const bool act = j < LK && item < end;
-            const int64_t si = item * LK + j;
+            const int64_t si = item * LK + j;                               // per head
+            const int64_t sl = msda_loc_item(item, M, p.G, p.Hg) * LK + j;  // per group
             const int l = act ? j / K : 0;
             float lx = 0.f, ly = 0.f, a = 0.f;
             if constexpr (kFused) {
@@ -133,7 +134,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
                 const float s = seg_sum<P>(e);
                 a = __fdiv_rn(e, s);
                 if (act) {
-                    const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + si);
+                    const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sl);
                     const int64_t nq = item / M;
                     if (p.ref_dim == 2) {
                         // point reference: offsets are level-l pixels
@@ -148,12 +149,12 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
                         lx = __fadd_rn(c.x, __fmul_rn(o.x, s2.x));
                         ly = __fadd_rn(c.y, __fmul_rn(o.y, s2.y));
                     }
-                    if (p.loc_out)
-                        __stcs(reinterpret_cast<float2 *>(p.loc_out) + si, make_float2(lx, ly));
+                    if (p.loc_out && (p.Hg == 1 || (item % M) % p.Hg == 0))  // group's first head
+                        __stcs(reinterpret_cast<float2 *>(p.loc_out) + sl, make_float2(lx, ly));
                     if (p.attn_out) __stcs(p.attn_out + si, a);
                 }
             } else if (act) {
-                const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
+                const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + sl);
                 lx = t.x;
                 ly = t.y;
                 a = __ldcs(p.attn + si);
@@ -373,14 +374,15 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
         const int64_t item = i0 + seg;
         pa = pb = pc = 0.f;
         if (jact && item < p.items) {
-            const int64_t si = item * LK + j;
+            const int64_t si = item * LK + j;                               // per head
+            const int64_t sl = msda_loc_item(item, M, p.G, p.Hg) * LK + j;  // per group
             if constexpr (kFused) {
                 pa = __ldcs(p.logits + si);
-                const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + si);
+                const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sl);
                 pb = o.x;
                 pc = o.y;
             } else {
-                const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
+                const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + sl);
                 pb = t.x;
                 pc = t.y;
                 pa = __ldcs(p.attn + si);
@@ -418,8 +420,10 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
                     lx = __fadd_rn(c.x, __fmul_rn(pb, s2.x));
                     ly = __fadd_rn(c.y, __fmul_rn(pc, s2.y));
                 }
-                if (p.loc_out)
-                    __stcs(reinterpret_cast<float2 *>(p.loc_out) + si, make_float2(lx, ly));
+                if (p.loc_out && (p.Hg == 1 || (item % M) % p.Hg == 0))  // group's first head
+                    __stcs(reinterpret_cast<float2 *>(p.loc_out) +
+                               msda_loc_item(item, M, p.G, p.Hg) * LK + j,
+                           make_float2(lx, ly));
                 if (p.attn_out) __stcs(p.attn_out + si, a);
             }
         } else {
@@ -503,6 +507,181 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
     }
 }
 
+// ---------------------------------------------------------------------------
+// Items of more than 32 samples (32 < L*K <= kMaxLK), any row width.
+//
+// One warp per item and round.  The fused softmax comes first: lane j holds
+// the logits of samples j, j + 32, ... in registers and the warp forms the
+// joint statistics (long_softmax).  The samples are then taken in blocks of
+// 32, lane j owning sample blk*32 + j: phase 1 writes the block's corner
+// entries, phase 2 gathers them into the same accumulators, and the item's
+// output is stored once after its last block.
+// ---------------------------------------------------------------------------
+template <typename VT, int EPL, int R, bool kFused>
+__global__ void __launch_bounds__(kWarps * 32, 3)
+    fwd_kernel_long(const __grid_constant__ FwdParams p)
+{
+    using LL = LaneLoad<VT, EPL>;
+    constexpr int kSlots = 32 / R;  // (sample, corner) pairs per warp instruction
+    constexpr int kStride = 34;     // = 2 mod 8: conflict-free entries
+    constexpr int kNP = EPL / 2;
+    constexpr int kB = MSDA_FWD_BATCH;
+    constexpr int kNB = kMaxLK / 32;
+    static_assert(128 % (kB * kSlots) == 0, "a batch must tile a block's entries");
+    __shared__ int2 ent[kWarps][4 * kStride];
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int M = p.M, D = p.D, K = p.K;
+    const int LK = p.L * K;
+    const int MD = M * D;
+    const int nblk = (LK + 31) / 32;
+    const int slot = lane / R;
+    const int chunk = lane % R;
+    const bool chunk_ok = chunk < p.nchunks;
+    const int lane_elem = (chunk_ok ? chunk : 0) * EPL;
+
+    for (int64_t item = (int64_t)blockIdx.x * kWarps + warp; item < p.items;
+         item += (int64_t)gridDim.x * kWarps) {
+        const int m = (int)(item % M);
+        const int64_t nq = item / M;
+        const int64_t n = nq / p.Lq;
+        const int64_t vbe = (n * p.S * M + m) * (int64_t)D + lane_elem;
+        const VT *vb = static_cast<const VT *>(p.value) + vbe;
+        const int64_t litem = msda_loc_item(item, M, p.G, p.Hg);
+        const bool first_head = p.Hg == 1 || m % p.Hg == 0;
+        float z[kNB];
+        float sum = 1.f;
+        if constexpr (kFused) {
+#pragma unroll
+            for (int b = 0; b < kNB; ++b) {
+                const int s = b * 32 + lane;
+                z[b] = s < LK ? __ldcs(p.logits + item * LK + s) : -INFINITY;
+            }
+            sum = long_softmax<kNB>(z);
+        }
+        float2 acc[kNP];
+#pragma unroll
+        for (int i = 0; i < kNP; ++i) acc[i] = make_float2(0.f, 0.f);
+
+#pragma unroll 1
+        for (int blk = 0; blk < nblk; ++blk) {
+            // ---- phase 1: sample blk*32 + lane --------------------------------
+            {
+                const int s = blk * 32 + lane;
+                const bool act = s < LK;
+                const int64_t si = item * LK + s;    // per head
+                const int64_t sl = litem * LK + s;   // per group
+                const int l = act ? s / K : 0;
+                const int H = p.lv.H[l], W = p.lv.W[l], start = p.lv.start[l];
+                float lx = 0.f, ly = 0.f, a = 0.f;
+                if (act) {
+                    if constexpr (kFused) {
+                        a = __fdiv_rn(pick<kNB>(z, blk), sum);
+                        const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sl);
+                        if (p.ref_dim == 2) {
+                            const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
+                            lx = __fadd_rn(r.x, __fdiv_rn(o.x, (float)W));
+                            ly = __fadd_rn(r.y, __fdiv_rn(o.y, (float)H));
+                        } else {
+                            const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
+                            const float2 s2 =
+                                __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
+                            lx = __fadd_rn(c.x, __fmul_rn(o.x, s2.x));
+                            ly = __fadd_rn(c.y, __fmul_rn(o.y, s2.y));
+                        }
+                        if (p.loc_out && first_head)
+                            __stcs(reinterpret_cast<float2 *>(p.loc_out) + sl, make_float2(lx, ly));
+                        if (p.attn_out) __stcs(p.attn_out + si, a);
+                    } else {
+                        const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + sl);
+                        lx = t.x;
+                        ly = t.y;
+                        a = __ldcs(p.attn + si);
+                    }
+                }
+                int2 e[4] = {{-1, 0}, {-1, 0}, {-1, 0}, {-1, 0}};
+                float x, y, fx, fy;
+                int x0, y0;
+                if (act && msda_cell(lx, ly, H, W, x, y, x0, y0, fx, fy)) {
+                    const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+                    const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int r = msda_row(start, H, W, y0 + (c >> 1), x0 + (c & 1));
+                        if (r >= 0) e[c] = make_int2(r * MD, __float_as_int(w[c] * a));
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) ent[warp][c * kStride + lane] = e[c];
+            }
+            __syncwarp();
+
+            // ---- phase 2: the block's (sample, corner) pairs ------------------
+            const int rem = LK - blk * 32;
+            const int npairs = 4 * (rem < 32 ? rem : 32);
+            for (int t0 = 0; t0 < npairs; t0 += kB * kSlots) {
+                int2 e[kB];
+                typename LL::Raw raw[kB];
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    const int t = t0 + b * kSlots + slot;  // < 128: entries past L*K hold -1
+                    e[b] = ent[warp][(t & 3) * kStride + (t >> 2)];
+                    if (e[b].x >= 0 && !msda_in_map(p.check, p.check_limit, vbe + e[b].x, EPL))
+                        e[b].x = -1;  // bounds-checked build: skipped, reads as zero
+                    if (e[b].x >= 0) raw[b] = LL::load(vb + e[b].x);
+                }
+#pragma unroll
+                for (int b = 0; b < kB; ++b) {
+                    if (e[b].x >= 0) {
+                        float2 v[kNP];
+                        LL::widen(raw[b], v);
+                        const float wb = __int_as_float(e[b].y);
+                        const float2 w2 = make_float2(wb, wb);
+#pragma unroll
+                        for (int i = 0; i < kNP; ++i) acc[i] = __ffma2_rn(w2, v[i], acc[i]);
+                    }
+                }
+            }
+            __syncwarp();  // the next block overwrites the entries
+        }
+#pragma unroll
+        for (int o = R; o < 32; o <<= 1)
+#pragma unroll
+            for (int i = 0; i < kNP; ++i) {
+                acc[i].x += __shfl_xor_sync(kFull, acc[i].x, o);
+                acc[i].y += __shfl_xor_sync(kFull, acc[i].y, o);
+            }
+        if (slot == 0 && chunk_ok) {
+            float4 *dst =
+                reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D + chunk * EPL);
+#pragma unroll
+            for (int i = 0; i < kNP / 2; ++i)
+                __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
+                                            acc[2 * i + 1].y));
+        }
+    }
+}
+
+template <typename VT, int EPL, bool kFused>
+cudaError_t launch_long(FwdParams p, cudaStream_t stream)
+{
+    const int lanes = (p.D + EPL - 1) / EPL;  // D*size is a multiple of 16 bytes
+    p.nchunks = lanes;
+    const dim3 block(kWarps * 32);
+    auto go = [&](auto kern) {
+        const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kWarps);
+        kern<<<(unsigned)ctas, block, 0, stream>>>(p);
+        return cudaGetLastError();
+    };
+    if (lanes <= 1) return go(fwd_kernel_long<VT, EPL, 1, kFused>);
+    if (lanes <= 2) return go(fwd_kernel_long<VT, EPL, 2, kFused>);
+    if (lanes <= 4) return go(fwd_kernel_long<VT, EPL, 4, kFused>);
+    if (lanes <= 8) return go(fwd_kernel_long<VT, EPL, 8, kFused>);
+    if (lanes <= 16) return go(fwd_kernel_long<VT, EPL, 16, kFused>);
+    return go(fwd_kernel_long<VT, EPL, 32, kFused>);
+}
+
 template <typename VT, int EPL, int R, int P, bool kFused>
 cudaError_t launch_fast(FwdParams p, cudaStream_t stream)
 {
@@ -563,6 +742,7 @@ template <typename VT, bool kFused>
 cudaError_t launch_fwd_vt(const FwdParams &p, int R, cudaStream_t stream)
 {
     constexpr int EPL = sizeof(VT) == 4 ? 4 : MSDA_FWD_BF16_EPL;
+    if (p.L * p.K > kLaneLK) return launch_long<VT, 16 / (int)sizeof(VT), kFused>(p, stream);
     // fast path: rows of at most 8 lanes of EPL elements
     const int lanes = (p.D + EPL - 1) / EPL;
     if (p.D % EPL == 0 && lanes <= 8) {

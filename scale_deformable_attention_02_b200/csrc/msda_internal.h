@@ -14,20 +14,21 @@ namespace msda {
 struct FwdParams {
     const void *value;
     // unfused inputs
-    const float *loc;   // [N,Lq,M,L,K,2]
+    const float *loc;   // [N,Lq,G,L,K,2]
     const float *attn;  // [N,Lq,M,L,K]
     // fused inputs
     const float *ref;     // [N,Lq,ref_dim]
-    const float *off;     // [N,Lq,M,L,K,2]
+    const float *off;     // [N,Lq,G,L,K,2]
     const float *logits;  // [N,Lq,M,L,K]
     int ref_dim;
     // outputs
     float *out;       // [N,Lq,M*D]
-    float *loc_out;   // nullable (fused)
+    float *loc_out;   // nullable (fused) [N,Lq,G,L,K,2]
     float *attn_out;  // nullable (fused)
     int64_t items;    // N*Lq*M
     int64_t chunk;    // items per CTA (set by the launcher)
     int Lq, S, M, D, L, K;
+    int G, Hg;    // deformable groups and heads per group (G = M: one per head)
     int nchunks;  // 16-byte chunks per value row
     Levels lv;
     // bounds-checked build only (-DMSDA_CHECKED): value elements an access
@@ -42,19 +43,20 @@ struct BwdParams {
     const float *loc;   // unfused inputs
     const float *attn;
     const float *ref;     // fused inputs: [N,Lq,ref_dim]
-    const float *off;     // [N,Lq,M,L,K,2]
+    const float *off;     // [N,Lq,G,L,K,2]
     const float *logits;  // [N,Lq,M,L,K]
     int ref_dim;
     const float *grad_out;
     float *grad_value;
-    float *grad_loc;     // nullable (unfused)
+    float *grad_loc;     // nullable (unfused) [N,Lq,G,L,K,2]; zeroed by the host if G < M
     float *grad_attn;    // nullable (unfused)
     float *grad_ref;     // nullable (fused; zeroed by the host, accumulated over heads)
-    float *grad_off;     // nullable (fused)
+    float *grad_off;     // nullable (fused) [N,Lq,G,L,K,2]; zeroed by the host if G < M
     float *grad_logits;  // nullable (fused)
     int64_t items;
     int64_t chunk;  // items per CTA (set by the launcher)
     int Lq, S, M, D, L, K;
+    int G, Hg;  // deformable groups and heads per group (G = M: one per head)
     int nchunks;
     Levels lv;
     // bounds-checked build only (-DMSDA_CHECKED): value elements an access

@@ -3,8 +3,9 @@
 
 namespace msda {
 
-constexpr int kMaxLK = 32;      // samples per (query, head): one per lane
-constexpr int kMaxLevels = 32;  // L <= L*K <= 32
+constexpr int kMaxLK = 128;     // samples per (query, head): up to four per lane
+constexpr int kLaneLK = 32;     // items of up to 32 samples: one sample per lane
+constexpr int kMaxLevels = 32;  // L <= 32
 
 // Per-level metadata, copied by value into every launch.
 struct Levels {

@@ -47,7 +47,7 @@ class Workload:
     Lq: int | None  # None: one query per pixel of every level (encoder)
     value_dtype: str  # "f32" or "bf16"
     seed: int
-    recipe: str  # "tiny", "decoder", "encoder", "stress"
+    recipe: str  # "tiny", "decoder", "encoder", "stress", "compass"
     offset_std: float = 0.0
     oob_fraction: float = 0.0
     notes: str = field(default="", compare=False)
@@ -87,9 +87,33 @@ ENCODER_BWD = Workload("encoder_bwd", N=2, M=8, D=32, K=4,
 STRESS = Workload("stress", N=8, M=8, D=32, K=8, shapes=STRESS_SHAPES,
                   Lq=None, value_dtype="bf16", seed=5, recipe="stress",
                   offset_std=4.0, oob_fraction=0.05)
+# The encoder at initialisation: every head samples along its compass
+# direction, k pixels out for point k, with uniform weights (zero logits).
+ENCODER_COMPASS = Workload("encoder_compass", N=2, M=8, D=32, K=4,
+                           shapes=ENCODER_SHAPES, Lq=None, value_dtype="f32",
+                           seed=6, recipe="compass")
 
 WORKLOADS = {w.name: w for w in (TINY, DECODER, ENCODER, ENCODER_BF16,
-                                 ENCODER_BWD, STRESS)}
+                                 ENCODER_BWD, STRESS, ENCODER_COMPASS)}
+
+# Offset directions (dx, dy) of the eight heads at initialisation, in the
+# order the "Deformable DETR" wiki page lists them ("Initialization"): head m
+# samples point k (k = 1..K) at k * COMPASS[m] pixels on every level.
+COMPASS = ((-1, -1), (-1, 0), (-1, 1), (0, -1), (0, 1), (1, -1), (1, 0), (1, 1))
+
+
+def compass_offsets(N: int, Lq: int, M: int, L: int, K: int, scale: float = 1.0) -> np.ndarray:
+    """[N,Lq,M,L,K,2] float32 offsets of the compass initialisation: head m,
+    point k (0-based) at (k+1) * COMPASS[m] * scale pixels, the same for every
+    query and level.  scale = 1/(2K) gives the iterative-refinement variant
+    (box units).  Needs M = 8."""
+    if M != len(COMPASS):
+        raise ValueError("the compass pattern has one direction per head: M must be 8")
+    dirs = np.asarray(COMPASS, dtype=np.float32)                      # [M, 2]
+    ks = np.arange(1, K + 1, dtype=np.float32) * np.float32(scale)    # [K]
+    one = dirs[:, None, None, :] * ks[None, None, :, None]           # [M, 1, K, 2]
+    return np.ascontiguousarray(
+        np.broadcast_to(one[None, None], (N, Lq, M, L, K, 2)).astype(np.float32))
 
 
 def round_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -170,11 +194,17 @@ def make_inputs(w: Workload, with_grad: bool = True) -> dict:
             ref = pixel_centre_queries(w.shapes)
             d["reference_points"] = np.ascontiguousarray(
                 np.broadcast_to(ref, (N, Lq, 2)))
-        off = _normal(rng, (N, Lq, M, L, K, 2), w.offset_std)
-        if w.oob_fraction > 0.0:
-            push_offsets_out_of_range(rng, off, w.shapes, w.oob_fraction)
-        d["offsets"] = off
-    d["logits"] = _normal(rng, (N, Lq, M, L, K))
+        if w.recipe == "compass":
+            d["offsets"] = compass_offsets(N, Lq, M, L, K)
+        else:
+            off = _normal(rng, (N, Lq, M, L, K, 2), w.offset_std)
+            if w.oob_fraction > 0.0:
+                push_offsets_out_of_range(rng, off, w.shapes, w.oob_fraction)
+            d["offsets"] = off
+    if w.recipe == "compass":
+        d["logits"] = np.zeros((N, Lq, M, L, K), dtype=np.float32)
+    else:
+        d["logits"] = _normal(rng, (N, Lq, M, L, K))
     if with_grad:
         d["grad_out"] = _normal(rng, (N, Lq, M * D))
     return d

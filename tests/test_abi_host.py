@@ -159,9 +159,9 @@ def test_forward_argument_errors(lib):
     bad = Prob()
     bad.dims.N = -1
     assert fwd(lib, bad) == SHAPE
-    # L*K beyond one lane per sample
-    big = Prob(K=17)
-    assert fwd(lib, big) == UNSUP
+    # L*K beyond four samples per lane, more than 32 levels
+    assert fwd(lib, Prob(K=65)) == UNSUP
+    assert fwd(lib, Prob(K=1, shapes=tuple((1, 1) for _ in range(33)))) == UNSUP
     # level metadata that disagrees with S or with the prefix sum
     bad = Prob()
     bad.dims.S += 1

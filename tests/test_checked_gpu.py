@@ -43,6 +43,8 @@ CASES = [
     (1, 23, 2, 64, 2, ((8, 8), (4, 4)), "f32"),                      # wide, 256-B rows
     (1, 17, 3, 256, 2, ((5, 4), (2, 3)), "bf16"),                    # wide, 512-B rows
     (1, 12, 2, 32, 16, ((6, 8), (3, 4)), "f32"),                     # L*K = 32
+    (1, 9, 2, 32, 16, ((6, 8), (3, 4), (2, 2)), "f32"),              # L*K = 48, blocks
+    (1, 7, 2, 64, 9, ((5, 5), (3, 3), (2, 2), (1, 1)), "f32"),       # wide, L*K = 36
 ]
 IDS = [f"case{i}" for i in range(len(CASES))]
 

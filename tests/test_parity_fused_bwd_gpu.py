@@ -74,6 +74,26 @@ def test_fused_backward_widths(D, dt):
     _check(d, d["reference_points"], d["offsets"], d["logits"], box=False)
 
 
+@pytest.mark.parametrize("K,shapes,dt,box", [
+    (16, ((6, 8), (3, 4), (2, 2)), "f32", False),              # L*K = 48
+    (32, ((5, 7), (3, 3), (2, 2), (1, 1)), "f32", False),      # L*K = 128
+    (10, ((6, 6), (3, 3), (2, 2), (1, 2), (1, 1)), "bf16", False),  # L*K = 50
+    (12, ((8, 8), (4, 4), (2, 2)), "f32", True),               # box, L*K = 36
+])
+def test_fused_backward_more_than_32_samples(K, shapes, dt, box):
+    """Items of more than 32 samples: the joint softmax over all blocks of
+    32, and the softmax Jacobian's sum taken over every block."""
+    d = wl.make_random_problem(90 + K, N=2, Lq=11, M=3, D=16, K=K, shapes=shapes,
+                               value_dtype=dt)
+    ref, off = d["reference_points"], d["offsets"]
+    if box:
+        rng = np.random.default_rng(91)
+        ref = np.concatenate([rng.uniform(0.1, 0.9, (2, 11, 2)),
+                              rng.uniform(0.05, 0.5, (2, 11, 2))], axis=-1).astype(np.float32)
+        off = (rng.standard_normal(off.shape) * 0.25).astype(np.float32)
+    _check(d, ref, off, d["logits"], box=box)
+
+
 def test_fused_backward_box():
     d = wl.make_random_problem(77, N=2, Lq=29, M=4, D=16, K=4,
                                shapes=((12, 10), (6, 5), (3, 3)))

@@ -132,6 +132,29 @@ def test_encoder_fused_forward_fp32():
     assert_close(host(out), ora, **F32, what="encoder out")
 
 
+def test_encoder_compass_fused_forward_and_backward():
+    """The encoder at the compass initialisation (uniform weights, every head
+    k pixels along its own direction): a highly regular access pattern."""
+    d = wl.make_inputs(wl.ENCODER_COMPASS)
+    sh = d["spatial_shapes"]
+    out, loc_o, a_o = msda_forward_fused(to_dev(d["value"]), sh, None,
+                                         to_dev(d["reference_points"]), to_dev(d["offsets"]),
+                                         to_dev(d["logits"]), return_sampling=True)
+    ora, oloc, oA = oracle.forward_fused(d["value"], sh, d["reference_points"], d["offsets"],
+                                         d["logits"])
+    assert_bits_equal(host(loc_o), oloc, what="compass loc")
+    assert np.all(host(a_o) == np.float32(1.0 / 16))  # exp(0)/16 is exact
+    assert_close(host(out), ora, **F32, what="compass out")
+    A = oA.astype(np.float32)
+    gv, gl, ga = msda_backward(to_dev(d["value"]), sh, None, to_dev(oloc), to_dev(A),
+                               to_dev(d["grad_out"]))
+    ogv, ogl, oga, mgl, mga = oracle.backward(d["value"], sh, oloc, A, d["grad_out"],
+                                              with_mass=True)
+    assert_close(host(gv), ogv, **GRAD, what="compass grad_value")
+    assert_close(host(gl), ogl, **GRAD, what="compass grad_loc", mass=mgl)
+    assert_close(host(ga), oga, **GRAD, what="compass grad_attn", mass=mga)
+
+
 def test_encoder_fused_forward_bf16():
     d = wl.make_inputs(wl.ENCODER_BF16, with_grad=False)
     sh = d["spatial_shapes"]
@@ -222,6 +245,12 @@ CASES = [
     (1, 12, 2, 32, 16, ((6, 8), (3, 4)), "f32"),  # L*K = 32: every lane a sample
     (1, 12, 2, 32, 1, tuple((2 + i, 3) for i in range(32)), "f32"),  # L = 32 levels
     (2, 15, 2, 8, 2, ((0, 4), (3, 3), (5, 0)), "f32"),  # empty levels
+    # more than 32 samples per (query, head): blocks of 32, up to 4 per lane
+    (1, 9, 2, 32, 16, ((6, 8), (3, 4), (2, 2)), "f32"),          # L*K = 48
+    (2, 13, 3, 16, 32, ((5, 7), (3, 3), (2, 2), (1, 1)), "f32"),  # L*K = 128, R = 4
+    (1, 11, 2, 32, 10, ((6, 6), (3, 3), (2, 2), (1, 2), (1, 1)), "bf16"),  # L*K = 50
+    (1, 7, 2, 64, 9, ((5, 5), (3, 3), (2, 2), (1, 1)), "f32"),    # wide rows, L*K = 36
+    (1, 5, 1, 128, 33, ((4, 4),), "f32"),                         # 512-B rows, tail of 1
 ]
 
 
