@@ -277,3 +277,21 @@ def sample_points(loc: np.ndarray, shapes: np.ndarray) -> dict:
                                 _ptr(out["x0"]), _ptr(out["y0"]), _ptr(out["x"]),
                                 _ptr(out["y"]), _ptr(out["rows"]))
     return out
+
+
+def expand_groups(x: np.ndarray, M: int) -> np.ndarray:
+    """Deformable groups ("Deformable Attention" glossary page: heads grouped
+    into deformable groups that share the same sampled keys): a per-group
+    tensor [N, Lq, G, ...] as the per-head tensor [N, Lq, M, ...] it stands
+    for, head m reading group m // (M/G)."""
+    G = x.shape[2]
+    if M % G != 0:
+        raise ValueError("groups must divide the heads")
+    return np.ascontiguousarray(np.repeat(x, M // G, axis=2))
+
+
+def sum_groups(g: np.ndarray, G: int) -> np.ndarray:
+    """Gradient with respect to a per-group input shared by M/G heads: the sum
+    of the per-head gradients over each group.  [N, Lq, M, ...] -> [N, Lq, G, ...]."""
+    N, Lq, M = g.shape[:3]
+    return g.reshape((N, Lq, G, M // G) + g.shape[3:]).sum(axis=3)

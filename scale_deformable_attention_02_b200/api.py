@@ -142,6 +142,7 @@ def msda_level_start_index(spatial_shapes) -> tuple[np.ndarray, int]:
 
 
 def _value_dims(value: torch.Tensor, shapes: np.ndarray, lead):
+    """Dims from value [N,S,M,D] and a per-head tensor's shape [N,Lq,M,L,K]."""
     if value.dim() != 4:
         raise ValueError("value must be [N, S, M, D]")
     N, S, M, D = value.shape
@@ -155,24 +156,41 @@ def _value_dims(value: torch.Tensor, shapes: np.ndarray, lead):
     return _lib.Dims(N, Lq, S, M, D, L, K)
 
 
+def _groups(d, groups) -> int:
+    """Deformable groups: None means one group per head (the ungrouped calls)."""
+    if groups is None:
+        return d.M
+    g = int(groups)
+    if g < 1 or d.M % g != 0:
+        raise ValueError(f"groups={g} must divide the {d.M} heads")
+    return g
+
+
 def msda_forward(value: torch.Tensor, spatial_shapes, level_start_index,
                  sampling_locations: torch.Tensor, attention_weights: torch.Tensor,
-                 out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """out[n,q,m*D:(m+1)*D] = sum_{l,k} A * bilinear(value level l, head m, loc)."""
+                 out: torch.Tensor | None = None, groups: int | None = None,
+                 stream=None) -> torch.Tensor:
+    """out[n,q,m*D:(m+1)*D] = sum_{l,k} A * bilinear(value level l, head m, loc).
+    With `groups` G, sampling_locations is [N,Lq,G,L,K,2], shared by the M/G
+    heads of each group (msda_forward_grouped)."""
     dev = value.device
     shapes, starts = _levels(spatial_shapes, level_start_index)
-    d = _value_dims(value, shapes, tuple(sampling_locations.shape))
-    _need(sampling_locations, "sampling_locations", (d.N, d.Lq, d.M, d.L, d.K, 2), dev)
+    d = _value_dims(value, shapes, tuple(attention_weights.shape))
+    G = _groups(d, groups)
+    _need(sampling_locations, "sampling_locations", (d.N, d.Lq, G, d.L, d.K, 2), dev)
     _need(attention_weights, "attention_weights", (d.N, d.Lq, d.M, d.L, d.K), dev)
     if not value.is_contiguous():
         raise ValueError("value must be contiguous")
     if out is None:
         out = torch.empty((d.N, d.Lq, d.M * d.D), device=dev, dtype=torch.float32)
     _need(out, "out", (d.N, d.Lq, d.M * d.D), dev)
-    _check(_lib.load().msda_forward(_dptr(value), _value_dtype(value), _hptr(shapes),
-                                    _hptr(starts), _dptr(sampling_locations),
-                                    _dptr(attention_weights), _dptr(out), d,
-                                    _stream_handle(dev, stream)), "msda_forward")
+    args = (_dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
+            _dptr(sampling_locations), _dptr(attention_weights), _dptr(out), d)
+    if groups is None:
+        _check(_lib.load().msda_forward(*args, _stream_handle(dev, stream)), "msda_forward")
+    else:
+        _check(_lib.load().msda_forward_grouped(*args, G, _stream_handle(dev, stream)),
+               "msda_forward_grouped")
     return out
 
 
@@ -181,19 +199,23 @@ def msda_forward_fused(value: torch.Tensor, spatial_shapes, level_start_index,
                        logits: torch.Tensor, out: torch.Tensor | None = None,
                        sampling_locations_out: torch.Tensor | None = None,
                        attention_weights_out: torch.Tensor | None = None,
-                       return_sampling: bool = False, stream=None):
+                       return_sampling: bool = False, groups: int | None = None,
+                       stream=None):
     """Fused forward: softmax over the L*K logits of each head and the
     location map (ref + off/W_l, or box: (cx,cy) + off*(w,h)) inside the
     kernel.  Returns out, or (out, sampling_locations, attention_weights) when
-    return_sampling is true (those outputs are then allocated if not given)."""
+    return_sampling is true (those outputs are then allocated if not given).
+    With `groups` G, offsets (and sampling_locations_out) are [N,Lq,G,L,K,2]
+    (msda_forward_fused_grouped)."""
     dev = value.device
     shapes, starts = _levels(spatial_shapes, level_start_index)
-    d = _value_dims(value, shapes, tuple(offsets.shape))
+    d = _value_dims(value, shapes, tuple(logits.shape))
+    G = _groups(d, groups)
     rdim = reference_points.shape[-1] if reference_points.dim() == 3 else -1
     if rdim not in (2, 4):
         raise ValueError("reference_points must be [N, Lq, 2] or [N, Lq, 4]")
     _need(reference_points, "reference_points", (d.N, d.Lq, rdim), dev)
-    _need(offsets, "offsets", (d.N, d.Lq, d.M, d.L, d.K, 2), dev)
+    _need(offsets, "offsets", (d.N, d.Lq, G, d.L, d.K, 2), dev)
     _need(logits, "logits", (d.N, d.Lq, d.M, d.L, d.K), dev)
     if not value.is_contiguous():
         raise ValueError("value must be contiguous")
@@ -209,11 +231,15 @@ def msda_forward_fused(value: torch.Tensor, spatial_shapes, level_start_index,
         _need(sampling_locations_out, "sampling_locations_out", tuple(offsets.shape), dev)
     if attention_weights_out is not None:
         _need(attention_weights_out, "attention_weights_out", tuple(logits.shape), dev)
-    _check(_lib.load().msda_forward_fused(
-        _dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
-        _dptr(reference_points), int(rdim), _dptr(offsets), _dptr(logits), _dptr(out),
-        _dptr(sampling_locations_out), _dptr(attention_weights_out), d,
-        _stream_handle(dev, stream)), "msda_forward_fused")
+    args = (_dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
+            _dptr(reference_points), int(rdim), _dptr(offsets), _dptr(logits), _dptr(out),
+            _dptr(sampling_locations_out), _dptr(attention_weights_out), d)
+    if groups is None:
+        _check(_lib.load().msda_forward_fused(*args, _stream_handle(dev, stream)),
+               "msda_forward_fused")
+    else:
+        _check(_lib.load().msda_forward_fused_grouped(*args, G, _stream_handle(dev, stream)),
+               "msda_forward_fused_grouped")
     if return_sampling:
         return out, sampling_locations_out, attention_weights_out
     return out
@@ -225,13 +251,15 @@ def msda_backward(value: torch.Tensor, spatial_shapes, level_start_index,
                   grad_sampling_locations: torch.Tensor | None = None,
                   grad_attention_weights: torch.Tensor | None = None,
                   need_sampling_grad: bool = True, need_weight_grad: bool = True,
-                  stream=None):
+                  groups: int | None = None, stream=None):
     """Gradients of msda_forward.  Returns (grad_value [fp32], grad_loc or
-    None, grad_attn or None)."""
+    None, grad_attn or None).  With `groups`, the locations and their
+    gradient are per group (msda_backward_grouped)."""
     dev = value.device
     shapes, starts = _levels(spatial_shapes, level_start_index)
-    d = _value_dims(value, shapes, tuple(sampling_locations.shape))
-    _need(sampling_locations, "sampling_locations", (d.N, d.Lq, d.M, d.L, d.K, 2), dev)
+    d = _value_dims(value, shapes, tuple(attention_weights.shape))
+    G = _groups(d, groups)
+    _need(sampling_locations, "sampling_locations", (d.N, d.Lq, G, d.L, d.K, 2), dev)
     _need(attention_weights, "attention_weights", (d.N, d.Lq, d.M, d.L, d.K), dev)
     _need(grad_out, "grad_out", (d.N, d.Lq, d.M * d.D), dev)
     if not value.is_contiguous():
@@ -249,11 +277,14 @@ def msda_backward(value: torch.Tensor, spatial_shapes, level_start_index,
     if grad_attention_weights is not None:
         _need(grad_attention_weights, "grad_attention_weights",
               tuple(attention_weights.shape), dev)
-    _check(_lib.load().msda_backward(
-        _dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
-        _dptr(sampling_locations), _dptr(attention_weights), _dptr(grad_out),
-        _dptr(grad_value), _dptr(grad_sampling_locations), _dptr(grad_attention_weights), d,
-        _stream_handle(dev, stream)), "msda_backward")
+    args = (_dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
+            _dptr(sampling_locations), _dptr(attention_weights), _dptr(grad_out),
+            _dptr(grad_value), _dptr(grad_sampling_locations), _dptr(grad_attention_weights), d)
+    if groups is None:
+        _check(_lib.load().msda_backward(*args, _stream_handle(dev, stream)), "msda_backward")
+    else:
+        _check(_lib.load().msda_backward_grouped(*args, G, _stream_handle(dev, stream)),
+               "msda_backward_grouped")
     return grad_value, grad_sampling_locations, grad_attention_weights
 
 
@@ -265,18 +296,22 @@ def msda_backward_fused(value: torch.Tensor, spatial_shapes, level_start_index,
                         grad_offsets: torch.Tensor | None = None,
                         grad_logits: torch.Tensor | None = None,
                         need_reference_grad: bool = True, need_offset_grad: bool = True,
-                        need_logit_grad: bool = True, stream=None):
+                        need_logit_grad: bool = True, groups: int | None = None,
+                        stream=None):
     """Gradients of msda_forward_fused with respect to the value map, the
     reference points, the offsets and the logits.  Returns (grad_value,
-    grad_reference_points or None, grad_offsets or None, grad_logits or None)."""
+    grad_reference_points or None, grad_offsets or None, grad_logits or None).
+    With `groups`, offsets and their gradient are per group
+    (msda_backward_fused_grouped)."""
     dev = value.device
     shapes, starts = _levels(spatial_shapes, level_start_index)
-    d = _value_dims(value, shapes, tuple(offsets.shape))
+    d = _value_dims(value, shapes, tuple(logits.shape))
+    G = _groups(d, groups)
     rdim = reference_points.shape[-1] if reference_points.dim() == 3 else -1
     if rdim not in (2, 4):
         raise ValueError("reference_points must be [N, Lq, 2] or [N, Lq, 4]")
     _need(reference_points, "reference_points", (d.N, d.Lq, rdim), dev)
-    _need(offsets, "offsets", (d.N, d.Lq, d.M, d.L, d.K, 2), dev)
+    _need(offsets, "offsets", (d.N, d.Lq, G, d.L, d.K, 2), dev)
     _need(logits, "logits", (d.N, d.Lq, d.M, d.L, d.K), dev)
     _need(grad_out, "grad_out", (d.N, d.Lq, d.M * d.D), dev)
     if not value.is_contiguous():
@@ -296,11 +331,16 @@ def msda_backward_fused(value: torch.Tensor, spatial_shapes, level_start_index,
         _need(grad_offsets, "grad_offsets", tuple(offsets.shape), dev)
     if grad_logits is not None:
         _need(grad_logits, "grad_logits", tuple(logits.shape), dev)
-    _check(_lib.load().msda_backward_fused(
-        _dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
-        _dptr(reference_points), int(rdim), _dptr(offsets), _dptr(logits), _dptr(grad_out),
-        _dptr(grad_value), _dptr(grad_reference_points), _dptr(grad_offsets),
-        _dptr(grad_logits), d, _stream_handle(dev, stream)), "msda_backward_fused")
+    args = (_dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
+            _dptr(reference_points), int(rdim), _dptr(offsets), _dptr(logits), _dptr(grad_out),
+            _dptr(grad_value), _dptr(grad_reference_points), _dptr(grad_offsets),
+            _dptr(grad_logits), d)
+    if groups is None:
+        _check(_lib.load().msda_backward_fused(*args, _stream_handle(dev, stream)),
+               "msda_backward_fused")
+    else:
+        _check(_lib.load().msda_backward_fused_grouped(*args, G, _stream_handle(dev, stream)),
+               "msda_backward_fused_grouped")
     return grad_value, grad_reference_points, grad_offsets, grad_logits
 
 

@@ -270,3 +270,29 @@ def test_backward_fused_argument_errors(lib):
                                    None) == UNSUP
     assert lib.msda_backward_fused(fake(0), 0, pr.sp(), pr.st(), None, 2, fake(2), fake(3),
                                    fake(4), fake(5), None, None, None, pr.dims, None) == NULL
+
+
+def test_grouped_argument_errors(lib):
+    """Group counts must divide M (MSDA_ERR_SHAPE); per-group tensors are
+    G/M the size of per-head ones in the alias check."""
+    pr = Prob(M=4)
+
+    def fwd_g(G, loc=None, out=None):
+        return lib.msda_forward_grouped(fake(0), 0, pr.sp(), pr.st(), loc or fake(1), fake(2),
+                                        out or fake(3), pr.dims, G, None)
+
+    for G in (0, -1, 3, 5, 8):
+        assert fwd_g(G) == SHAPE, G
+    # a grouped location tensor of G=1 spans N*Lq*1*L*K*2 floats: an output
+    # placed right after it does not alias, one inside it does
+    n_loc = 2 * 5 * 1 * 2 * 2 * 2 * 4  # bytes, G = 1
+    assert lib.msda_forward_grouped(fake(0), 0, pr.sp(), pr.st(), fake(1), fake(2),
+                                    fake(1, n_loc - 16), pr.dims, 1, None) == ALIAS
+    assert lib.msda_backward_grouped(fake(0), 0, pr.sp(), pr.st(), fake(1), fake(2), fake(3),
+                                     fake(4), None, None, pr.dims, 3, None) == SHAPE
+    assert lib.msda_forward_fused_grouped(fake(0), 0, pr.sp(), pr.st(), fake(1), 2, fake(2),
+                                          fake(4), fake(3), None, None, pr.dims, 0,
+                                          None) == SHAPE
+    assert lib.msda_backward_fused_grouped(fake(0), 0, pr.sp(), pr.st(), fake(1), 2, fake(2),
+                                           fake(3), fake(4), fake(5), None, None, None,
+                                           pr.dims, 6, None) == SHAPE

@@ -218,3 +218,41 @@ def test_finite_differences_fused_chain_box():
         m_[ii] -= h
         fd = (F(p_, off, z) - F(m_, off, z)) / (2 * h)
         assert abs(fd - g_box[ii]) <= 1e-6 * (1 + abs(fd))
+
+
+def test_finite_differences_grouped_locations():
+    """Deformable groups: G groups of M/G heads share one set of locations.
+    The gradient of a shared location is the sum over the group's heads of
+    the per-head gradients (oracle.sum_groups); checked by central
+    differences of <g, F(expand_groups(loc_g))> in every group coordinate."""
+    d = wl.make_random_problem(61, N=1, Lq=5, M=4, D=4, K=2, shapes=((7, 6), (3, 4)))
+    shapes = d["spatial_shapes"]
+    G = 2
+    loc_g = d["sampling_locations"][:, :, :G].astype(np.float64)
+    A = oracle.softmax(d["logits"])
+    g = d["grad_out"].astype(np.float64)
+    loc_h = oracle.expand_groups(loc_g, 4)
+    assert np.array_equal(loc_h[:, :, 1], loc_g[:, :, 0]) and np.array_equal(
+        loc_h[:, :, 2], loc_g[:, :, 1])
+    _, gl, _ = oracle.backward(d["value"], shapes, loc_h, A, g, loc_f32=False)
+    gl_g = oracle.sum_groups(gl, G)
+    assert gl_g.shape == loc_g.shape
+    skip = _kink_mask(loc_h, shapes, 1e-3).reshape(1, 5, G, 2, 2, 2).any(axis=3)
+    h = 1e-6
+    checked = 0
+    for ii in np.argwhere(~skip):
+        ii = tuple(ii)
+        for c in range(2):
+            lp, lm = loc_g.copy(), loc_g.copy()
+            lp[ii + (c,)] += h
+            lm[ii + (c,)] -= h
+            fp = np.sum(g * oracle.forward(d["value"], shapes, oracle.expand_groups(lp, 4), A,
+                                           loc_f32=False))
+            fm = np.sum(g * oracle.forward(d["value"], shapes, oracle.expand_groups(lm, 4), A,
+                                           loc_f32=False))
+            fd = (fp - fm) / (2 * h)
+            assert abs(fd - gl_g[ii + (c,)]) <= 1e-6 * (1 + abs(fd)), (ii, c)
+            checked += 1
+    assert checked >= 40
+    # one group per head is the ungrouped problem
+    assert np.array_equal(oracle.sum_groups(gl, 4), gl)
