@@ -121,8 +121,8 @@ MSDA_API msda_status msda_level_start_index(const int64_t *spatial_shapes, int64
 /*
  * Forward from given sampling locations and attention weights
  * ("Deformable DETR" wiki page, "Multi-scale deformable attention"
- * equation, with bilinear interpolation of the four surrounding pixels as in
- * "Deformable attention module").
+ * equation, each sample read by bilinear interpolation between the four
+ * pixels around it, as in "Deformable attention module").
  *
  *   value               device [N,S,M,D] of value_dtype, 16-byte aligned
  *   spatial_shapes      host   [L,2] int64 (H_l, W_l), H_l, W_l >= 0
@@ -188,8 +188,8 @@ MSDA_API msda_status msda_forward_fused(const void *value, msda_dtype value_dtyp
  * interpolation to the value map, to the sampling locations and to the
  * attention weights ("Deformable DETR" wiki page, "Deformable attention
  * module": interpolation makes the offsets differentiable; "Deformable
- * Attention" glossary page: gradients flow back through the interpolation
- * grid).  With g = grad_out[n,q,m*D:(m+1)*D] and corner weights w_j:
+ * Attention" glossary page: the interpolation passes gradients on to the
+ * offset prediction).  With g = grad_out[n,q,m*D:(m+1)*D] and corner weights w_j:
  *   grad_attention_weights = sum_j w_j <v_j, g>
  *   grad_value[corner j]  += A w_j g        (corners inside the level)
  *   grad_sampling_locations = A * (W_l, H_l) * sum_j (dw_j/dfx, dw_j/dfy) <v_j, g>
@@ -256,9 +256,9 @@ MSDA_API msda_status msda_backward_fused(const void *value, msda_dtype value_dty
                                          msda_stream_t stream);
 
 /*
- * Deformable groups ("Deformable Attention" glossary page: heads grouped
- * into deformable groups that share the same set of sampled keys, with
- * different projection weights).  The M heads form `groups` groups of
+ * Deformable groups ("Deformable Attention" glossary page, multi-head
+ * paragraph: heads may be gathered into fewer groups whose members look up
+ * the same key locations while keeping their own projections).  The M heads form `groups` groups of
  * Hg = M/groups consecutive heads (head m is in group m / Hg); the heads of a
  * group sample the same locations, each with its own attention weights and
  * its own value channels.  The four calls below are msda_forward,

@@ -1,4 +1,4 @@
-"""CPU oracle for the multi-scale deformable attention core.
+"""CPU oracle of the MSDeformAttn (multi-scale deformable attention) core.
 
 TEST INFRASTRUCTURE ONLY: the test suite, the package smoke check and the
 benchmark's CPU-baseline leg are the only users.  The product path (the CUDA
@@ -280,8 +280,8 @@ def sample_points(loc: np.ndarray, shapes: np.ndarray) -> dict:
 
 
 def expand_groups(x: np.ndarray, M: int) -> np.ndarray:
-    """Deformable groups ("Deformable Attention" glossary page: heads grouped
-    into deformable groups that share the same sampled keys): a per-group
+    """Deformable groups ("Deformable Attention" glossary page, multi-head
+    paragraph: the heads of a group look up the same key locations): a per-group
     tensor [N, Lq, G, ...] as the per-head tensor [N, Lq, M, ...] it stands
     for, head m reading group m // (M/G)."""
     G = x.shape[2]

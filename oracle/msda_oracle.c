@@ -1,5 +1,5 @@
 /*
- * msda_oracle.c -- plain CPU oracle for the multi-scale deformable attention
+ * msda_oracle.c -- plain CPU oracle of the multi-scale deformable attention
  * (MSDeformAttn) core.
  *
  * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or
@@ -161,8 +161,8 @@ static int64_t pixel_row(const int64_t *shapes, const int64_t *starts,
 
 /*
  * Forward ("Deformable DETR" wiki page, "Multi-scale deformable attention"
- * equation; bilinear interpolation of the four surrounding pixels, same
- * page, "Deformable attention module").
+ * equation; each sample interpolated bilinearly between the four pixels
+ * around it, same page, "Deformable attention module").
  *
  *   value [N,S,M,D]  fp32 or bf16 bits      loc  [N,Lq,M,L,K,2] (x,y)
  *   attn  [N,Lq,M,L,K] (fp64)              out  [N,Lq,M*D] (fp64)
@@ -313,8 +313,8 @@ void ora_locations_f64(const double *ref, const double *off, const int64_t *shap
  * Backward of ora_forward: the gradients flow through the interpolation to
  * the value, the locations and the weights ("Deformable DETR" wiki page,
  * "Deformable attention module": the interpolation makes the offsets
- * differentiable; "Deformable Attention" glossary page: gradients flow back
- * through the interpolation grid).
+ * differentiable; "Deformable Attention" glossary page: the interpolation
+ * passes gradients on to the offset prediction).
  *
  * With g = grad_out[n,q,m,:] and corner weights w_j(fx, fy):
  *   grad_attn[i]       = sum_j w_j <v_j, g>

@@ -3,7 +3,7 @@
 // Gradients flow through the bilinear interpolation to the value map, the
 // sampling locations and the attention weights ("Deformable DETR" wiki
 // page, "Deformable attention module"; "Deformable Attention" glossary
-// page, gradients through the interpolation grid).  Per sample, with
+// page, the interpolation passes gradients on).  Per sample, with
 // g = grad_out[n,q,m,:], corner weights w_j(fx, fy) and t_j = <v_j, g>:
 //   dA        = sum_j w_j t_j
 //   dloc_x    = A * W * sum_j (dw_j/dfx) t_j,  dloc_y = A * H * sum_j (dw_j/dfy) t_j

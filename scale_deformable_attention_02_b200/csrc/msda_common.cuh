@@ -64,9 +64,9 @@ __device__ __forceinline__ bool msda_in_map(unsigned long long *check, int64_t l
 
 // Item of the per-sample location tensors (sampling locations, offsets and
 // their gradients) that item = (n*Lq + q)*M + m reads: the heads of one
-// deformable group share one set of sampling locations ("Deformable
-// Attention" glossary page, heads grouped into deformable groups that share
-// the sampled keys), so with G groups of Hg = M/G consecutive heads it is
+// deformable group look up the same key locations ("Deformable Attention"
+// glossary page, multi-head paragraph), so with G groups of Hg = M/G
+// consecutive heads it is
 // (n*Lq + q)*G + m/Hg.  Hg = 1 (a group per head) gives the item itself.
 __device__ __forceinline__ int64_t msda_loc_item(int64_t item, int M, int G, int Hg)
 {

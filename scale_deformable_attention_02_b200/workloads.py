@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs for the multi-scale deformable attention core.
+"""Seeded synthetic inputs of the MSDeformAttn (multi-scale deformable attention) core.
 
 This module only draws random numbers and lays them out; it holds none of the
 method's arithmetic (no level prefix sums, no softmax, no location or sampling
@@ -138,7 +138,7 @@ def spatial_shapes_array(shapes) -> np.ndarray:
 def pixel_centre_queries(shapes) -> np.ndarray:
     """Encoder queries: one per pixel of every level, level-major then
     row-major, each with its own pixel centre as normalised (x, y) reference
-    point ("the reference point is the pixel itself", Deformable DETR wiki
+    point (an encoder query refers to its own pixel: Deformable DETR wiki
     page, "Architecture / Encoder").  Computed in fp32: ((w+0.5)/W, (h+0.5)/H).
     Returns [S, 2] float32."""
     out = []
