@@ -23,6 +23,7 @@ import datetime
 import hashlib
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -128,11 +129,17 @@ def algorithmic_bytes(w: wl.Workload, step: str = "split") -> dict:
 
 
 def kernel_source_hash() -> str:
+    """sha256 of the CUDA/C++ sources with comments and blank space removed,
+    so that a counter taken on a kernel stays valid across comment edits."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "scale_deformable_attention_02_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), "rb") as fh:
-            h.update(f.encode() + b"\0" + fh.read())
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        text = " ".join(text.split())
+        h.update(f.encode() + b"\0" + text.encode())
     return h.hexdigest()
 
 
