@@ -67,6 +67,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle leg")
     ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--no-floors", action="store_true",
+                    help="skip the memory-floor replay of the workload's corner rows")
     ap.add_argument("--graph", action="store_true",
                     help="capture the forward and the backward as two CUDA graphs and time "
                          "their replays (the launch-latency path for small problems such "
@@ -129,17 +131,26 @@ def algorithmic_bytes(w: wl.Workload, step: str = "split") -> dict:
 
 
 def kernel_source_hash() -> str:
-    """sha256 of the CUDA/C++ sources with comments and blank space removed,
-    so that a counter taken on a kernel stays valid across comment edits."""
+    """sha256 of the forward and backward kernels' device code: msda_fwd.cu,
+    msda_bwd.cu, msda_common.cuh, msda_types.h and the FwdParams / BwdParams
+    structs, with comments and blank space removed, so that a counter taken on
+    those kernels stays valid across edits that do not touch them."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "scale_deformable_attention_02_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
-            text = fh.read()
+
+    def norm(text):
         text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
         text = re.sub(r"//[^\n]*", " ", text)
-        text = " ".join(text.split())
-        h.update(f.encode() + b"\0" + text.encode())
+        return " ".join(text.split())
+
+    for f in ("msda_fwd.cu", "msda_bwd.cu", "msda_common.cuh", "msda_types.h"):
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + b"\0" + norm(fh.read()).encode())
+    with open(os.path.join(csrc, "msda_internal.h"), encoding="utf-8") as fh:
+        internal = norm(fh.read())
+    for name in ("FwdParams", "BwdParams"):
+        m = re.search(r"struct " + name + r" \{.*?\};", internal)
+        h.update(name.encode() + b"\0" + (m.group(0) if m else "").encode())
     return h.hexdigest()
 
 
@@ -394,6 +405,13 @@ def run_ours(args):
         "algorithmic_bytes_per_launch": ab[dom],
     }
 
+    floors = None
+    if not args.no_floors:
+        floors = memory_floors(torch, w, sh, starts, value, ref, off, logits, flush)
+        if floors:
+            kernels["fwd"]["frac_of_row_floor"] = floors["gather_us"] / (ms_fwd * 1e3)
+            kernels["bwd"]["frac_of_row_floor"] = floors["gather_reduce_us"] / (ms_bwd * 1e3)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w, inp)
@@ -430,6 +448,7 @@ def run_ours(args):
             "effective_GB_s": (ab["fwd"] + ab["bwd"]) / (ms_step / 1e3) / 1e9,
             "kernels": kernels,
             "roofline": roofline,
+            "row_floors": floors,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": 2 * K,
@@ -440,6 +459,49 @@ def run_ours(args):
     del graphs
     if world > 1:
         dist.destroy_process_group()
+
+
+def memory_floors(torch, w, sh, starts, value, ref, off, logits, flush, reps=5):
+    """Times the corner rows of this workload, in kernel order, as bare
+    gathers, bare vector reductions and both (msda_debug_row_traffic): the
+    floor below which no kernel's gathers and reductions can go on this GPU.
+    fp32 rows of 128 bytes (D = 32) only; else None."""
+    from scale_deformable_attention_02_b200 import (msda_debug_row_traffic,
+                                                    msda_debug_sample_points,
+                                                    msda_forward_fused)
+    if w.value_dtype != "f32" or w.D != 32:
+        return None
+    loc = torch.empty_like(off)
+    msda_forward_fused(value, sh, starts, ref, off, logits, sampling_locations_out=loc)
+    rec = msda_debug_sample_points(sh, starts, loc)
+    rows = rec["rows"].view(w.N, w.queries, w.M, w.L * w.K * 4)
+    dev = value.device
+    n = torch.arange(w.N, device=dev, dtype=torch.int64).view(-1, 1, 1, 1)
+    m = torch.arange(w.M, device=dev, dtype=torch.int64).view(1, 1, -1, 1)
+    elem = ((n * w.S + rows) * w.M + m) * w.D
+    offs = elem[rows >= 0].to(torch.int32).contiguous()  # row-major: item, sample, corner
+    del rec, rows, elem, loc
+    grad = torch.zeros_like(value)
+    sink = torch.empty(8 * 256 * torch.cuda.get_device_properties(dev).multi_processor_count,
+                       device=dev)
+    out = {"rows": int(offs.numel()),
+           "source": "msda_debug_row_traffic on this run's corner rows, median of "
+                     f"{reps} launches after an L2 flush"}
+    for mode, key in ((0, "gather_us"), (1, "reduce_us"), (2, "gather_reduce_us")):
+        ts = []
+        for _ in range(reps + 1):
+            flush.zero_()
+            if mode:
+                grad.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            msda_debug_row_traffic(mode, offs, value=value if mode != 1 else None,
+                                   grad=grad if mode else None, sink=sink)
+            e1.record()
+            torch.cuda.synchronize()
+            ts.append(e0.elapsed_time(e1) * 1e3)
+        out[key] = statistics.median(ts[1:])
+    return out
 
 
 def _pci_bus_id(torch, device):

@@ -1,10 +1,12 @@
 /*
- * msda_debug.h -- test-support entry point of the MSDeformAttn library.
+ * msda_debug.h -- test and benchmark support of the MSDeformAttn library.
  *
- * Not part of the compute path: it exposes the per-sample cell arithmetic
- * that the forward and backward kernels share, so a test can compare the
- * integer side of the computation (pixel coordinate, cell, corner rows) bit
- * for bit with an independent implementation.
+ * Not part of the compute path.  msda_debug_sample_points exposes the
+ * per-sample cell arithmetic that the forward and backward kernels share, so
+ * a test can compare the integer side of the computation (pixel coordinate,
+ * cell, corner rows) bit for bit with an independent implementation.
+ * msda_debug_row_traffic replays a row list as bare gathers and reductions:
+ * the memory-system floor the kernels are measured against.
  */
 #ifndef MSDA_DEBUG_H
 #define MSDA_DEBUG_H
@@ -38,6 +40,35 @@ MSDA_API msda_status msda_debug_sample_points(const int64_t *spatial_shapes,
                                      int32_t *valid, int32_t *x0, int32_t *y0,
                                      float *x, float *y, int64_t *rows,
                                      msda_stream_t stream);
+
+/*
+ * The memory-system floor of the path.  Replays a list of 128-byte rows
+ * (32 fp32 elements each) in list order, with no index arithmetic:
+ *   mode 0  gather every row (what the forward's corner loads do);
+ *   mode 1  add a row of ones into grad at every row with one vector
+ *           reduction per 16 bytes (what the backward's scatter does);
+ *   mode 2  gather every row and add it into grad (the backward's memory
+ *           operations).
+ * Timing it on the corner rows of a workload gives the floor that the
+ * gathers and reductions of the kernels cannot go below on this GPU.
+ *
+ *   value, grad     device [n_value] fp32, 16-byte aligned (grad unused in
+ *                   mode 0, value unused in mode 1; either may then be NULL)
+ *   row_offsets     device [n_rows] int32 element offsets; rows that start
+ *                   below 0, end past n_value or are not 16-byte aligned are
+ *                   skipped
+ *   sink            device [sink_len] fp32, receives per-lane sums of the
+ *                   gathered rows so the loads cannot be dropped; may be NULL
+ *                   when sink_len is 0
+ *   ctas            thread blocks of 256 threads; <= 0 gives 8 per SM
+ * Errors: MSDA_ERR_NULL, MSDA_ERR_SHAPE (mode, n_rows < 0, n_value < 32,
+ * sink_len < 0), MSDA_ERR_ALIGN, MSDA_ERR_ALIAS (grad overlapping value,
+ * row_offsets or sink).
+ */
+MSDA_API msda_status msda_debug_row_traffic(int mode, const float *value, float *grad,
+                                            int64_t n_value, const int32_t *row_offsets,
+                                            int64_t n_rows, float *sink, int64_t sink_len,
+                                            int ctas, msda_stream_t stream);
 
 #ifdef __cplusplus
 }

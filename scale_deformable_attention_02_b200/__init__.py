@@ -6,11 +6,12 @@ seeded synthetic workloads used by the tests and the benchmark.
 """
 from ._lib import LIB_CHECKED_PATH, LIB_PATH, MSDA_BF16, MSDA_F32
 from .api import (MsdaError, checked_library, last_violation, msda_backward,
-                  msda_backward_fused, msda_debug_sample_points, msda_forward,
-                  msda_forward_fused, msda_level_start_index)
+                  msda_backward_fused, msda_debug_row_traffic, msda_debug_sample_points,
+                  msda_forward, msda_forward_fused, msda_level_start_index)
 
 __all__ = [
     "LIB_CHECKED_PATH", "LIB_PATH", "MSDA_BF16", "MSDA_F32", "MsdaError", "checked_library",
-    "last_violation", "msda_backward", "msda_backward_fused", "msda_debug_sample_points",
+    "last_violation", "msda_backward", "msda_backward_fused", "msda_debug_row_traffic",
+    "msda_debug_sample_points",
     "msda_forward", "msda_forward_fused", "msda_level_start_index",
 ]

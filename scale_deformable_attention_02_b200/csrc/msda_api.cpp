@@ -595,6 +595,36 @@ msda_status msda_debug_sample_points(const int64_t *spatial_shapes,
     return cuda_status(msda::launch_sample_points(p, static_cast<cudaStream_t>(stream)));
 }
 
+msda_status msda_debug_row_traffic(int mode, const float *value, float *grad, int64_t n_value,
+                                   const int32_t *row_offsets, int64_t n_rows, float *sink,
+                                   int64_t sink_len, int ctas, msda_stream_t stream)
+{
+    if (mode < 0 || mode > 2 || n_rows < 0 || n_value < 32 || sink_len < 0)
+        return MSDA_ERR_SHAPE;
+    if (n_rows > 0 && !row_offsets) return MSDA_ERR_NULL;
+    if (mode != 1 && !value) return MSDA_ERR_NULL;
+    if (mode != 0 && !grad) return MSDA_ERR_NULL;
+    if (sink_len > 0 && !sink) return MSDA_ERR_NULL;
+    if (!aligned(value, 16) || !aligned(grad, 16) || !aligned(row_offsets, 4) ||
+        !aligned(sink, 4))
+        return MSDA_ERR_ALIGN;
+    const Span outs[] = {{grad, n_value * 4}, {sink, sink_len * 4}};
+    const Span ins[] = {{value, n_value * 4}, {row_offsets, n_rows * 4}};
+    if (any_alias(outs, 2, ins, 2)) return MSDA_ERR_ALIAS;
+    if (n_rows == 0) return MSDA_OK;
+    msda::TrafficParams p;
+    memset(&p, 0, sizeof p);
+    p.value = value;
+    p.grad = grad;
+    p.rows = row_offsets;
+    p.n_rows = n_rows;
+    p.n_value = n_value;
+    p.sink = sink;
+    p.sink_len = sink_len;
+    return cuda_status(
+        msda::launch_row_traffic(p, mode, ctas, static_cast<cudaStream_t>(stream)));
+}
+
 #ifdef MSDA_CHECKED
 msda_status msda_checked_set_limit(int64_t value_elements)
 {

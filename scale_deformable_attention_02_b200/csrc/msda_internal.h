@@ -90,6 +90,19 @@ cudaError_t launch_backward(const BwdParams &p, bool bf16, int lanes_per_row,
 cudaError_t launch_backward_fused(const BwdParams &p, bool bf16, cudaStream_t stream);
 cudaError_t launch_sample_points(const PointsParams &p, cudaStream_t stream);
 
+// Row replay of msda_debug_row_traffic (msda_traffic.cu).
+struct TrafficParams {
+    const float *value;
+    float *grad;
+    const int32_t *rows;  // element offsets of 128-byte rows
+    int64_t n_rows;
+    int64_t n_value;      // elements in value and in grad
+    float *sink;          // per-lane sums of the gathered rows (nullable if sink_len == 0)
+    int64_t sink_len;
+    int64_t per_warp;     // set by the launcher
+};
+cudaError_t launch_row_traffic(TrafficParams p, int mode, int ctas, cudaStream_t stream);
+
 #ifdef MSDA_CHECKED
 // The current device's check word (two zero-initialised 64-bit counters in a
 // file-scope __device__ array), or nullptr if the runtime cannot give its

@@ -296,3 +296,19 @@ def test_grouped_argument_errors(lib):
     assert lib.msda_backward_fused_grouped(fake(0), 0, pr.sp(), pr.st(), fake(1), 2, fake(2),
                                            fake(3), fake(4), fake(5), None, None, None,
                                            pr.dims, 6, None) == SHAPE
+
+
+def test_row_traffic_argument_errors(lib):
+    """msda_debug_row_traffic rejects bad modes, sizes, pointers and aliasing
+    before any device work."""
+    f = lib.msda_debug_row_traffic
+    assert f(3, fake(0), fake(1), 64, fake(2), 10, None, 0, 0, None) == SHAPE
+    assert f(0, fake(0), None, 16, fake(2), 10, None, 0, 0, None) == SHAPE
+    assert f(0, fake(0), None, 64, fake(2), -1, None, 0, 0, None) == SHAPE
+    assert f(0, None, None, 64, fake(2), 10, None, 0, 0, None) == NULL
+    assert f(1, fake(0), None, 64, fake(2), 10, None, 0, 0, None) == NULL
+    assert f(0, fake(0), None, 64, None, 10, None, 0, 0, None) == NULL
+    assert f(0, fake(0, 8), None, 64, fake(2), 10, None, 0, 0, None) == ALIGN
+    assert f(2, fake(0), fake(0, 64), 64, fake(2), 10, None, 0, 0, None) == ALIAS
+    assert f(2, fake(0), fake(1), 64, fake(2), 10, fake(1, 16), 8, 0, None) == ALIAS
+    assert f(2, fake(0), fake(1), 64, fake(2), 0, None, 0, 0, None) == OK  # nothing to do
