@@ -482,25 +482,36 @@ def memory_floors(torch, w, sh, starts, value, ref, off, logits, flush, reps=5):
     offs = elem[rows >= 0].to(torch.int32).contiguous()  # row-major: item, sample, corner
     del rec, rows, elem, loc
     grad = torch.zeros_like(value)
-    sink = torch.empty(8 * 256 * torch.cuda.get_device_properties(dev).multi_processor_count,
+    sink = torch.empty(16 * 256 * torch.cuda.get_device_properties(dev).multi_processor_count,
                        device=dev)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    shapes = [(dp, c * sms) for dp in (4, 8, 16) for c in (4, 8, 16)]
     out = {"rows": int(offs.numel()),
-           "source": "msda_debug_row_traffic on this run's corner rows, median of "
-                     f"{reps} launches after an L2 flush"}
+           "source": "msda_debug_row_traffic on this run's corner rows: fastest of "
+                     f"{len(shapes)} (rows in flight, CTAs) launch shapes, median of {reps} "
+                     "launches each after an L2 flush"}
     for mode, key in ((0, "gather_us"), (1, "reduce_us"), (2, "gather_reduce_us")):
-        ts = []
-        for _ in range(reps + 1):
-            flush.zero_()
-            if mode:
-                grad.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            msda_debug_row_traffic(mode, offs, value=value if mode != 1 else None,
-                                   grad=grad if mode else None, sink=sink)
-            e1.record()
-            torch.cuda.synchronize()
-            ts.append(e0.elapsed_time(e1) * 1e3)
-        out[key] = statistics.median(ts[1:])
+        best = None
+        for dp, ctas in shapes:
+            ts = []
+            for _ in range(reps + 1):
+                flush.zero_()
+                if mode:
+                    grad.zero_()
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record()
+                msda_debug_row_traffic(mode, offs, value=value if mode != 1 else None,
+                                       grad=grad if mode else None, sink=sink, depth=dp,
+                                       ctas=ctas)
+                e1.record()
+                torch.cuda.synchronize()
+                ts.append(e0.elapsed_time(e1) * 1e3)
+            t = statistics.median(ts[1:])
+            if best is None or t < best[0]:
+                best = (t, dp, ctas)
+        out[key] = best[0]
+        out[key.replace("_us", "_shape")] = {"rows_in_flight": best[1], "ctas": best[2]}
     return out
 
 

@@ -60,15 +60,18 @@ MSDA_API msda_status msda_debug_sample_points(const int64_t *spatial_shapes,
  *   sink            device [sink_len] fp32, receives per-lane sums of the
  *                   gathered rows so the loads cannot be dropped; may be NULL
  *                   when sink_len is 0
+ *   depth           rows in flight per lane: 2, 4, 8 or 16 (0 gives 8)
  *   ctas            thread blocks of 256 threads; <= 0 gives 8 per SM
- * Errors: MSDA_ERR_NULL, MSDA_ERR_SHAPE (mode, n_rows < 0, n_value < 32,
- * sink_len < 0), MSDA_ERR_ALIGN, MSDA_ERR_ALIAS (grad overlapping value,
- * row_offsets or sink).
+ * A caller after the floor times a few (depth, ctas) pairs and keeps the
+ * fastest.
+ * Errors: MSDA_ERR_NULL, MSDA_ERR_SHAPE (mode, depth, n_rows < 0,
+ * n_value < 32, sink_len < 0), MSDA_ERR_ALIGN, MSDA_ERR_ALIAS (grad
+ * overlapping value, row_offsets or sink).
  */
 MSDA_API msda_status msda_debug_row_traffic(int mode, const float *value, float *grad,
                                             int64_t n_value, const int32_t *row_offsets,
                                             int64_t n_rows, float *sink, int64_t sink_len,
-                                            int ctas, msda_stream_t stream);
+                                            int depth, int ctas, msda_stream_t stream);
 
 #ifdef __cplusplus
 }

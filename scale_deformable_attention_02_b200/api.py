@@ -373,7 +373,7 @@ def msda_debug_sample_points(spatial_shapes, level_start_index,
 
 def msda_debug_row_traffic(mode: int, rows: torch.Tensor, value: torch.Tensor | None = None,
                            grad: torch.Tensor | None = None, sink: torch.Tensor | None = None,
-                           ctas: int = 0, stream=None) -> None:
+                           depth: int = 0, ctas: int = 0, stream=None) -> None:
     """Replay 128-byte rows (int32 element offsets `rows`) as bare gathers
     (mode 0), vector reductions of a row of ones into `grad` (mode 1), or
     both (mode 2): the memory-system floor of the kernels (include/msda_debug.h)."""
@@ -392,5 +392,5 @@ def msda_debug_row_traffic(mode: int, rows: torch.Tensor, value: torch.Tensor | 
         _need(sink, "sink", tuple(sink.shape), dev)
     _check(_lib.load().msda_debug_row_traffic(
         int(mode), _dptr(value), _dptr(grad), n_value, _dptr(rows), rows.numel(), _dptr(sink),
-        0 if sink is None else sink.numel(), int(ctas), _stream_handle(dev, stream)),
+        0 if sink is None else sink.numel(), int(depth), int(ctas), _stream_handle(dev, stream)),
         "msda_debug_row_traffic")

@@ -597,9 +597,11 @@ msda_status msda_debug_sample_points(const int64_t *spatial_shapes,
 
 msda_status msda_debug_row_traffic(int mode, const float *value, float *grad, int64_t n_value,
                                    const int32_t *row_offsets, int64_t n_rows, float *sink,
-                                   int64_t sink_len, int ctas, msda_stream_t stream)
+                                   int64_t sink_len, int depth, int ctas, msda_stream_t stream)
 {
     if (mode < 0 || mode > 2 || n_rows < 0 || n_value < 32 || sink_len < 0)
+        return MSDA_ERR_SHAPE;
+    if (depth != 0 && depth != 2 && depth != 4 && depth != 8 && depth != 16)
         return MSDA_ERR_SHAPE;
     if (n_rows > 0 && !row_offsets) return MSDA_ERR_NULL;
     if (mode != 1 && !value) return MSDA_ERR_NULL;
@@ -622,7 +624,7 @@ msda_status msda_debug_row_traffic(int mode, const float *value, float *grad, in
     p.sink = sink;
     p.sink_len = sink_len;
     return cuda_status(
-        msda::launch_row_traffic(p, mode, ctas, static_cast<cudaStream_t>(stream)));
+        msda::launch_row_traffic(p, mode, depth, ctas, static_cast<cudaStream_t>(stream)));
 }
 
 #ifdef MSDA_CHECKED

@@ -703,6 +703,12 @@ cudaError_t launch_fast_r(const FwdParams &p, cudaStream_t stream)
     return launch_fast<VT, EPL, R, 32, kFused>(p, stream);
 }
 
+// Items of up to this many samples take the fast path; larger ones the wide
+// kernel's one-warp-per-item loop.
+#ifndef MSDA_FWD_FAST_MAX_LK
+#define MSDA_FWD_FAST_MAX_LK 32
+#endif
+
 // Elements per lane for bf16 values: 8 (16-byte loads, 2x the rows per
 // instruction) or 4 (8-byte loads, the fp32 lane layout).
 #ifndef MSDA_FWD_BF16_EPL
@@ -745,7 +751,7 @@ cudaError_t launch_fwd_vt(const FwdParams &p, int R, cudaStream_t stream)
     if (p.L * p.K > kLaneLK) return launch_long<VT, 16 / (int)sizeof(VT), kFused>(p, stream);
     // fast path: rows of at most 8 lanes of EPL elements
     const int lanes = (p.D + EPL - 1) / EPL;
-    if (p.D % EPL == 0 && lanes <= 8) {
+    if (p.D % EPL == 0 && lanes <= 8 && p.L * p.K <= MSDA_FWD_FAST_MAX_LK) {
         FwdParams q = p;
         q.nchunks = lanes;
         if (lanes <= 1) return launch_fast_r<VT, EPL, 1, kFused>(q, stream);

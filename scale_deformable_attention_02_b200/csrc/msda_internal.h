@@ -101,7 +101,8 @@ struct TrafficParams {
     int64_t sink_len;
     int64_t per_warp;     // set by the launcher
 };
-cudaError_t launch_row_traffic(TrafficParams p, int mode, int ctas, cudaStream_t stream);
+cudaError_t launch_row_traffic(TrafficParams p, int mode, int depth, int ctas,
+                               cudaStream_t stream);
 
 #ifdef MSDA_CHECKED
 // The current device's check word (two zero-initialised 64-bit counters in a

@@ -11,11 +11,10 @@ namespace {
 
 // Warps sweep contiguous ranges of the row list; eight lanes move one row
 // (16 bytes each), so a warp instruction covers four rows, and each lane
-// keeps eight rows in flight.
-template <int MODE>  // 0: gather, 1: reduce a row of ones, 2: gather and reduce it
+// keeps kB rows in flight.
+template <int MODE, int kB>  // MODE 0: gather, 1: reduce a row of ones, 2: both; kB rows in flight
 __global__ void __launch_bounds__(256) row_traffic_kernel(const __grid_constant__ TrafficParams p)
 {
-    constexpr int kB = 8;
     const int lane = threadIdx.x & 31;
     const int64_t gw = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int slot = lane >> 3, chunk = lane & 7;
@@ -48,9 +47,24 @@ __global__ void __launch_bounds__(256) row_traffic_kernel(const __grid_constant_
 
 }  // namespace
 
-cudaError_t launch_row_traffic(TrafficParams p, int mode, int ctas, cudaStream_t stream)
+template <int MODE>
+cudaError_t launch_mode(const TrafficParams &p, int depth, int ctas, cudaStream_t stream)
+{
+    switch (depth) {
+    case 2: row_traffic_kernel<MODE, 2><<<ctas, 256, 0, stream>>>(p); break;
+    case 4: row_traffic_kernel<MODE, 4><<<ctas, 256, 0, stream>>>(p); break;
+    case 8: row_traffic_kernel<MODE, 8><<<ctas, 256, 0, stream>>>(p); break;
+    case 16: row_traffic_kernel<MODE, 16><<<ctas, 256, 0, stream>>>(p); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_row_traffic(TrafficParams p, int mode, int depth, int ctas,
+                               cudaStream_t stream)
 {
     if (p.n_rows == 0) return cudaSuccess;
+    if (depth <= 0) depth = 8;
     if (ctas <= 0) {
         int dev = 0, sms = 148;
         if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -60,14 +74,13 @@ cudaError_t launch_row_traffic(TrafficParams p, int mode, int ctas, cudaStream_t
     }
     const int64_t warps = (int64_t)ctas * 8;
     p.per_warp = (p.n_rows + warps - 1) / warps;
-    p.per_warp = (p.per_warp + 31) / 32 * 32;
+    p.per_warp = (p.per_warp + 63) / 64 * 64;
     switch (mode) {
-    case 0: row_traffic_kernel<0><<<ctas, 256, 0, stream>>>(p); break;
-    case 1: row_traffic_kernel<1><<<ctas, 256, 0, stream>>>(p); break;
-    case 2: row_traffic_kernel<2><<<ctas, 256, 0, stream>>>(p); break;
+    case 0: return launch_mode<0>(p, depth, ctas, stream);
+    case 1: return launch_mode<1>(p, depth, ctas, stream);
+    case 2: return launch_mode<2>(p, depth, ctas, stream);
     default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace msda

@@ -299,16 +299,20 @@ def test_grouped_argument_errors(lib):
 
 
 def test_row_traffic_argument_errors(lib):
-    """msda_debug_row_traffic rejects bad modes, sizes, pointers and aliasing
-    before any device work."""
-    f = lib.msda_debug_row_traffic
-    assert f(3, fake(0), fake(1), 64, fake(2), 10, None, 0, 0, None) == SHAPE
-    assert f(0, fake(0), None, 16, fake(2), 10, None, 0, 0, None) == SHAPE
-    assert f(0, fake(0), None, 64, fake(2), -1, None, 0, 0, None) == SHAPE
-    assert f(0, None, None, 64, fake(2), 10, None, 0, 0, None) == NULL
-    assert f(1, fake(0), None, 64, fake(2), 10, None, 0, 0, None) == NULL
-    assert f(0, fake(0), None, 64, None, 10, None, 0, 0, None) == NULL
-    assert f(0, fake(0, 8), None, 64, fake(2), 10, None, 0, 0, None) == ALIGN
-    assert f(2, fake(0), fake(0, 64), 64, fake(2), 10, None, 0, 0, None) == ALIAS
-    assert f(2, fake(0), fake(1), 64, fake(2), 10, fake(1, 16), 8, 0, None) == ALIAS
-    assert f(2, fake(0), fake(1), 64, fake(2), 0, None, 0, 0, None) == OK  # nothing to do
+    """msda_debug_row_traffic rejects bad modes, depths, sizes, pointers and
+    aliasing before any device work."""
+    def f(mode, value, grad, n_value, rows, n_rows, sink=None, sink_len=0, depth=0):
+        return lib.msda_debug_row_traffic(mode, value, grad, n_value, rows, n_rows, sink,
+                                          sink_len, depth, 0, None)
+
+    assert f(3, fake(0), fake(1), 64, fake(2), 10) == SHAPE
+    assert f(0, fake(0), None, 16, fake(2), 10) == SHAPE
+    assert f(0, fake(0), None, 64, fake(2), -1) == SHAPE
+    assert f(0, fake(0), None, 64, fake(2), 10, depth=3) == SHAPE
+    assert f(0, None, None, 64, fake(2), 10) == NULL
+    assert f(1, fake(0), None, 64, fake(2), 10) == NULL
+    assert f(0, fake(0), None, 64, None, 10) == NULL
+    assert f(0, fake(0, 8), None, 64, fake(2), 10) == ALIGN
+    assert f(2, fake(0), fake(0, 64), 64, fake(2), 10) == ALIAS
+    assert f(2, fake(0), fake(1), 64, fake(2), 10, fake(1, 16), 8) == ALIAS
+    assert f(2, fake(0), fake(1), 64, fake(2), 0) == OK  # nothing to do
