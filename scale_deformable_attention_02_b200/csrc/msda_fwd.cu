@@ -682,6 +682,161 @@ cudaError_t launch_long(FwdParams p, cudaStream_t stream)
     return go(fwd_kernel_long<VT, EPL, 32, kFused>);
 }
 
+// ---------------------------------------------------------------------------
+// Items of 17..32 samples, rows of at most 8 lanes: one warp per item and a
+// grid over all items (no persistent loop), two corner-row groups in flight,
+// so the kernel needs few registers and the GPU keeps 48 (fp32) or 64 (bf16)
+// warps per SM in flight.  On B200 that beats the fast kernel for these items
+// (stress workload, bf16: 2.06 ms against 2.53 ms; fp32 L*K = 32: 6-7%
+// faster), while for items of at most 16 samples the fast kernel's batching
+// wins (encoder: 181 us against 218 us).
+// ---------------------------------------------------------------------------
+#ifndef MSDA_FWD_ITEM_BATCH
+#define MSDA_FWD_ITEM_BATCH 2  // corner-row groups loaded before the first is used
+#endif
+
+// Resident CTAs of 8 warps per SM: bf16 at 32 registers (64 warps per SM),
+// fp32 at 40 (48 warps), the best of the measured shapes.
+template <typename VT>
+constexpr int item_min_ctas()
+{
+    return sizeof(VT) == 2 ? 8 : 6;
+}
+
+template <typename VT, int EPL, int R, bool kFused>
+__global__ void __launch_bounds__(kWarps * 32, item_min_ctas<VT>())
+    fwd_kernel_item(const __grid_constant__ FwdParams p)
+{
+    using LL = LaneLoad<VT, EPL>;
+    constexpr int kSlots = 32 / R;  // (sample, corner) pairs per warp instruction
+    constexpr int kNP = EPL / 2;
+    constexpr int kStride = 34;     // corner-major entries, conflict-free
+    __shared__ int2 ent[kWarps][4 * kStride];
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t item = (int64_t)blockIdx.x * kWarps + warp;
+    if (item >= p.items) return;  // whole warp; no block-wide barrier follows
+    const int M = p.M, D = p.D, K = p.K;
+    const int LK = p.L * K;
+    const int MD = M * D;
+    const int m = (int)(item % M);
+    const int64_t nq = item / M;
+    const int64_t n = nq / p.Lq;
+
+    // ---- phase 1: sample `lane` -------------------------------------------
+    {
+        const bool act = lane < LK;
+        const int64_t si = item * LK + lane;                               // per head
+        const int64_t sl = msda_loc_item(item, M, p.G, p.Hg) * LK + lane;  // per group
+        const int l = act ? lane / K : 0;
+        const int H = p.lv.H[l], W = p.lv.W[l], start = p.lv.start[l];
+        float lx = 0.f, ly = 0.f, a = 0.f;
+        if constexpr (kFused) {
+            const float z = act ? __ldcs(p.logits + si) : -INFINITY;
+            const float mx = warp_max(z);
+            const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
+            const float sum = warp_sum(e);
+            a = __fdiv_rn(e, sum);
+            if (act) {
+                const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sl);
+                if (p.ref_dim == 2) {
+                    const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
+                    lx = __fadd_rn(r.x, __fdiv_rn(o.x, (float)W));
+                    ly = __fadd_rn(r.y, __fdiv_rn(o.y, (float)H));
+                } else {
+                    const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
+                    const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
+                    lx = __fadd_rn(c.x, __fmul_rn(o.x, s2.x));
+                    ly = __fadd_rn(c.y, __fmul_rn(o.y, s2.y));
+                }
+                if (p.loc_out && (p.Hg == 1 || m % p.Hg == 0))  // the group's first head
+                    __stcs(reinterpret_cast<float2 *>(p.loc_out) + sl, make_float2(lx, ly));
+                if (p.attn_out) __stcs(p.attn_out + si, a);
+            }
+        } else if (act) {
+            const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + sl);
+            lx = t.x;
+            ly = t.y;
+            a = __ldcs(p.attn + si);
+        }
+        int2 e[4] = {{-1, 0}, {-1, 0}, {-1, 0}, {-1, 0}};
+        float x, y, fx, fy;
+        int x0, y0;
+        if (act && msda_cell(lx, ly, H, W, x, y, x0, y0, fx, fy)) {
+            const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+            const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int r = msda_row(start, H, W, y0 + (c >> 1), x0 + (c & 1));
+                if (r >= 0) e[c] = make_int2(r * MD, __float_as_int(w[c] * a));
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) ent[warp][c * kStride + lane] = e[c];
+    }
+    __syncwarp();
+
+    // ---- phase 2: the item's (sample, corner) pairs, four loads in flight ----
+    const int slot = lane / R;
+    const int chunk = lane % R;
+    const bool chunk_ok = chunk < p.nchunks;
+    const int lane_elem = (chunk_ok ? chunk : 0) * EPL;
+    const int64_t vbe = (n * p.S * M + m) * (int64_t)D + lane_elem;
+    const VT *vb = static_cast<const VT *>(p.value) + vbe;
+    float2 acc[kNP];
+#pragma unroll
+    for (int i = 0; i < kNP; ++i) acc[i] = make_float2(0.f, 0.f);
+    constexpr int kB = MSDA_FWD_ITEM_BATCH;
+    static_assert(128 % (kB * kSlots) == 0, "a batch must tile the entries");
+    const int npairs = 4 * LK;
+    for (int t0 = 0; t0 < npairs; t0 += kB * kSlots) {
+        int2 e[kB];
+        typename LL::Raw raw[kB];
+#pragma unroll
+        for (int b = 0; b < kB; ++b) {
+            const int t = t0 + b * kSlots + slot;  // < 128: entries past L*K hold -1
+            e[b] = ent[warp][(t & 3) * kStride + (t >> 2)];
+            if (e[b].x >= 0 && !msda_in_map(p.check, p.check_limit, vbe + e[b].x, EPL))
+                e[b].x = -1;  // bounds-checked build: skipped, reads as zero
+            if (e[b].x >= 0) raw[b] = LL::load(vb + e[b].x);
+        }
+#pragma unroll
+        for (int b = 0; b < kB; ++b) {
+            if (e[b].x >= 0) {
+                float2 v[kNP];
+                LL::widen(raw[b], v);
+                const float wb = __int_as_float(e[b].y);
+                const float2 w2 = make_float2(wb, wb);
+#pragma unroll
+                for (int i = 0; i < kNP; ++i) acc[i] = __ffma2_rn(w2, v[i], acc[i]);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = R; o < 32; o <<= 1)
+#pragma unroll
+        for (int i = 0; i < kNP; ++i) {
+            acc[i].x += __shfl_xor_sync(kFull, acc[i].x, o);
+            acc[i].y += __shfl_xor_sync(kFull, acc[i].y, o);
+        }
+    if (slot == 0 && chunk_ok) {
+        float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D + chunk * EPL);
+#pragma unroll
+        for (int i = 0; i < kNP / 2; ++i)
+            __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
+                                        acc[2 * i + 1].y));
+    }
+}
+
+template <typename VT, int EPL, int R, bool kFused>
+cudaError_t launch_item(const FwdParams &p, cudaStream_t stream)
+{
+    const dim3 grid((unsigned)((p.items + kWarps - 1) / kWarps));
+    fwd_kernel_item<VT, EPL, R, kFused><<<grid, kWarps * 32, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
 template <typename VT, int EPL, int R, int P, bool kFused>
 cudaError_t launch_fast(FwdParams p, cudaStream_t stream)
 {
@@ -692,12 +847,17 @@ cudaError_t launch_fast(FwdParams p, cudaStream_t stream)
     return cudaGetLastError();
 }
 
+#ifndef MSDA_FWD_ITEM_MIN_LK
+#define MSDA_FWD_ITEM_MIN_LK 17  // items of at least this many samples: fwd_kernel_item
+#endif
+
 template <typename VT, int EPL, int R, bool kFused>
 cudaError_t launch_fast_r(const FwdParams &p, cudaStream_t stream)
 {
     // P: a power of two >= L*K, >= 8 (conflict-free entry stride) and >= the
     // 8/R samples one warp instruction gathers
     const int LK = p.L * p.K;
+    if (LK >= MSDA_FWD_ITEM_MIN_LK) return launch_item<VT, EPL, R, kFused>(p, stream);
     if (LK <= 8) return launch_fast<VT, EPL, R, 8, kFused>(p, stream);
     if (LK <= 16) return launch_fast<VT, EPL, R, 16, kFused>(p, stream);
     return launch_fast<VT, EPL, R, 32, kFused>(p, stream);
