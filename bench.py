@@ -534,12 +534,15 @@ def _nvml_index(local: int) -> int:
 
 def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_dev, queries):
     """The same step through the public binding, starting from pinned host
-    buffers: H2D of the step's inputs, fused forward, backward, D2H of the
-    step's results (out, grad_value, grad_sampling_locations,
-    grad_attention_weights), all inside the timed events."""
+    buffers: every step copies its inputs host -> device, runs the fused
+    forward and the backward, and copies its results (out and the gradients)
+    device -> host, all inside the timed events.  Steps are pipelined over
+    two device buffer sets and three streams (copy in, compute, copy out), so
+    step i+1's upload and step i-1's download overlap step i's kernels."""
     from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fused,
                                                     msda_forward_fused)
     fused = args.step == "fused"
+    nbuf = 2
 
     def pinned(a):
         a = np.ascontiguousarray(a)
@@ -548,41 +551,68 @@ def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_
 
     names = ["value", "reference_points", "offsets", "logits", "grad_out"]
     h_in = {k: pinned(inp[k]) for k in names}
-    d_in = {k: torch.empty(h_in[k].shape, dtype=h_in[k].dtype, device=device) for k in names}
     res_shapes = {"out": (w.N, w.queries, w.M * w.D), "grad_value": (w.N, w.S, w.M, w.D),
                   "grad_loc": tuple(inp["offsets"].shape), "grad_attn": tuple(inp["logits"].shape)}
     if fused:
         res_shapes["grad_ref"] = tuple(inp["reference_points"].shape)
     h_out = {k: torch.empty(s, dtype=torch.float32).pin_memory() for k, s in res_shapes.items()}
-    d_out = {k: torch.empty(s, dtype=torch.float32, device=device) for k, s in res_shapes.items()}
-    loc = torch.empty(tuple(inp["offsets"].shape), device=device)
-    attn = torch.empty(tuple(inp["logits"].shape), device=device)
+    bufs = []
+    for _ in range(nbuf):
+        bufs.append({
+            "in": {k: torch.empty(h_in[k].shape, dtype=h_in[k].dtype, device=device)
+                   for k in names},
+            "out": {k: torch.empty(s, dtype=torch.float32, device=device)
+                    for k, s in res_shapes.items()},
+            "loc": torch.empty(tuple(inp["offsets"].shape), device=device),
+            "attn": torch.empty(tuple(inp["logits"].shape), device=device),
+            "loaded": torch.cuda.Event(), "computed": torch.cuda.Event(),
+            "stored": torch.cuda.Event(), "used": False,
+        })
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    s_comp = stream
     bf16 = w.value_dtype == "bf16"
 
-    def one():
-        for k in names:
-            d_in[k].copy_(h_in[k], non_blocking=True)
+    def compute(b):
+        d_in, d_out = b["in"], b["out"]
         v = d_in["value"].view(torch.bfloat16) if bf16 else d_in["value"]
         if fused:
             msda_forward_fused(v, sh, starts, d_in["reference_points"], d_in["offsets"],
-                               d_in["logits"], out=d_out["out"], stream=stream)
+                               d_in["logits"], out=d_out["out"], stream=s_comp)
             msda_backward_fused(v, sh, starts, d_in["reference_points"], d_in["offsets"],
                                 d_in["logits"], d_in["grad_out"], grad_value=d_out["grad_value"],
                                 grad_reference_points=d_out["grad_ref"],
                                 grad_offsets=d_out["grad_loc"], grad_logits=d_out["grad_attn"],
-                                stream=stream)
+                                stream=s_comp)
         else:
             msda_forward_fused(v, sh, starts, d_in["reference_points"], d_in["offsets"],
-                               d_in["logits"], out=d_out["out"], sampling_locations_out=loc,
-                               attention_weights_out=attn, stream=stream)
-            msda_backward(v, sh, starts, loc, attn, d_in["grad_out"],
+                               d_in["logits"], out=d_out["out"], sampling_locations_out=b["loc"],
+                               attention_weights_out=b["attn"], stream=s_comp)
+            msda_backward(v, sh, starts, b["loc"], b["attn"], d_in["grad_out"],
                           grad_value=d_out["grad_value"], grad_sampling_locations=d_out["grad_loc"],
-                          grad_attention_weights=d_out["grad_attn"], stream=stream)
-        for k in res_shapes:
-            h_out[k].copy_(d_out[k], non_blocking=True)
+                          grad_attention_weights=d_out["grad_attn"], stream=s_comp)
 
-    for _ in range(2):
-        one()
+    def step(i):
+        b = bufs[i % nbuf]
+        if b["used"]:
+            s_in.wait_event(b["computed"])    # step i-2 has read this input set
+        with torch.cuda.stream(s_in):
+            for k in names:
+                b["in"][k].copy_(h_in[k], non_blocking=True)
+        b["loaded"].record(s_in)
+        s_comp.wait_event(b["loaded"])
+        if b["used"]:
+            s_comp.wait_event(b["stored"])    # step i-2's results have left this set
+        compute(b)
+        b["computed"].record(s_comp)
+        s_out.wait_event(b["computed"])
+        with torch.cuda.stream(s_out):
+            for k in res_shapes:
+                h_out[k].copy_(b["out"][k], non_blocking=True)
+        b["stored"].record(s_out)
+        b["used"] = True
+
+    for i in range(2 * nbuf):
+        step(i)
     torch.cuda.synchronize()
     n = max(1, args.e2e_steps)
     e0 = torch.cuda.Event(enable_timing=True)
@@ -590,10 +620,14 @@ def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(n):
-        one()
-    e1.record(stream)
+    e0.record(s_in)
+    s_comp.wait_event(e0)
+    s_out.wait_event(e0)
+    for i in range(n):
+        step(i)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_comp)
+    e1.record(s_out)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -602,8 +636,10 @@ def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_
     d2h = sum(h_out[k].numel() * h_out[k].element_size() for k in res_shapes)
     return {"value": queries * world / (ms / 1e3), "unit": "queries/s", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
-            "api": "scale_deformable_attention_02_b200.msda_forward_fused + msda_backward "
-                   "on pinned host buffers copied in and out every step"}
+            "pipelining": f"{nbuf} device buffer sets; copy-in, compute and copy-out streams",
+            "api": "scale_deformable_attention_02_b200.msda_forward_fused + "
+                   + ("msda_backward_fused" if fused else "msda_backward")
+                   + " on pinned host buffers copied in and out every step"}
 
 
 # ---------------------------------------------------------------------------

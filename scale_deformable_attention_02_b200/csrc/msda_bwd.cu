@@ -328,18 +328,22 @@ struct Lane4<__nv_bfloat16> {
 #ifndef MSDA_BWD_MIN_CTAS
 #define MSDA_BWD_MIN_CTAS 3
 #endif
+#ifndef MSDA_BWD_MIN_CTAS_F32
+#define MSDA_BWD_MIN_CTAS_F32 2
+#endif
 
-// Resident CTAs of 8 warps per SM.  The fused variant carries the chain rule's
-// state as well: fp32 runs it at 2 CTAs (128 registers, no spills; encoder
-// 556 -> 529 us), bf16 keeps 3 (its value chunks take half the registers).
-template <typename VT, bool kFused>
+// Resident CTAs of 8 warps per SM.  fp32 rows of eight lanes (D = 32) run at
+// 2 CTAs (128 registers, no spills; encoder backward 471 -> 448 us, fused
+// 556 -> 529 us on B200); bf16, whose value chunks take half the registers,
+// and narrower rows, which need fewer, are fastest at 3.
+template <typename VT, int R>
 constexpr int bwd_min_ctas()
 {
-    return (kFused && sizeof(VT) == 4) ? 2 : MSDA_BWD_MIN_CTAS;
+    return (sizeof(VT) == 4 && R == 8) ? MSDA_BWD_MIN_CTAS_F32 : MSDA_BWD_MIN_CTAS;
 }
 
 template <typename VT, int R, int P, bool kFused>
-__global__ void __launch_bounds__(kWarps * 32, bwd_min_ctas<VT, kFused>())
+__global__ void __launch_bounds__(kWarps * 32, bwd_min_ctas<VT, R>())
     bwd_kernel(const __grid_constant__ BwdParams p)
 {
     static_assert(R <= 8, "fast path: at least four pairs per warp instruction");
