@@ -416,24 +416,12 @@ __global__ void __launch_bounds__(kWarps * 32, bwd_min_ctas<VT, R>())
             if constexpr (kFused) {
                 // the fused forward's softmax and location map, bit for bit
                 const float ox = pl_x, oy = pl_y;
-                const float z = act ? pa : -INFINITY;
-                const float mx = seg_max<P>(z);
-                const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
-                const float sum = seg_sum<P>(e);
-                a = __fdiv_rn(e, sum);
+                a = seg_softmax<P>(pa, act);
                 lx = ly = 0.f;
                 if (act) {
-                    const int64_t nq = item / M;
-                    if (p.ref_dim == 2) {
-                        const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
-                        lx = __fadd_rn(r.x, __fdiv_rn(ox, (float)W));
-                        ly = __fadd_rn(r.y, __fdiv_rn(oy, (float)H));
-                    } else {
-                        const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
-                        const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
-                        lx = __fadd_rn(c.x, __fmul_rn(ox, s2.x));
-                        ly = __fadd_rn(c.y, __fmul_rn(oy, s2.y));
-                    }
+                    const float2 loc = msda_fused_location(p.ref, p.ref_dim, item / M, ox, oy, H, W);
+                    lx = loc.x;
+                    ly = loc.y;
                 }
                 smq[warp][seg][j] = make_float4(act ? a : 0.f, ox, oy, 0.f);
             }
@@ -694,15 +682,9 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
                             __ldcs(reinterpret_cast<const float2 *>(p.off) + lbase + s);
                         ox = o.x;
                         oy = o.y;
-                        if (p.ref_dim == 2) {
-                            const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
-                            lx = __fadd_rn(r.x, __fdiv_rn(ox, (float)W));
-                            ly = __fadd_rn(r.y, __fdiv_rn(oy, (float)H));
-                        } else {
-                            const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
-                            lx = __fadd_rn(c.x, __fmul_rn(ox, bwh.x));
-                            ly = __fadd_rn(c.y, __fmul_rn(oy, bwh.y));
-                        }
+                        const float2 loc = msda_fused_location(p.ref, p.ref_dim, nq, ox, oy, H, W);
+                        lx = loc.x;
+                        ly = loc.y;
                     }
                     smq[warp][lane] = make_float4(a, ox, oy, 0.f);
                 } else if (act) {

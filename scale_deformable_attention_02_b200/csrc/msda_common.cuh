@@ -39,6 +39,27 @@ __device__ __forceinline__ bool msda_cell(float lx, float ly, int H, int W, floa
     return true;
 }
 
+// Sampling location of one sample of the fused path ("Deformable DETR" wiki
+// page: the reference point plus the predicted offset, "Multi-scale
+// deformable attention"; offsets scaled by the box in iterative refinement,
+// "Variants").  Point reference ref[nq] = (x, y) with offsets in pixels of a
+// level of H x W: loc = ref + off / (W, H).  Box reference
+// ref[nq] = (cx, cy, w, h) with offsets in box units: loc = (cx, cy) +
+// off * (w, h).  Each component is one IEEE fp32 divide or multiply, then one
+// fp32 add, so every kernel forms the same bits.
+__device__ __forceinline__ float2 msda_fused_location(const float *ref, int ref_dim, int64_t nq,
+                                                      float ox, float oy, int H, int W)
+{
+    if (ref_dim == 2) {
+        const float2 r = __ldg(reinterpret_cast<const float2 *>(ref) + nq);
+        return make_float2(__fadd_rn(r.x, __fdiv_rn(ox, (float)W)),
+                           __fadd_rn(r.y, __fdiv_rn(oy, (float)H)));
+    }
+    const float2 c = __ldg(reinterpret_cast<const float2 *>(ref) + 2 * nq);
+    const float2 s = __ldg(reinterpret_cast<const float2 *>(ref) + 2 * nq + 1);
+    return make_float2(__fadd_rn(c.x, __fmul_rn(ox, s.x)), __fadd_rn(c.y, __fmul_rn(oy, s.y)));
+}
+
 // Bounds check of one access to the value map (or to grad_value, which has
 // the same layout): value elements [first, first + count) against [0, limit).
 // Only the bounds-checked build (-DMSDA_CHECKED) tests anything: there an
@@ -170,6 +191,22 @@ __device__ __forceinline__ float seg_sum(float v)
 #pragma unroll
     for (int o = P / 2; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
     return v;
+}
+
+// Joint softmax weight of this lane's sample over its aligned segment of P
+// lanes, which holds the L*K logits of one (query, head) ("Deformable DETR"
+// wiki page, "Multi-scale deformable attention": the weights of a head sum to
+// one over all levels and points).  Max-subtracted; lanes with act false hold
+// no sample and add nothing.  Every kernel with at most 32 samples per item
+// forms its weights here, so the fused forward and backward agree bit for bit.
+template <int P>
+__device__ __forceinline__ float seg_softmax(float logit, bool act)
+{
+    const float z = act ? logit : -INFINITY;
+    const float mx = seg_max<P>(z);
+    const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
+    const float sum = seg_sum<P>(e);
+    return __fdiv_rn(e, sum);
 }
 
 // Joint softmax statistics of one item of more than 32 samples, held by one

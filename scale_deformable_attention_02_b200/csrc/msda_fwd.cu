@@ -128,27 +128,13 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
             const int l = act ? j / K : 0;
             float lx = 0.f, ly = 0.f, a = 0.f;
             if constexpr (kFused) {
-                const float z = act ? __ldcs(p.logits + si) : -INFINITY;
-                const float mx = seg_max<P>(z);
-                const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
-                const float s = seg_sum<P>(e);
-                a = __fdiv_rn(e, s);
+                a = seg_softmax<P>(act ? __ldcs(p.logits + si) : 0.f, act);
                 if (act) {
                     const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sl);
-                    const int64_t nq = item / M;
-                    if (p.ref_dim == 2) {
-                        // point reference: offsets are level-l pixels
-                        const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
-                        lx = __fadd_rn(r.x, __fdiv_rn(o.x, (float)sW[l]));
-                        ly = __fadd_rn(r.y, __fdiv_rn(o.y, (float)sH[l]));
-                    } else {
-                        // box reference (cx, cy, w, h): offsets are in box units
-                        const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
-                        const float2 s2 =
-                            __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
-                        lx = __fadd_rn(c.x, __fmul_rn(o.x, s2.x));
-                        ly = __fadd_rn(c.y, __fmul_rn(o.y, s2.y));
-                    }
+                    const float2 loc =
+                        msda_fused_location(p.ref, p.ref_dim, item / M, o.x, o.y, sH[l], sW[l]);
+                    lx = loc.x;
+                    ly = loc.y;
                     if (p.loc_out && (p.Hg == 1 || (item % M) % p.Hg == 0))  // group's first head
                         __stcs(reinterpret_cast<float2 *>(p.loc_out) + sl, make_float2(lx, ly));
                     if (p.attn_out) __stcs(p.attn_out + si, a);
@@ -399,27 +385,12 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
         const int64_t si = item * LK + j;
         float lx, ly, a;
         if constexpr (kFused) {
-            // joint softmax over the item's L*K logits, max-subtracted
-            const float z = act ? pa : -INFINITY;
-            const float mx = seg_max<P>(z);
-            const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
-            const float sum = seg_sum<P>(e);
-            a = __fdiv_rn(e, sum);
+            a = seg_softmax<P>(pa, act);  // joint over the item's L*K logits
             lx = ly = 0.f;
             if (act) {
-                const int64_t nq = item / M;
-                if (p.ref_dim == 2) {
-                    // point reference: offsets are level-l pixels
-                    const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
-                    lx = __fadd_rn(r.x, __fdiv_rn(pb, (float)W));
-                    ly = __fadd_rn(r.y, __fdiv_rn(pc, (float)H));
-                } else {
-                    // box reference (cx, cy, w, h): offsets are in box units
-                    const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
-                    const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
-                    lx = __fadd_rn(c.x, __fmul_rn(pb, s2.x));
-                    ly = __fadd_rn(c.y, __fmul_rn(pc, s2.y));
-                }
+                const float2 loc = msda_fused_location(p.ref, p.ref_dim, item / M, pb, pc, H, W);
+                lx = loc.x;
+                ly = loc.y;
                 if (p.loc_out && (p.Hg == 1 || (item % M) % p.Hg == 0))  // group's first head
                     __stcs(reinterpret_cast<float2 *>(p.loc_out) +
                                msda_loc_item(item, M, p.G, p.Hg) * LK + j,
@@ -579,17 +550,9 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
                     if constexpr (kFused) {
                         a = __fdiv_rn(pick<kNB>(z, blk), sum);
                         const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sl);
-                        if (p.ref_dim == 2) {
-                            const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
-                            lx = __fadd_rn(r.x, __fdiv_rn(o.x, (float)W));
-                            ly = __fadd_rn(r.y, __fdiv_rn(o.y, (float)H));
-                        } else {
-                            const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
-                            const float2 s2 =
-                                __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
-                            lx = __fadd_rn(c.x, __fmul_rn(o.x, s2.x));
-                            ly = __fadd_rn(c.y, __fmul_rn(o.y, s2.y));
-                        }
+                        const float2 loc = msda_fused_location(p.ref, p.ref_dim, nq, o.x, o.y, H, W);
+                        lx = loc.x;
+                        ly = loc.y;
                         if (p.loc_out && first_head)
                             __stcs(reinterpret_cast<float2 *>(p.loc_out) + sl, make_float2(lx, ly));
                         if (p.attn_out) __stcs(p.attn_out + si, a);
@@ -733,23 +696,12 @@ __global__ void __launch_bounds__(kWarps * 32, item_min_ctas<VT>())
         const int H = p.lv.H[l], W = p.lv.W[l], start = p.lv.start[l];
         float lx = 0.f, ly = 0.f, a = 0.f;
         if constexpr (kFused) {
-            const float z = act ? __ldcs(p.logits + si) : -INFINITY;
-            const float mx = warp_max(z);
-            const float e = act ? expf(__fsub_rn(z, mx)) : 0.f;
-            const float sum = warp_sum(e);
-            a = __fdiv_rn(e, sum);
+            a = seg_softmax<32>(act ? __ldcs(p.logits + si) : 0.f, act);
             if (act) {
                 const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sl);
-                if (p.ref_dim == 2) {
-                    const float2 r = __ldg(reinterpret_cast<const float2 *>(p.ref) + nq);
-                    lx = __fadd_rn(r.x, __fdiv_rn(o.x, (float)W));
-                    ly = __fadd_rn(r.y, __fdiv_rn(o.y, (float)H));
-                } else {
-                    const float2 c = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq);
-                    const float2 s2 = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
-                    lx = __fadd_rn(c.x, __fmul_rn(o.x, s2.x));
-                    ly = __fadd_rn(c.y, __fmul_rn(o.y, s2.y));
-                }
+                const float2 loc = msda_fused_location(p.ref, p.ref_dim, nq, o.x, o.y, H, W);
+                lx = loc.x;
+                ly = loc.y;
                 if (p.loc_out && (p.Hg == 1 || m % p.Hg == 0))  // the group's first head
                     __stcs(reinterpret_cast<float2 *>(p.loc_out) + sl, make_float2(lx, ly));
                 if (p.attn_out) __stcs(p.attn_out + si, a);
