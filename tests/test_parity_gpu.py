@@ -254,7 +254,20 @@ CASES = [
 ]
 
 
-@pytest.mark.parametrize("case", CASES, ids=[f"case{i}" for i in range(len(CASES))])
+# Larger problems (16800 (query, head) items, several rounds per persistent
+# warp): every lane layout of the fast kernels.
+LARGE_CASES = [
+    (1, 4200, 4, 4, 4, ((9, 11), (5, 6), (3, 3)), "f32"),    # R = 1
+    (1, 4200, 4, 8, 4, ((9, 11), (5, 6), (3, 3)), "f32"),    # R = 2
+    (1, 4200, 4, 16, 4, ((9, 11), (5, 6), (3, 3)), "f32"),   # R = 4
+    (1, 2100, 8, 32, 2, ((12, 14), (6, 7)), "f32"),          # R = 8, L*K = 4
+    (1, 4200, 4, 16, 4, ((9, 11), (5, 6), (3, 3)), "bf16"),  # 16-byte bf16 rows
+]
+
+
+@pytest.mark.parametrize("case", CASES + LARGE_CASES,
+                         ids=[f"case{i}" for i in range(len(CASES))] +
+                             [f"large{i}" for i in range(len(LARGE_CASES))])
 def test_random_problems(case):
     N, Lq, M, D, K, shapes, dt = case
     d = wl.make_random_problem(1000 + len(shapes) * 7 + D, N=N, Lq=Lq, M=M, D=D, K=K,
