@@ -107,16 +107,18 @@ def max_over_ranks(vals, world: int, device):
 # ---------------------------------------------------------------------------
 # algorithmic (unique) bytes per launch
 # ---------------------------------------------------------------------------
-def algorithmic_bytes(w: wl.Workload, step: str = "split") -> dict:
+def algorithmic_bytes(w: wl.Workload, step: str = "split", touched_rows=None) -> dict:
     """Minimum HBM traffic of each launch: every input read once, every
-    output written once (the value map counted once although its rows are
-    gathered many times; the backward's zero-fill of grad_value is not
-    counted).  split: the forward also writes locations and weights, which
-    the backward reads; fused: neither pass stores them."""
+    output written once.  The value map counts once per (pixel, head) row
+    that some sample touches (all rows when touched_rows is None), although
+    its rows are gathered many times; grad_value is an output of every row;
+    the backward's zero-fill of it is not counted.  split: the forward also
+    writes locations and weights, which the backward reads; fused: neither
+    pass stores them."""
     N, Lq, S, M, D, L, K = (w.N, w.queries, w.S, w.M, w.D, w.L, w.K)
     esz = 2 if w.value_dtype == "bf16" else 4
     samples = N * Lq * M * L * K
-    value = N * S * M * D * esz
+    value = (N * S * M if touched_rows is None else touched_rows) * D * esz
     gvalue = N * S * M * D * 4
     ref = N * Lq * 2 * 4
     outb = N * Lq * M * D * 4
@@ -378,8 +380,10 @@ def run_ours(args):
                       queries)
 
     # ---- roofline of the dominant launch ----------------------------------
+    offs = corner_rows(torch, w, sh, starts, value, ref, off, logits)
+    touched = int(torch.unique(offs).numel())
     peak, peak_kind = read_peaks()
-    ab = algorithmic_bytes(w, args.step)
+    ab = algorithmic_bytes(w, args.step, touched)
     dom = "bwd" if ms_bwd >= ms_fwd else "fwd"
     dom_ms = ms_bwd if dom == "bwd" else ms_fwd
     achieved = ab[dom] / (dom_ms / 1e3) / 1e9
@@ -397,7 +401,8 @@ def run_ours(args):
         k["frac_of_" + peak_kind] = k["GB_s"] / peak
     roofline = {
         "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-        "frac": achieved / peak, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
+        "frac": achieved / peak, "frac_of_nominal_8000": achieved / 8000.0,
+        "value_rows_touched": touched, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
         if peak_kind == "measured" else "fallback 6.65 TB/s",
         "traffic": read_traffic(args.workload if args.step == "split" else
                                 args.workload + "/fused", dom),
@@ -407,10 +412,11 @@ def run_ours(args):
 
     floors = None
     if not args.no_floors:
-        floors = memory_floors(torch, w, sh, starts, value, ref, off, logits, flush)
+        floors = memory_floors(torch, w, offs, value, flush)
         if floors:
             kernels["fwd"]["frac_of_row_floor"] = floors["gather_us"] / (ms_fwd * 1e3)
             kernels["bwd"]["frac_of_row_floor"] = floors["gather_reduce_us"] / (ms_bwd * 1e3)
+    del offs
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -461,26 +467,31 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def memory_floors(torch, w, sh, starts, value, ref, off, logits, flush, reps=5):
-    """Times the corner rows of this workload, in kernel order, as bare
-    gathers, bare vector reductions and both (msda_debug_row_traffic): the
-    floor below which no kernel's gathers and reductions can go on this GPU.
-    fp32 rows of 128 bytes (D = 32) only; else None."""
-    from scale_deformable_attention_02_b200 import (msda_debug_row_traffic,
-                                                    msda_debug_sample_points,
-                                                    msda_forward_fused)
-    if w.value_dtype != "f32" or w.D != 32:
-        return None
+def corner_rows(torch, w, sh, starts, value, ref, off, logits):
+    """The in-level corner rows of every sample of the workload, in kernel
+    order, as element offsets into the value map (int64, on the device), from
+    the kernels' own cell arithmetic (msda_debug_sample_points)."""
+    from scale_deformable_attention_02_b200 import msda_debug_sample_points, msda_forward_fused
     loc = torch.empty_like(off)
     msda_forward_fused(value, sh, starts, ref, off, logits, sampling_locations_out=loc)
-    rec = msda_debug_sample_points(sh, starts, loc)
-    rows = rec["rows"].view(w.N, w.queries, w.M, w.L * w.K * 4)
+    rows = msda_debug_sample_points(sh, starts, loc)["rows"].view(w.N, w.queries, w.M, -1)
     dev = value.device
     n = torch.arange(w.N, device=dev, dtype=torch.int64).view(-1, 1, 1, 1)
     m = torch.arange(w.M, device=dev, dtype=torch.int64).view(1, 1, -1, 1)
     elem = ((n * w.S + rows) * w.M + m) * w.D
-    offs = elem[rows >= 0].to(torch.int32).contiguous()  # row-major: item, sample, corner
-    del rec, rows, elem, loc
+    return elem[rows >= 0]  # row-major: item, sample, corner
+
+
+def memory_floors(torch, w, offs, value, flush, reps=5):
+    """Times the corner rows of this workload, in kernel order, as bare
+    gathers, bare vector reductions and both (msda_debug_row_traffic): the
+    floor below which no kernel's gathers and reductions can go on this GPU.
+    fp32 rows of 128 bytes (D = 32) only; else None."""
+    from scale_deformable_attention_02_b200 import msda_debug_row_traffic
+    if w.value_dtype != "f32" or w.D != 32:
+        return None
+    dev = value.device
+    offs = offs.to(torch.int32).contiguous()
     grad = torch.zeros_like(value)
     sink = torch.empty(16 * 256 * torch.cuda.get_device_properties(dev).multi_processor_count,
                        device=dev)
@@ -675,11 +686,21 @@ def cpu_baseline(w, inp, min_seconds: float = 10.0):
         el = time.perf_counter() - t0
         if el >= min_seconds or passes >= 20:
             break
+    # one thread, on every 16th query
+    oracle.set_threads(1)
+    s1 = _oracle_sample(w, inp, 16)
+    t1 = time.perf_counter()
+    _oracle_step(oracle, s1)
+    el1 = time.perf_counter() - t1
+    oracle.set_threads(threads)
     return {"value": s["queries"] * passes / el, "unit": "queries/s", "cores": threads,
             "kind": "oracle",
             "sample": f"{passes} full pass(es) of the workload ({s['queries']} queries each: "
                       f"fused forward + backward) on the plain C oracle, fp64 accumulation, "
-                      f"OpenMP over {threads} threads, {el:.1f} s"}
+                      f"OpenMP over {threads} threads, {el:.1f} s",
+            "single_thread": {"value": s1["queries"] / el1, "unit": "queries/s", "cores": 1,
+                              "sample": f"every 16th query ({s1['queries']} queries), one pass, "
+                                        f"{el1:.1f} s"}}
 
 
 def run_reference(args):
