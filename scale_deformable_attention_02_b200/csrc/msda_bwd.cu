@@ -37,33 +37,6 @@ struct __align__(16) CornerB {
     float dwy;  // d w / d fy
 };
 
-// A raw 16-byte chunk of a value row, widened to fp32 (bf16 widening is exact).
-template <typename VT>
-__device__ __forceinline__ void widen(const uint4 &r, float (&v)[Chunk<VT>::kVec]);
-
-template <>
-__device__ __forceinline__ void widen<float>(const uint4 &r, float (&v)[4])
-{
-    v[0] = __uint_as_float(r.x);
-    v[1] = __uint_as_float(r.y);
-    v[2] = __uint_as_float(r.z);
-    v[3] = __uint_as_float(r.w);
-}
-
-template <>
-__device__ __forceinline__ void widen<__nv_bfloat16>(const uint4 &r, float (&v)[8])
-{
-    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        v[2 * i] = __uint_as_float(w[i] << 16);
-        v[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-    }
-}
-
-// 512 bytes of zeros: the row that corners outside the level read.
-__device__ __align__(128) float4 kZeroRowB[32] = {};
-
 // Butterfly reduce-scatter over aligned groups of SPAN lanes.  Before: every
 // lane holds N partial values.  After: lane (lane % SPAN) = b holds, in
 // v[0 .. N/SPAN), the group totals of values b*N/SPAN .. (b+1)*N/SPAN - 1.
