@@ -809,7 +809,6 @@ cudaError_t launch_fast_r(const FwdParams &p, cudaStream_t stream)
     // P: a power of two >= L*K, >= 8 (conflict-free entry stride) and >= the
     // 8/R samples one warp instruction gathers
     const int LK = p.L * p.K;
-    if (LK >= MSDA_FWD_ITEM_MIN_LK) return launch_item<VT, EPL, R, kFused>(p, stream);
     if (LK <= 8) return launch_fast<VT, EPL, R, 8, kFused>(p, stream);
     if (LK <= 16) return launch_fast<VT, EPL, R, 16, kFused>(p, stream);
     return launch_fast<VT, EPL, R, 32, kFused>(p, stream);
@@ -821,11 +820,25 @@ cudaError_t launch_fast_r(const FwdParams &p, cudaStream_t stream)
 #define MSDA_FWD_FAST_MAX_LK 32
 #endif
 
-// Elements per lane for bf16 values: 8 (16-byte loads, 2x the rows per
-// instruction) or 4 (8-byte loads, the fp32 lane layout).
-#ifndef MSDA_FWD_BF16_EPL
-#define MSDA_FWD_BF16_EPL 8
-#endif
+template <typename VT, int EPL, bool kFused>
+cudaError_t launch_item_r(FwdParams p, int lanes, cudaStream_t stream)
+{
+    p.nchunks = lanes;
+    if (lanes <= 1) return launch_item<VT, EPL, 1, kFused>(p, stream);
+    if (lanes <= 2) return launch_item<VT, EPL, 2, kFused>(p, stream);
+    if (lanes <= 4) return launch_item<VT, EPL, 4, kFused>(p, stream);
+    return launch_item<VT, EPL, 8, kFused>(p, stream);
+}
+
+template <typename VT, int EPL, bool kFused>
+cudaError_t launch_fast_lanes(FwdParams p, int lanes, cudaStream_t stream)
+{
+    p.nchunks = lanes;
+    if (lanes <= 1) return launch_fast_r<VT, EPL, 1, kFused>(p, stream);
+    if (lanes <= 2) return launch_fast_r<VT, EPL, 2, kFused>(p, stream);
+    if (lanes <= 4) return launch_fast_r<VT, EPL, 4, kFused>(p, stream);
+    return launch_fast_r<VT, EPL, 8, kFused>(p, stream);
+}
 
 template <typename VT, int R, int P, bool kFused>
 cudaError_t launch_p(FwdParams p, bool exact, cudaStream_t stream)
@@ -859,17 +872,19 @@ cudaError_t launch_r(const FwdParams &p, bool exact, cudaStream_t stream)
 template <typename VT, bool kFused>
 cudaError_t launch_fwd_vt(const FwdParams &p, int R, cudaStream_t stream)
 {
-    constexpr int EPL = sizeof(VT) == 4 ? 4 : MSDA_FWD_BF16_EPL;
-    if (p.L * p.K > kLaneLK) return launch_long<VT, 16 / (int)sizeof(VT), kFused>(p, stream);
-    // fast path: rows of at most 8 lanes of EPL elements
-    const int lanes = (p.D + EPL - 1) / EPL;
-    if (p.D % EPL == 0 && lanes <= 8 && p.L * p.K <= MSDA_FWD_FAST_MAX_LK) {
-        FwdParams q = p;
-        q.nchunks = lanes;
-        if (lanes <= 1) return launch_fast_r<VT, EPL, 1, kFused>(q, stream);
-        if (lanes <= 2) return launch_fast_r<VT, EPL, 2, kFused>(q, stream);
-        if (lanes <= 4) return launch_fast_r<VT, EPL, 4, kFused>(q, stream);
-        return launch_fast_r<VT, EPL, 8, kFused>(q, stream);
+    constexpr int E16 = 16 / (int)sizeof(VT);  // elements of a 16-byte lane
+    const int LK = p.L * p.K;
+    if (LK > kLaneLK) return launch_long<VT, E16, kFused>(p, stream);
+    // items of 17..32 samples, rows of at most eight 16-byte lanes
+    if (LK >= MSDA_FWD_ITEM_MIN_LK && p.D % E16 == 0 && p.D / E16 <= 8)
+        return launch_item_r<VT, E16, kFused>(p, p.D / E16, stream);
+    // fast path: lanes of four elements where a row needs at most eight of
+    // them (bf16: 8-byte loads, 5% faster on the encoder than 16-byte lanes),
+    // else 16-byte lanes
+    if (LK <= MSDA_FWD_FAST_MAX_LK) {
+        if (p.D % 4 == 0 && p.D / 4 <= 8) return launch_fast_lanes<VT, 4, kFused>(p, p.D / 4, stream);
+        if (E16 != 4 && p.D % E16 == 0 && p.D / E16 <= 8)
+            return launch_fast_lanes<VT, E16, kFused>(p, p.D / E16, stream);
     }
     const bool exact = p.nchunks == R;
     switch (R) {
