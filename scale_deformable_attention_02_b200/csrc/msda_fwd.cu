@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
     const int M = p.M, D = p.D, K = p.K;
     const int LK = p.L * K;
     const int MD = M * D;
-    const int npairs = 4 * LK;
+    static_assert(kSlots % 4 == 0, "a warp instruction covers whole samples");
 
     // phase-1 role: sample j of the round's item `seg`
     const int seg = lane / P;
@@ -435,13 +435,15 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
             float2 acc[kNP];
 #pragma unroll
             for (int i = 0; i < kNP; ++i) acc[i] = make_float2(0.f, 0.f);
-            for (int t0 = 0; t0 < npairs; t0 += kB * kSlots) {
+            // pair t = (sample t/4, corner t%4); slot s takes corner s%4 of sample
+            // s/4 + kSlots/4 * (instruction), so its entries sit at one lane base
+            const int2 *enl = en + (slot & 3) * kStride + (slot >> 2);
+            for (int s0 = 0; s0 < LK; s0 += kB * (kSlots / 4)) {
                 int2 e[kB];
                 typename LL::Raw raw[kB];
 #pragma unroll
                 for (int b = 0; b < kB; ++b) {
-                    const int t = t0 + b * kSlots + slot;  // pair (sample t/4, corner t%4)
-                    e[b] = en[(t & 3) * kStride + (t >> 2)];
+                    e[b] = enl[s0 + b * (kSlots / 4)];
                     if (e[b].x >= 0 && !msda_in_map(p.check, p.check_limit, vbe + e[b].x, EPL))
                         e[b].x = -1;  // bounds-checked build: skipped, reads as zero
                     if (e[b].x >= 0) raw[b] = LL::load(vb + e[b].x);
@@ -741,14 +743,16 @@ __global__ void __launch_bounds__(kWarps * 32, item_min_ctas<VT>())
     for (int i = 0; i < kNP; ++i) acc[i] = make_float2(0.f, 0.f);
     constexpr int kB = MSDA_FWD_ITEM_BATCH;
     static_assert(128 % (kB * kSlots) == 0, "a batch must tile the entries");
-    const int npairs = 4 * LK;
-    for (int t0 = 0; t0 < npairs; t0 += kB * kSlots) {
+    static_assert(kSlots % 4 == 0, "a warp instruction covers whole samples");
+    // slot s takes corner s%4 of samples s/4, s/4 + kSlots/4, ... (entries
+    // past L*K hold -1)
+    const int2 *enl = ent[warp] + (slot & 3) * kStride + (slot >> 2);
+    for (int s0 = 0; s0 < LK; s0 += kB * (kSlots / 4)) {
         int2 e[kB];
         typename LL::Raw raw[kB];
 #pragma unroll
         for (int b = 0; b < kB; ++b) {
-            const int t = t0 + b * kSlots + slot;  // < 128: entries past L*K hold -1
-            e[b] = ent[warp][(t & 3) * kStride + (t >> 2)];
+            e[b] = enl[s0 + b * (kSlots / 4)];
             if (e[b].x >= 0 && !msda_in_map(p.check, p.check_limit, vbe + e[b].x, EPL))
                 e[b].x = -1;  // bounds-checked build: skipped, reads as zero
             if (e[b].x >= 0) raw[b] = LL::load(vb + e[b].x);
