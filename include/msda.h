@@ -241,9 +241,8 @@ MSDA_API msda_status msda_backward(const void *value, msda_dtype value_dtype,
  *   grad_offsets            NULL or device [N,Lq,M,L,K,2] fp32 (written)
  *   grad_logits             NULL or device [N,Lq,M,L,K] fp32 (written)
  *
- * Limits: D <= 32 for either value dtype (MSDA_ERR_UNSUPPORTED otherwise).
- * Errors: as msda_forward_fused; every gradient buffer is an output for the
- * alias check.
+ * Limits: as msda_forward_fused.  Errors: as msda_forward_fused; every
+ * gradient buffer is an output for the alias check.
  */
 MSDA_API msda_status msda_backward_fused(const void *value, msda_dtype value_dtype,
                                          const int64_t *spatial_shapes,

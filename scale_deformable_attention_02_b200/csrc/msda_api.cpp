@@ -396,7 +396,6 @@ msda_status backward_fused_impl(const void *value, msda_dtype value_dtype,
     if (st != MSDA_OK) return st;
     if ((st = check_groups(d, G, &pr)) != MSDA_OK) return st;
     if (reference_dim != 2 && reference_dim != 4) return MSDA_ERR_SHAPE;
-    if (d.D > 32) return MSDA_ERR_UNSUPPORTED;
     if (pr.n_value > 0 && !grad_value) return MSDA_ERR_NULL;
     if (pr.n_out > 0 && (!reference_points || !offsets || !logits || !grad_out))
         return MSDA_ERR_NULL;
@@ -448,7 +447,7 @@ msda_status backward_fused_impl(const void *value, msda_dtype value_dtype,
     p.grad_logits = grad_logits;
     set_dims(&p, d, G, pr);
     if ((st = set_checks(&p, pr)) != MSDA_OK) return st;
-    return launched(msda::launch_backward_fused(p, value_dtype == MSDA_BF16, s), s);
+    return launched(msda::launch_backward_fused(p, value_dtype == MSDA_BF16, pr.lanes, s), s);
 }
 
 }  // namespace

@@ -82,7 +82,7 @@ __device__ __forceinline__ void reduce_scatter_n(float (&v)[N], int lane)
 // reduced every 8 samples.  Used for rows wider than 128 bytes.  The item's
 // samples are taken in blocks of 32 (one per lane in phase 1), so any L*K up
 // to kMaxLK works.
-template <typename VT, int R>
+template <typename VT, int R, bool kFused>
 __global__ void __launch_bounds__(kWarps * 32)
     bwd_kernel_wide(const __grid_constant__ BwdParams p)
 {
@@ -92,10 +92,15 @@ __global__ void __launch_bounds__(kWarps * 32)
     constexpr int kCornerSlots = kSpan / R;           // 4, 2 or 1
     constexpr int kCpl = 4 / kCornerSlots;            // corners per lane
     constexpr int kPer = kNV / kSpan;                 // finished sums per lane
+    constexpr int kNB = kMaxLK / 32;
 
     __shared__ CornerB corners[kWarps][32 * 4];
     __shared__ float sA[kWarps][32];
     __shared__ int sH[kMaxLevels], sW[kMaxLevels], sStart[kMaxLevels];
+    // fused: every sample's weight and its gradient, and the block's offsets
+    __shared__ float sAll[kWarps][kFused ? kMaxLK : 1];
+    __shared__ float sdA[kWarps][kFused ? kMaxLK : 1];
+    __shared__ float2 sOff[kWarps][kFused ? 32 : 1];
 
     const int tid = threadIdx.x;
     if (tid < p.L) {
@@ -144,6 +149,27 @@ __global__ void __launch_bounds__(kWarps * 32)
 
     const int64_t litem = msda_loc_item(item, M, p.G, p.Hg);
     const bool shared_loc = p.Hg > 1;
+
+    float2 bwh = make_float2(0.f, 0.f);       // fused, box reference: (w, h)
+    float rx = 0.f, ry = 0.f, rw = 0.f, rh = 0.f;  // fused: this lane's reference-point terms
+    if constexpr (kFused) {
+        // the joint softmax over all L*K logits, as the fused forward forms it
+        float z[kNB];
+#pragma unroll
+        for (int b = 0; b < kNB; ++b) {
+            const int s = b * 32 + lane;
+            z[b] = s < LK ? __ldcs(p.logits + item * LK + s) : -INFINITY;
+        }
+        const float sum = long_softmax<kNB>(z);
+#pragma unroll
+        for (int b = 0; b < kNB; ++b) {
+            const int s = b * 32 + lane;
+            if (s < LK) sAll[warp][s] = __fdiv_rn(z[b], sum);
+        }
+        if (p.ref_dim == 4) bwh = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
+        __syncwarp();
+    }
+
     for (int blk0 = 0; blk0 < LK; blk0 += 32) {
         const int nb = LK - blk0 < 32 ? LK - blk0 : 32;  // samples in this block
         const int64_t sbase = item * LK + blk0;   // per head
@@ -152,8 +178,16 @@ __global__ void __launch_bounds__(kWarps * 32)
         if (lane < nb) {
             const int l = (blk0 + lane) / K;
             const int H = sH[l], W = sW[l], start = sStart[l];
-            const float2 t = __ldg(reinterpret_cast<const float2 *>(p.loc) + lbase + lane);
-            sA[warp][lane] = __ldg(p.attn + sbase + lane);
+            float2 t;
+            if constexpr (kFused) {
+                const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + lbase + lane);
+                t = msda_fused_location(p.ref, p.ref_dim, nq, o.x, o.y, H, W);
+                sA[warp][lane] = sAll[warp][blk0 + lane];
+                sOff[warp][lane] = o;
+            } else {
+                t = __ldg(reinterpret_cast<const float2 *>(p.loc) + lbase + lane);
+                sA[warp][lane] = __ldg(p.attn + sbase + lane);
+            }
             CornerB c[4] = {{-1, 0.f, 0.f, 0.f}, {-1, 0.f, 0.f, 0.f}, {-1, 0.f, 0.f, 0.f},
                             {-1, 0.f, 0.f, 0.f}};
             float x, y, fx, fy;
@@ -222,22 +256,73 @@ __global__ void __launch_bounds__(kWarps * 32)
                 const int s = b0 + it * kGroups + grp;
                 if (qty < 3 && s < nb) {
                     const int64_t si = sbase + s;
+                    const float a = sA[warp][s];
                     if (qty == 0) {
-                        if (p.grad_attn) p.grad_attn[si] = v[i];
-                    } else if (p.grad_loc) {
-                        const int l = (blk0 + s) / K;
-                        const float scale = (qty == 1) ? (float)sW[l] : (float)sH[l];
-                        float *dst = p.grad_loc + 2 * (lbase + s) + (qty - 1);
-                        const float gl = sA[warp][s] * (scale * v[i]);
-                        if (shared_loc)
-                            atomicAdd(dst, gl);  // the group's heads add into one location
+                        if constexpr (kFused)
+                            sdA[warp][blk0 + s] = v[i];
+                        else if (p.grad_attn)
+                            p.grad_attn[si] = v[i];
+                        continue;
+                    }
+                    const int l = (blk0 + s) / K;
+                    const float scale = (qty == 1) ? (float)sW[l] : (float)sH[l];
+                    const float gl = a * (scale * v[i]);  // d loc
+                    float go = gl;                        // the value written per location
+                    float *base = p.grad_loc;
+                    if constexpr (kFused) {
+                        base = p.grad_off;
+                        if (p.ref_dim == 2) {
+                            go = a * v[i];  // loc = ref + off / W_l: d off = d loc / W_l
+                        } else {
+                            const float2 o = sOff[warp][s];
+                            go = gl * (qty == 1 ? bwh.x : bwh.y);  // loc = c + off * (w, h)
+                            if (qty == 1)
+                                rw = fmaf(gl, o.x, rw);
+                            else
+                                rh = fmaf(gl, o.y, rh);
+                        }
+                        if (qty == 1)
+                            rx += gl;
                         else
-                            *dst = gl;
+                            ry += gl;
+                    }
+                    if (base) {
+                        float *dst = base + 2 * (lbase + s) + (qty - 1);
+                        if (shared_loc)
+                            atomicAdd(dst, go);  // the group's heads add into one location
+                        else
+                            *dst = go;
                     }
                 }
             }
         }
         __syncwarp();  // the next block overwrites corners and weights
+    }
+
+    if constexpr (kFused) {
+        // softmax Jacobian over all L*K samples: d z_s = A_s (dA_s - sum_j A_j dA_j)
+        float dpart = 0.f;
+        for (int s = lane; s < LK; s += 32) dpart = fmaf(sAll[warp][s], sdA[warp][s], dpart);
+        const float dot = warp_sum(dpart);
+        if (p.grad_logits)
+            for (int s = lane; s < LK; s += 32)
+                __stcs(p.grad_logits + item * LK + s, sAll[warp][s] * (sdA[warp][s] - dot));
+        // reference point: sum over this head's samples, then add over heads
+        rx = warp_sum(rx);
+        ry = warp_sum(ry);
+        if (p.ref_dim == 4) {
+            rw = warp_sum(rw);
+            rh = warp_sum(rh);
+        }
+        if (lane == 0 && p.grad_ref) {
+            float *gr = p.grad_ref + nq * p.ref_dim;
+            atomicAdd(gr, rx);
+            atomicAdd(gr + 1, ry);
+            if (p.ref_dim == 4) {
+                atomicAdd(gr + 2, rw);
+                atomicAdd(gr + 3, rh);
+            }
+        }
     }
 }
 
@@ -825,11 +910,30 @@ cudaError_t launch_fast_r(const BwdParams &p, cudaStream_t stream)
     return launch_fast<VT, R, 32, kFused>(p, stream);
 }
 
+// Rows wider than the fast path's eight 4-element lanes (or not a multiple
+// of 4 elements): one warp per item, R lanes of 16 bytes per row.
+template <typename VT, bool kFused>
+cudaError_t launch_wide(const BwdParams &p, int R, cudaStream_t stream)
+{
+    const dim3 block(kWarps * 32);
+    const dim3 grid((unsigned)((p.items + kWarps - 1) / kWarps));
+    switch (R) {
+    case 1: bwd_kernel_wide<VT, 1, kFused><<<grid, block, 0, stream>>>(p); break;
+    case 2: bwd_kernel_wide<VT, 2, kFused><<<grid, block, 0, stream>>>(p); break;
+    case 4: bwd_kernel_wide<VT, 4, kFused><<<grid, block, 0, stream>>>(p); break;
+    case 8: bwd_kernel_wide<VT, 8, kFused><<<grid, block, 0, stream>>>(p); break;
+    case 16: bwd_kernel_wide<VT, 16, kFused><<<grid, block, 0, stream>>>(p); break;
+    case 32: bwd_kernel_wide<VT, 32, kFused><<<grid, block, 0, stream>>>(p); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
 template <typename VT>
-cudaError_t launch_bwd_fused_vt(const BwdParams &p, cudaStream_t stream)
+cudaError_t launch_bwd_fused_vt(const BwdParams &p, int R, cudaStream_t stream)
 {
     const int r4 = p.D / 4;
-    if (p.D % 4 != 0 || r4 > 8) return cudaErrorInvalidValue;
+    if (p.D % 4 != 0 || r4 > 8) return launch_wide<VT, true>(p, R, stream);
     if (p.L * p.K > kLaneLK) return launch_long<VT, true>(p, stream);
     BwdParams q = p;
     q.nchunks = r4;
@@ -853,27 +957,17 @@ cudaError_t launch_bwd_vt(const BwdParams &p, int R, cudaStream_t stream)
         if (r4 <= 4) return launch_fast_r<VT, 4>(q, stream);
         return launch_fast_r<VT, 8>(q, stream);
     }
-    const dim3 block(kWarps * 32);
-    const dim3 grid((unsigned)((p.items + kWarps - 1) / kWarps));
-    switch (R) {
-    case 1: bwd_kernel_wide<VT, 1><<<grid, block, 0, stream>>>(p); break;
-    case 2: bwd_kernel_wide<VT, 2><<<grid, block, 0, stream>>>(p); break;
-    case 4: bwd_kernel_wide<VT, 4><<<grid, block, 0, stream>>>(p); break;
-    case 8: bwd_kernel_wide<VT, 8><<<grid, block, 0, stream>>>(p); break;
-    case 16: bwd_kernel_wide<VT, 16><<<grid, block, 0, stream>>>(p); break;
-    case 32: bwd_kernel_wide<VT, 32><<<grid, block, 0, stream>>>(p); break;
-    default: return cudaErrorInvalidValue;
-    }
-    return cudaGetLastError();
+    return launch_wide<VT, false>(p, R, stream);
 }
 
 }  // namespace
 
-cudaError_t launch_backward_fused(const BwdParams &p, bool bf16, cudaStream_t stream)
+cudaError_t launch_backward_fused(const BwdParams &p, bool bf16, int lanes_per_row,
+                                  cudaStream_t stream)
 {
     if (p.items == 0) return cudaSuccess;
-    return bf16 ? launch_bwd_fused_vt<__nv_bfloat16>(p, stream)
-                : launch_bwd_fused_vt<float>(p, stream);
+    return bf16 ? launch_bwd_fused_vt<__nv_bfloat16>(p, lanes_per_row, stream)
+                : launch_bwd_fused_vt<float>(p, lanes_per_row, stream);
 }
 
 cudaError_t launch_backward(const BwdParams &p, bool bf16, int lanes_per_row,

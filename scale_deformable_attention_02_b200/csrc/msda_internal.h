@@ -85,9 +85,9 @@ cudaError_t launch_forward(const FwdParams &p, bool bf16, bool fused, int lanes_
                            cudaStream_t stream);
 cudaError_t launch_backward(const BwdParams &p, bool bf16, int lanes_per_row,
                             cudaStream_t stream);
-// Backward of the fused forward (chained to ref, offsets and logits); needs
-// D <= 32 (returns cudaErrorInvalidValue otherwise, caught by the host checks).
-cudaError_t launch_backward_fused(const BwdParams &p, bool bf16, cudaStream_t stream);
+// Backward of the fused forward (chained to ref, offsets and logits).
+cudaError_t launch_backward_fused(const BwdParams &p, bool bf16, int lanes_per_row,
+                                  cudaStream_t stream);
 cudaError_t launch_sample_points(const PointsParams &p, cudaStream_t stream);
 
 // Row replay of msda_debug_row_traffic (msda_traffic.cu).

@@ -264,10 +264,6 @@ def test_backward_fused_argument_errors(lib):
     assert call(go=fake(2)) == ALIAS           # grad_offsets over the offsets
     assert call(gz=fake(5, 64)) == ALIAS       # grad_logits inside grad_value
     assert call(gr=fake(6), go=fake(6, 8)) == ALIAS
-    wide = Prob(D=64)
-    assert lib.msda_backward_fused(fake(0), 0, wide.sp(), wide.st(), fake(1), 2, fake(2),
-                                   fake(3), fake(4), fake(5), None, None, None, wide.dims,
-                                   None) == UNSUP
     assert lib.msda_backward_fused(fake(0), 0, pr.sp(), pr.st(), None, 2, fake(2), fake(3),
                                    fake(4), fake(5), None, None, None, pr.dims, None) == NULL
 

@@ -67,7 +67,8 @@ def test_fused_backward_point_random():
 
 
 @pytest.mark.parametrize("D,dt", [(8, "f32"), (16, "f32"), (24, "f32"), (8, "bf16"),
-                                  (32, "bf16")])
+                                  (32, "bf16"), (36, "f32"), (64, "f32"), (128, "f32"),
+                                  (64, "bf16"), (256, "bf16")])
 def test_fused_backward_widths(D, dt):
     d = wl.make_random_problem(40 + D, N=1, Lq=29, M=3, D=D, K=3,
                                shapes=((9, 11), (5, 6), (3, 3)), value_dtype=dt)
@@ -136,3 +137,18 @@ def test_fused_backward_matches_fused_forward_sampling():
     lhs = float((g * out).sum())
     rhs = float((gv * value.float()).sum())
     assert abs(lhs - rhs) <= 1e-5 * (1 + abs(lhs))
+
+
+@pytest.mark.parametrize("D,K,box", [(64, 12, False), (128, 4, True), (64, 4, True)])
+def test_fused_backward_wide_rows(D, K, box):
+    """Rows wider than 128 bytes (one warp per item, 16-byte lanes), with more
+    than 32 samples per item and with box references."""
+    shapes = ((8, 8), (4, 4), (2, 2))
+    d = wl.make_random_problem(120 + D + K, N=2, Lq=9, M=2, D=D, K=K, shapes=shapes)
+    ref, off = d["reference_points"], d["offsets"]
+    if box:
+        rng = np.random.default_rng(121)
+        ref = np.concatenate([rng.uniform(0.1, 0.9, (2, 9, 2)),
+                              rng.uniform(0.05, 0.5, (2, 9, 2))], axis=-1).astype(np.float32)
+        off = (rng.standard_normal(off.shape) * 0.25).astype(np.float32)
+    _check(d, ref, off, d["logits"], box=box)
