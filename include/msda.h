@@ -149,8 +149,8 @@ MSDA_API msda_status msda_forward(const void *value, msda_dtype value_dtype,
  *
  *  - A[n,q,m,:,:] = softmax over the L*K logits of head m, jointly across
  *    levels ("Deformable DETR" wiki page, "Multi-scale deformable attention":
- *    sum_l sum_k A_mlqk = 1; "Deformable attention module": the last MK
- *    channels of the 3MK query projection go through a softmax).
+ *    sum_l sum_k A_mlqk = 1; "Deformable attention module": the query
+ *    projection's final MK channels are normalised by a softmax).
  *  - loc = phi_l(p_q) + dp in level-l pixels, i.e. in normalised units
  *    loc_x = ref_x + off_x / W_l and loc_y = ref_y + off_y / H_l (fp32 IEEE
  *    divide, then fp32 add) ("Deformable DETR" wiki page, "Multi-scale
@@ -187,7 +187,7 @@ MSDA_API msda_status msda_forward_fused(const void *value, msda_dtype value_dtyp
  * Backward of msda_forward: gradients flow through the bilinear
  * interpolation to the value map, to the sampling locations and to the
  * attention weights ("Deformable DETR" wiki page, "Deformable attention
- * module": interpolation makes the offsets differentiable; "Deformable
+ * module": the interpolation lets gradients reach the offsets; "Deformable
  * Attention" glossary page: the interpolation passes gradients on to the
  * offset prediction).  With g = grad_out[n,q,m*D:(m+1)*D] and corner weights w_j:
  *   grad_attention_weights = sum_j w_j <v_j, g>

@@ -312,8 +312,8 @@ void ora_locations_f64(const double *ref, const double *off, const int64_t *shap
 /*
  * Backward of ora_forward: the gradients flow through the interpolation to
  * the value, the locations and the weights ("Deformable DETR" wiki page,
- * "Deformable attention module": the interpolation makes the offsets
- * differentiable; "Deformable Attention" glossary page: the interpolation
+ * "Deformable attention module": the interpolation lets gradients reach
+ * the offsets; "Deformable Attention" glossary page: the interpolation
  * passes gradients on to the offset prediction).
  *
  * With g = grad_out[n,q,m,:] and corner weights w_j(fx, fy):

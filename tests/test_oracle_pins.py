@@ -226,7 +226,7 @@ def test_multi_level_equals_weighted_grid_samples():
 
 
 def test_points_on_every_pixel_is_dense_attention():
-    """When the sampling points cover every location the module is ordinary
+    """With a sampling point on every location the module reduces to ordinary
     attention ("Deformable DETR" wiki page, "Multi-scale deformable
     attention"): K = H*W points on the pixel centres of a power-of-two map
     give out[m] = A[m] @ V[:, m, :], a plain matrix-vector product."""
