@@ -486,13 +486,14 @@ def memory_floors(torch, w, offs, value, flush, reps=5):
     """Times the corner rows of this workload, in kernel order, as bare
     gathers, bare vector reductions and both (msda_debug_row_traffic): the
     floor below which no kernel's gathers and reductions can go on this GPU.
-    fp32 rows of 128 bytes (D = 32) only; else None."""
+    Rows of 32 elements (D = 32: fp32 or bf16 value, fp32 gradient) only;
+    else None."""
     from scale_deformable_attention_02_b200 import msda_debug_row_traffic
-    if w.value_dtype != "f32" or w.D != 32:
+    if w.D != 32:
         return None
     dev = value.device
     offs = offs.to(torch.int32).contiguous()
-    grad = torch.zeros_like(value)
+    grad = torch.zeros(value.shape, dtype=torch.float32, device=dev)
     sink = torch.empty(16 * 256 * torch.cuda.get_device_properties(dev).multi_processor_count,
                        device=dev)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -645,7 +646,36 @@ def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_
     ms = max_over_ranks([e0.elapsed_time(e1) / n], world, device)[0]
     h2d = sum(h_in[k].numel() * h_in[k].element_size() for k in names)
     d2h = sum(h_out[k].numel() * h_out[k].element_size() for k in res_shapes)
+
+    # The copy floor: the same copies with no kernels, one direction at a
+    # time and both at once (the pipelined step cannot beat the latter).
+    def copies(do_in, do_out):
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        c0.record(s_in)
+        s_out.wait_event(c0)
+        for i in range(n):
+            b = bufs[i % nbuf]
+            if do_in:
+                with torch.cuda.stream(s_in):
+                    for k in names:
+                        b["in"][k].copy_(h_in[k], non_blocking=True)
+            if do_out:
+                with torch.cuda.stream(s_out):
+                    for k in res_shapes:
+                        h_out[k].copy_(b["out"][k], non_blocking=True)
+        s_in.wait_stream(s_out)
+        c1.record(s_in)
+        torch.cuda.synchronize()
+        return max_over_ranks([c0.elapsed_time(c1) / n], world, device)[0]
+
+    h2d_ms, d2h_ms, both_ms = copies(True, False), copies(False, True), copies(True, True)
+    floor = {"h2d_ms": h2d_ms, "d2h_ms": d2h_ms, "both_ms": both_ms,
+             "h2d_GB_s": h2d / h2d_ms / 1e6, "d2h_GB_s": d2h / d2h_ms / 1e6,
+             "source": "the step's own pinned copies with no kernels, same streams"}
     return {"value": queries * world / (ms / 1e3), "unit": "queries/s", "ms_per_step": ms,
+            "copy_floor": floor, "frac_of_copy_floor": both_ms / ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
             "pipelining": f"{nbuf} device buffer sets; copy-in, compute and copy-out streams",
             "api": "scale_deformable_attention_02_b200.msda_forward_fused + "

@@ -42,21 +42,25 @@ MSDA_API msda_status msda_debug_sample_points(const int64_t *spatial_shapes,
                                      msda_stream_t stream);
 
 /*
- * The memory-system floor of the path.  Replays a list of 128-byte rows
- * (32 fp32 elements each) in list order, with no index arithmetic:
- *   mode 0  gather every row (what the forward's corner loads do);
+ * The memory-system floor of the path.  Replays a list of 32-element rows
+ * (128 bytes of fp32 or 64 bytes of bf16 value; the gradient is always fp32,
+ * 128 bytes a row) in list order, with no index arithmetic:
+ *   mode 0  gather every value row (what the forward's corner loads do);
  *   mode 1  add a row of ones into grad at every row with one vector
  *           reduction per 16 bytes (what the backward's scatter does);
- *   mode 2  gather every row and add it into grad (the backward's memory
- *           operations).
+ *   mode 2  gather every value row and add it into grad (the backward's
+ *           memory operations).
  * Timing it on the corner rows of a workload gives the floor that the
  * gathers and reductions of the kernels cannot go below on this GPU.
  *
- *   value, grad     device [n_value] fp32, 16-byte aligned (grad unused in
- *                   mode 0, value unused in mode 1; either may then be NULL)
+ *   value           device [n_value] of value_dtype, 16-byte aligned (unused
+ *                   in mode 1; may then be NULL)
+ *   value_dtype     MSDA_F32 or MSDA_BF16
+ *   grad            device [n_value] fp32, 16-byte aligned (unused in mode 0;
+ *                   may then be NULL)
  *   row_offsets     device [n_rows] int32 element offsets; rows that start
- *                   below 0, end past n_value or are not 16-byte aligned are
- *                   skipped
+ *                   below 0, end past n_value, or are not a multiple of 4
+ *                   (fp32) or 8 (bf16) elements are skipped
  *   sink            device [sink_len] fp32, receives per-lane sums of the
  *                   gathered rows so the loads cannot be dropped; may be NULL
  *                   when sink_len is 0
@@ -64,14 +68,15 @@ MSDA_API msda_status msda_debug_sample_points(const int64_t *spatial_shapes,
  *   ctas            thread blocks of 256 threads; <= 0 gives 8 per SM
  * A caller after the floor times a few (depth, ctas) pairs and keeps the
  * fastest.
- * Errors: MSDA_ERR_NULL, MSDA_ERR_SHAPE (mode, depth, n_rows < 0,
- * n_value < 32, sink_len < 0), MSDA_ERR_ALIGN, MSDA_ERR_ALIAS (grad
- * overlapping value, row_offsets or sink).
+ * Errors: MSDA_ERR_NULL, MSDA_ERR_DTYPE, MSDA_ERR_SHAPE (mode, depth,
+ * n_rows < 0, n_value < 32, sink_len < 0), MSDA_ERR_ALIGN, MSDA_ERR_ALIAS
+ * (grad or sink overlapping value, row_offsets or each other).
  */
-MSDA_API msda_status msda_debug_row_traffic(int mode, const float *value, float *grad,
-                                            int64_t n_value, const int32_t *row_offsets,
-                                            int64_t n_rows, float *sink, int64_t sink_len,
-                                            int depth, int ctas, msda_stream_t stream);
+MSDA_API msda_status msda_debug_row_traffic(int mode, const void *value, msda_dtype value_dtype,
+                                            float *grad, int64_t n_value,
+                                            const int32_t *row_offsets, int64_t n_rows,
+                                            float *sink, int64_t sink_len, int depth, int ctas,
+                                            msda_stream_t stream);
 
 #ifdef __cplusplus
 }

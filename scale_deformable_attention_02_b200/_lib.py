@@ -46,7 +46,7 @@ SIGNATURES = {
     "msda_backward_fused_grouped": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, P, P, Dims, I64,
                                           P]),
     "msda_debug_sample_points": (INT, [P, P, P, Dims, P, P, P, P, P, P, P]),
-    "msda_debug_row_traffic": (INT, [INT, P, P, I64, P, I64, P, I64, INT, INT, P]),
+    "msda_debug_row_traffic": (INT, [INT, P, INT, P, I64, P, I64, P, I64, INT, INT, P]),
 }
 
 # Only in libmsda_checked.so (include/msda_checked.h).

@@ -374,23 +374,28 @@ def msda_debug_sample_points(spatial_shapes, level_start_index,
 def msda_debug_row_traffic(mode: int, rows: torch.Tensor, value: torch.Tensor | None = None,
                            grad: torch.Tensor | None = None, sink: torch.Tensor | None = None,
                            depth: int = 0, ctas: int = 0, stream=None) -> None:
-    """Replay 128-byte rows (int32 element offsets `rows`) as bare gathers
-    (mode 0), vector reductions of a row of ones into `grad` (mode 1), or
-    both (mode 2): the memory-system floor of the kernels (include/msda_debug.h)."""
+    """Replay 32-element rows (int32 element offsets `rows`) as bare gathers
+    of fp32 or bf16 `value` (mode 0), vector reductions of a row of ones into
+    the fp32 `grad` (mode 1), or both (mode 2): the memory-system floor of
+    the kernels (include/msda_debug.h)."""
     ref = value if value is not None else grad
     if ref is None:
         raise ValueError("value or grad is required")
     dev = ref.device
     n_value = ref.numel()
-    for t, name in ((value, "value"), (grad, "grad")):
-        if t is not None:
-            _need(t, name, tuple(t.shape), dev)
-            if t.numel() != n_value:
-                raise ValueError("value and grad must have the same number of elements")
+    vdt = _lib.MSDA_F32
+    if value is not None:
+        vdt = _value_dtype(value)
+        _need(value, "value", tuple(value.shape), dev, dtype=value.dtype)
+    if grad is not None:
+        _need(grad, "grad", tuple(grad.shape), dev)
+        if grad.numel() != n_value:
+            raise ValueError("value and grad must have the same number of elements")
     _need(rows, "rows", tuple(rows.shape), dev, dtype=torch.int32)
     if sink is not None:
         _need(sink, "sink", tuple(sink.shape), dev)
     _check(_lib.load().msda_debug_row_traffic(
-        int(mode), _dptr(value), _dptr(grad), n_value, _dptr(rows), rows.numel(), _dptr(sink),
-        0 if sink is None else sink.numel(), int(depth), int(ctas), _stream_handle(dev, stream)),
+        int(mode), _dptr(value), vdt, _dptr(grad), n_value, _dptr(rows), rows.numel(),
+        _dptr(sink), 0 if sink is None else sink.numel(), int(depth), int(ctas),
+        _stream_handle(dev, stream)),
         "msda_debug_row_traffic")

@@ -594,10 +594,12 @@ msda_status msda_debug_sample_points(const int64_t *spatial_shapes,
     return cuda_status(msda::launch_sample_points(p, static_cast<cudaStream_t>(stream)));
 }
 
-msda_status msda_debug_row_traffic(int mode, const float *value, float *grad, int64_t n_value,
-                                   const int32_t *row_offsets, int64_t n_rows, float *sink,
-                                   int64_t sink_len, int depth, int ctas, msda_stream_t stream)
+msda_status msda_debug_row_traffic(int mode, const void *value, msda_dtype value_dtype,
+                                   float *grad, int64_t n_value, const int32_t *row_offsets,
+                                   int64_t n_rows, float *sink, int64_t sink_len, int depth,
+                                   int ctas, msda_stream_t stream)
 {
+    if (value_dtype != MSDA_F32 && value_dtype != MSDA_BF16) return MSDA_ERR_DTYPE;
     if (mode < 0 || mode > 2 || n_rows < 0 || n_value < 32 || sink_len < 0)
         return MSDA_ERR_SHAPE;
     if (depth != 0 && depth != 2 && depth != 4 && depth != 8 && depth != 16)
@@ -610,12 +612,14 @@ msda_status msda_debug_row_traffic(int mode, const float *value, float *grad, in
         !aligned(sink, 4))
         return MSDA_ERR_ALIGN;
     const Span outs[] = {{grad, n_value * 4}, {sink, sink_len * 4}};
-    const Span ins[] = {{value, n_value * 4}, {row_offsets, n_rows * 4}};
+    const int64_t vbytes = value_dtype == MSDA_BF16 ? 2 : 4;
+    const Span ins[] = {{value, n_value * vbytes}, {row_offsets, n_rows * 4}};
     if (any_alias(outs, 2, ins, 2)) return MSDA_ERR_ALIAS;
     if (n_rows == 0) return MSDA_OK;
     msda::TrafficParams p;
     memset(&p, 0, sizeof p);
     p.value = value;
+    p.bf16 = value_dtype == MSDA_BF16;
     p.grad = grad;
     p.rows = row_offsets;
     p.n_rows = n_rows;

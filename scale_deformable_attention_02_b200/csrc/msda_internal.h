@@ -92,14 +92,15 @@ cudaError_t launch_sample_points(const PointsParams &p, cudaStream_t stream);
 
 // Row replay of msda_debug_row_traffic (msda_traffic.cu).
 struct TrafficParams {
-    const float *value;
+    const void *value;    // fp32 or bf16 (bf16 set)
     float *grad;
-    const int32_t *rows;  // element offsets of 128-byte rows
+    const int32_t *rows;  // element offsets of 32-element rows
     int64_t n_rows;
     int64_t n_value;      // elements in value and in grad
     float *sink;          // per-lane sums of the gathered rows (nullable if sink_len == 0)
     int64_t sink_len;
     int64_t per_warp;     // set by the launcher
+    bool bf16;
 };
 cudaError_t launch_row_traffic(TrafficParams p, int mode, int depth, int ctas,
                                cudaStream_t stream);

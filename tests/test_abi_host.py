@@ -297,8 +297,8 @@ def test_grouped_argument_errors(lib):
 def test_row_traffic_argument_errors(lib):
     """msda_debug_row_traffic rejects bad modes, depths, sizes, pointers and
     aliasing before any device work."""
-    def f(mode, value, grad, n_value, rows, n_rows, sink=None, sink_len=0, depth=0):
-        return lib.msda_debug_row_traffic(mode, value, grad, n_value, rows, n_rows, sink,
+    def f(mode, value, grad, n_value, rows, n_rows, sink=None, sink_len=0, depth=0, dt=0):
+        return lib.msda_debug_row_traffic(mode, value, dt, grad, n_value, rows, n_rows, sink,
                                           sink_len, depth, 0, None)
 
     assert f(3, fake(0), fake(1), 64, fake(2), 10) == SHAPE
@@ -312,3 +312,7 @@ def test_row_traffic_argument_errors(lib):
     assert f(2, fake(0), fake(0, 64), 64, fake(2), 10) == ALIAS
     assert f(2, fake(0), fake(1), 64, fake(2), 10, fake(1, 16), 8) == ALIAS
     assert f(2, fake(0), fake(1), 64, fake(2), 0) == OK  # nothing to do
+    assert f(0, fake(0), None, 64, fake(2), 10, dt=2) == DTYPE
+    # a bf16 value map of 64 elements is 128 bytes: a grad 128 bytes on does not overlap it
+    assert f(2, fake(0), fake(0, 128), 64, fake(2), 0, dt=1) == OK
+    assert f(2, fake(0), fake(0, 112), 64, fake(2), 0, dt=1) == ALIAS

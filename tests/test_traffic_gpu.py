@@ -2,7 +2,8 @@
 traffic it claims: every listed row is gathered once (mode 0, checked
 through the sums it leaves in the sink), reduced once (mode 1: grad counts
 the rows' occurrences) or gathered and reduced (mode 2), and rows outside
-the buffers or off the 16-byte grid are skipped."""
+the buffers or off the vector grid (4 elements for fp32 value, 8 for bf16)
+are skipped."""
 import numpy as np
 import pytest
 import torch
@@ -44,5 +45,27 @@ def test_row_traffic_modes():
                                   np.repeat(counts[:, None], 32, axis=1))
     grad.zero_()
     msda_debug_row_traffic(2, trows, value=value, grad=grad)
+    np.testing.assert_allclose(grad.cpu().numpy().reshape(n_map, 32),
+                               counts[:, None] * vr.reshape(n_map, 32), rtol=1e-5, atol=1e-4)
+
+
+def test_row_traffic_bf16_value():
+    """bf16 value rows (64 bytes) gathered, and added into an fp32 gradient
+    (128-byte rows); offsets must sit on the 8-element grid."""
+    n_map = 3000
+    value = torch.randn(n_map * 32, device="cuda").to(torch.bfloat16)
+    rows = _rows(n_map, 100_001, 2)
+    rows[7:9] = [4, 36]  # on the fp32 grid, off the bf16 one: skipped
+    valid = (rows >= 0) & (rows + 32 <= n_map * 32) & (rows % 8 == 0)
+    vr = value.float().cpu().numpy().reshape(-1)
+    trows = torch.from_numpy(rows).cuda()
+    ctas = 16
+    sink = torch.zeros(ctas * 256, device="cuda")
+    msda_debug_row_traffic(0, trows, value=value, sink=sink, ctas=ctas, depth=4)
+    expect = sum(vr[o:o + 32].astype(np.float64).sum() for o in rows[valid])
+    assert abs(float(sink.double().sum()) - expect) <= 1e-3 * (1 + abs(expect))
+    grad = torch.zeros(n_map * 32, device="cuda")
+    msda_debug_row_traffic(2, trows, value=value, grad=grad, ctas=ctas)
+    counts = np.bincount(rows[valid] // 32, minlength=n_map).astype(np.float32)
     np.testing.assert_allclose(grad.cpu().numpy().reshape(n_map, 32),
                                counts[:, None] * vr.reshape(n_map, 32), rtol=1e-5, atol=1e-4)
