@@ -141,6 +141,11 @@ void set_dims(Params *p, const msda_dims &d, int64_t G, const Problem &pr)
     p->K = (int)d.K;
     p->G = (int)G;
     p->Hg = (int)(d.M / G);
+    // item indices N*Lq*M stay below 2^31 (element counts are capped at
+    // 2^31 - 1), so the kernels divide them in 32 bits
+    p->dM = msda::make_fastdiv((unsigned)(d.M > 0 ? d.M : 1));
+    p->dLq = msda::make_fastdiv((unsigned)(d.Lq > 0 ? d.Lq : 1));
+    p->dHg = msda::make_fastdiv((unsigned)(p->Hg > 0 ? p->Hg : 1));
     p->nchunks = pr.nchunks;
     p->lv = pr.lv;
 }

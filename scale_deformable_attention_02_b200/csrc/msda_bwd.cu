@@ -117,9 +117,10 @@ __global__ void __launch_bounds__(kWarps * 32)
 
     const int M = p.M, D = p.D, K = p.K;
     const int LK = p.L * K;
-    const int m = (int)(item % M);
-    const int64_t nq = item / M;
-    const int64_t n = nq / p.Lq;
+    const ItemIdx ix = msda_item_idx(item, p.dM, p.dLq);
+    const int m = ix.m;
+    const int64_t nq = ix.nq;
+    const int64_t n = ix.n;
 
     const int grp = lane / kSpan;
     const int lin = lane % kSpan;
@@ -147,7 +148,7 @@ __global__ void __launch_bounds__(kWarps * 32)
     const VT *vbase = static_cast<const VT *>(p.value) + rowbase;
     float *gvbase = p.grad_value + rowbase;
 
-    const int64_t litem = msda_loc_item(item, M, p.G, p.Hg);
+    const int64_t litem = msda_loc_item(item, p.dM, p.G, p.dHg);
     const bool shared_loc = p.Hg > 1;
 
     float2 bwh = make_float2(0.f, 0.f);       // fused, box reference: (w, h)
@@ -449,7 +450,7 @@ __global__ void __launch_bounds__(kWarps * 32, bwd_min_ctas<VT, R>())
         pl_x = pl_y = pa = 0.f;
         if (jact && item < p.items) {
             const int64_t si = item * LK + j;                               // per head
-            const int64_t sl = msda_loc_item(item, M, p.G, p.Hg) * LK + j;  // per group
+            const int64_t sl = msda_loc_item(item, p.dM, p.G, p.dHg) * LK + j;  // per group
             if constexpr (kFused) {
                 const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sl);
                 pl_x = o.x;
@@ -477,7 +478,7 @@ __global__ void __launch_bounds__(kWarps * 32, bwd_min_ctas<VT, R>())
                 a = seg_softmax<P>(pa, act);
                 lx = ly = 0.f;
                 if (act) {
-                    const float2 loc = msda_fused_location(p.ref, p.ref_dim, item / M, ox, oy, H, W);
+                    const float2 loc = msda_fused_location(p.ref, p.ref_dim, (int64_t)fastdiv(p.dM, (unsigned)item), ox, oy, H, W);
                     lx = loc.x;
                     ly = loc.y;
                 }
@@ -509,11 +510,12 @@ __global__ void __launch_bounds__(kWarps * 32, bwd_min_ctas<VT, R>())
         for (int it = 0; it < kItems; ++it) {
             const int64_t itm = item0 + it;
             if (itm >= p.items) break;  // uniform
-            const int m = (int)(itm % M);
-            const int64_t nq = itm / M;
-            const int64_t n = nq / p.Lq;
+            const ItemIdx ix = msda_item_idx(itm, p.dM, p.dLq);
+            const int m = ix.m;
+            const int64_t nq = ix.nq;
+            const int64_t n = ix.n;
             const int64_t sbase = itm * LK;                                 // per head
-            const int64_t lbase = msda_loc_item(itm, M, p.G, p.Hg) * LK;    // per group
+            const int64_t lbase = msda_loc_item(itm, p.dM, p.G, p.dHg) * LK;    // per group
             const int64_t mapoff = (n * p.S * M + m) * (int64_t)D;
             const int64_t vbe = mapoff + lane_elem;
             const VT *vb = static_cast<const VT *>(p.value) + vbe;
@@ -689,14 +691,15 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_BWD_MIN_CTAS)
 
     for (int64_t item = (int64_t)blockIdx.x * kWarps + warp; item < p.items;
          item += (int64_t)gridDim.x * kWarps) {
-        const int m = (int)(item % M);
-        const int64_t nq = item / M;
-        const int64_t n = nq / p.Lq;
+        const ItemIdx ix = msda_item_idx(item, p.dM, p.dLq);
+        const int m = ix.m;
+        const int64_t nq = ix.nq;
+        const int64_t n = ix.n;
         const int64_t mapoff = (n * p.S * M + m) * (int64_t)D;
         const int64_t vbe = mapoff + lane_elem;
         const VT *vb = static_cast<const VT *>(p.value) + vbe;
         float *gvb = p.grad_value + mapoff + chunk * kVec;
-        const int64_t lbase = msda_loc_item(item, M, p.G, p.Hg) * LK;  // per group
+        const int64_t lbase = msda_loc_item(item, p.dM, p.G, p.dHg) * LK;  // per group
         float gv[kVec];
         if (chunk_ok) {
             const float4 t = __ldcs(reinterpret_cast<const float4 *>(

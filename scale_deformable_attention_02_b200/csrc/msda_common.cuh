@@ -89,12 +89,46 @@ __device__ __forceinline__ bool msda_in_map(unsigned long long *check, int64_t l
 // glossary page, multi-head paragraph), so with G groups of Hg = M/G
 // consecutive heads it is
 // (n*Lq + q)*G + m/Hg.  Hg = 1 (a group per head) gives the item itself.
-__device__ __forceinline__ int64_t msda_loc_item(int64_t item, int M, int G, int Hg)
+__device__ __forceinline__ int64_t msda_loc_item(int64_t item, const FastDiv &dM, int G,
+                                                 const FastDiv &dHg)
 {
-    if (Hg == 1) return item;
-    const int64_t nq = item / M;
-    const int m = (int)(item - nq * M);
-    return nq * G + m / Hg;
+    if (dHg.d == 1) return item;
+    const unsigned u = (unsigned)item;
+    const unsigned nq = fastdiv(dM, u);
+    const unsigned m = u - nq * dM.d;
+    return (int64_t)nq * G + fastdiv(dHg, m);
+}
+
+// Whether head m (of item) is the first of its deformable group, the one that
+// stores the group's shared locations.
+__device__ __forceinline__ bool msda_group_first_m(int m, const FastDiv &dHg)
+{
+    return dHg.d == 1 || (unsigned)m == fastdiv(dHg, (unsigned)m) * dHg.d;
+}
+__device__ __forceinline__ bool msda_group_first(int64_t item, const FastDiv &dM,
+                                                 const FastDiv &dHg)
+{
+    if (dHg.d == 1) return true;
+    const unsigned u = (unsigned)item;
+    return msda_group_first_m((int)(u - fastdiv(dM, u) * dM.d), dHg);
+}
+
+// The (n*Lq + q, m) split of an item index, and n: items are (n, q, m) in
+// storage order, fewer than 2^31.
+struct ItemIdx {
+    int m;
+    int64_t nq, n;
+};
+__device__ __forceinline__ ItemIdx msda_item_idx(int64_t item, const FastDiv &dM,
+                                                 const FastDiv &dLq)
+{
+    const unsigned u = (unsigned)item;
+    const unsigned nq = fastdiv(dM, u);
+    ItemIdx r;
+    r.m = (int)(u - nq * dM.d);
+    r.nq = nq;
+    r.n = fastdiv(dLq, nq);
+    return r;
 }
 
 // Writes the gradient of one shared location: a plain store when every head

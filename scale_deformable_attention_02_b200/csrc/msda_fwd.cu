@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
             const int64_t item = item0 + seg;
             const bool act = j < LK && item < end;
             const int64_t si = item * LK + j;                               // per head
-            const int64_t sl = msda_loc_item(item, M, p.G, p.Hg) * LK + j;  // per group
+            const int64_t sl = msda_loc_item(item, p.dM, p.G, p.dHg) * LK + j;  // per group
             const int l = act ? j / K : 0;
             float lx = 0.f, ly = 0.f, a = 0.f;
             if constexpr (kFused) {
@@ -132,10 +132,10 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
                 if (act) {
                     const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sl);
                     const float2 loc =
-                        msda_fused_location(p.ref, p.ref_dim, item / M, o.x, o.y, sH[l], sW[l]);
+                        msda_fused_location(p.ref, p.ref_dim, (int64_t)fastdiv(p.dM, (unsigned)item), o.x, o.y, sH[l], sW[l]);
                     lx = loc.x;
                     ly = loc.y;
-                    if (p.loc_out && (p.Hg == 1 || (item % M) % p.Hg == 0))  // group's first head
+                    if (p.loc_out && msda_group_first(item, p.dM, p.dHg))  // group's first head
                         __stcs(reinterpret_cast<float2 *>(p.loc_out) + sl, make_float2(lx, ly));
                     if (p.attn_out) __stcs(p.attn_out + si, a);
                 }
@@ -147,8 +147,9 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
             }
             {  // every sample slot up to P gets four entries; unused ones read zeros
                 const int H = sH[l], W = sW[l], start = sStart[l];
-                const int m = (int)(item % M);
-                const int64_t n = item / M / p.Lq;
+                const ItemIdx ix = msda_item_idx(item, p.dM, p.dLq);
+                const int m = ix.m;
+                const int64_t n = ix.n;
                 const char *mapb = static_cast<const char *>(p.value) +
                                    ((n * p.S * M + m) * (int64_t)D) * (int64_t)sizeof(VT);
                 Corner c[4];
@@ -181,8 +182,9 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
         for (int it = 0; it < kItems; ++it) {
             const int64_t item = item0 + it;
             if (item >= end) break;  // uniform across the warp
-            const int m = (int)(item % M);
-            const int64_t nq = item / M;
+            const ItemIdx ix = msda_item_idx(item, p.dM, p.dLq);
+            const int m = ix.m;
+            const int64_t nq = ix.nq;
             // byte offset of this lane's chunk in a row; lanes past the last chunk
             // (D*size not a power-of-two multiple of 16 bytes) re-read chunk 0 and
             // their sums are discarded, so no lane reads past a row
@@ -361,7 +363,7 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
         pa = pb = pc = 0.f;
         if (jact && item < p.items) {
             const int64_t si = item * LK + j;                               // per head
-            const int64_t sl = msda_loc_item(item, M, p.G, p.Hg) * LK + j;  // per group
+            const int64_t sl = msda_loc_item(item, p.dM, p.G, p.dHg) * LK + j;  // per group
             if constexpr (kFused) {
                 pa = __ldcs(p.logits + si);
                 const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + sl);
@@ -388,12 +390,12 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
             a = seg_softmax<P>(pa, act);  // joint over the item's L*K logits
             lx = ly = 0.f;
             if (act) {
-                const float2 loc = msda_fused_location(p.ref, p.ref_dim, item / M, pb, pc, H, W);
+                const float2 loc = msda_fused_location(p.ref, p.ref_dim, (int64_t)fastdiv(p.dM, (unsigned)item), pb, pc, H, W);
                 lx = loc.x;
                 ly = loc.y;
-                if (p.loc_out && (p.Hg == 1 || (item % M) % p.Hg == 0))  // group's first head
+                if (p.loc_out && msda_group_first(item, p.dM, p.dHg))  // group's first head
                     __stcs(reinterpret_cast<float2 *>(p.loc_out) +
-                               msda_loc_item(item, M, p.G, p.Hg) * LK + j,
+                               msda_loc_item(item, p.dM, p.G, p.dHg) * LK + j,
                            make_float2(lx, ly));
                 if (p.attn_out) __stcs(p.attn_out + si, a);
             }
@@ -426,9 +428,10 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
         for (int it = 0; it < kItems; ++it) {
             const int64_t itm = item0 + it;
             if (itm >= p.items) break;  // uniform
-            const int m = (int)(itm % M);
-            const int64_t nq = itm / M;
-            const int64_t n = nq / p.Lq;
+            const ItemIdx ix = msda_item_idx(itm, p.dM, p.dLq);
+            const int m = ix.m;
+            const int64_t nq = ix.nq;
+            const int64_t n = ix.n;
             const int64_t vbe = (n * p.S * M + m) * (int64_t)D + lane_elem;
             const VT *vb = static_cast<const VT *>(p.value) + vbe;
             const int2 *en = ent[warp][it];
@@ -516,13 +519,14 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
 
     for (int64_t item = (int64_t)blockIdx.x * kWarps + warp; item < p.items;
          item += (int64_t)gridDim.x * kWarps) {
-        const int m = (int)(item % M);
-        const int64_t nq = item / M;
-        const int64_t n = nq / p.Lq;
+        const ItemIdx ix = msda_item_idx(item, p.dM, p.dLq);
+        const int m = ix.m;
+        const int64_t nq = ix.nq;
+        const int64_t n = ix.n;
         const int64_t vbe = (n * p.S * M + m) * (int64_t)D + lane_elem;
         const VT *vb = static_cast<const VT *>(p.value) + vbe;
-        const int64_t litem = msda_loc_item(item, M, p.G, p.Hg);
-        const bool first_head = p.Hg == 1 || m % p.Hg == 0;
+        const int64_t litem = msda_loc_item(item, p.dM, p.G, p.dHg);
+        const bool first_head = msda_group_first_m(m, p.dHg);
         float z[kNB];
         float sum = 1.f;
         if constexpr (kFused) {
@@ -685,15 +689,16 @@ __global__ void __launch_bounds__(kWarps * 32, item_min_ctas<VT>())
     const int M = p.M, D = p.D, K = p.K;
     const int LK = p.L * K;
     const int MD = M * D;
-    const int m = (int)(item % M);
-    const int64_t nq = item / M;
-    const int64_t n = nq / p.Lq;
+    const ItemIdx ix = msda_item_idx(item, p.dM, p.dLq);
+    const int m = ix.m;
+    const int64_t nq = ix.nq;
+    const int64_t n = ix.n;
 
     // ---- phase 1: sample `lane` -------------------------------------------
     {
         const bool act = lane < LK;
         const int64_t si = item * LK + lane;                               // per head
-        const int64_t sl = msda_loc_item(item, M, p.G, p.Hg) * LK + lane;  // per group
+        const int64_t sl = msda_loc_item(item, p.dM, p.G, p.dHg) * LK + lane;  // per group
         const int l = act ? lane / K : 0;
         const int H = p.lv.H[l], W = p.lv.W[l], start = p.lv.start[l];
         float lx = 0.f, ly = 0.f, a = 0.f;
@@ -704,7 +709,7 @@ __global__ void __launch_bounds__(kWarps * 32, item_min_ctas<VT>())
                 const float2 loc = msda_fused_location(p.ref, p.ref_dim, nq, o.x, o.y, H, W);
                 lx = loc.x;
                 ly = loc.y;
-                if (p.loc_out && (p.Hg == 1 || m % p.Hg == 0))  // the group's first head
+                if (p.loc_out && (msda_group_first_m(m, p.dHg)))  // the group's first head
                     __stcs(reinterpret_cast<float2 *>(p.loc_out) + sl, make_float2(lx, ly));
                 if (p.attn_out) __stcs(p.attn_out + si, a);
             }

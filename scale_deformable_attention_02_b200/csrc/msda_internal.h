@@ -29,6 +29,7 @@ struct FwdParams {
     int64_t chunk;    // items per CTA (set by the launcher)
     int Lq, S, M, D, L, K;
     int G, Hg;    // deformable groups and heads per group (G = M: one per head)
+    FastDiv dM, dLq, dHg;  // division by M, Lq and Hg
     int nchunks;  // 16-byte chunks per value row
     Levels lv;
     // bounds-checked build only (-DMSDA_CHECKED): value elements an access
@@ -57,6 +58,7 @@ struct BwdParams {
     int64_t chunk;  // items per CTA (set by the launcher)
     int Lq, S, M, D, L, K;
     int G, Hg;  // deformable groups and heads per group (G = M: one per head)
+    FastDiv dM, dLq, dHg;  // division by M, Lq and Hg
     int nchunks;
     Levels lv;
     // bounds-checked build only (-DMSDA_CHECKED): value elements an access
