@@ -418,7 +418,8 @@ __global__ void __launch_bounds__(kWarps * 32, bwd_min_ctas<VT, R>())
     constexpr int kNB = P / kBS;           // batches per item, at most
     __shared__ int2 ent[kWarps][kItems][4 * kStride];  // (row element offset | -1, A*w)
     __shared__ float4 smp[kWarps][kItems][P];          // (fx, fy, A*W, A*H)
-    __shared__ float4 smq[kWarps][kItems][kFused ? P : 1];  // fused: (A, off_x, off_y, -)
+    __shared__ float4 smq[kWarps][kItems][kFused ? P : 1];  // fused: (A, off_x, off_y, dA)
+    __shared__ float2 sdl[kWarps][kItems][kFused ? P : 1];  // fused: d loc per sample
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -537,9 +538,7 @@ __global__ void __launch_bounds__(kWarps * 32, bwd_min_ctas<VT, R>())
                 for (int i = 0; i < kVec; ++i) gv[i] = 0.f;
             }
             const int2 *en = ent[warp][it] + corner * kStride + sg;
-            // fused: chain accumulators of this lane's (writer) samples
-            float rx = 0.f, ry = 0.f, rw = 0.f, rh = 0.f;
-            float2 bwh = make_float2(0.f, 0.f);
+            float2 bwh = make_float2(0.f, 0.f);  // fused box reference: (w, h)
             if constexpr (kFused) {
                 if (p.ref_dim == 4) bwh = __ldg(reinterpret_cast<const float2 *>(p.ref) + 2 * nq + 1);
             }
@@ -608,39 +607,41 @@ __global__ void __launch_bounds__(kWarps * 32, bwd_min_ctas<VT, R>())
                         } else {
                             // loc = c + off * (w, h)
                             goff = make_float2(dlx * bwh.x, dly * bwh.y);
-                            rw = fmaf(dlx, r2.y, rw);
-                            rh = fmaf(dly, r2.z, rh);
                         }
                         if (p.grad_off)
                             msda_put_loc_grad(p.grad_off, lbase + s, goff.x, goff.y, p.Hg > 1);
-                        rx += dlx;
-                        ry += dly;
-                        smq[warp][it][s].w = q0;  // dA, for the softmax Jacobian
+                        smq[warp][it][s].w = q0;                 // dA, for the softmax Jacobian
+                        sdl[warp][it][s] = make_float2(dlx, dly);  // for the reference gradient
                     }
                 }
             }
-            if constexpr (kFused) {
-                // softmax Jacobian: d z_s = A_s (d A_s - sum_j A_j d A_j), lane j = sample j
-                __syncwarp();
-                const float4 ad = lane < LK ? smq[warp][it][lane] : make_float4(0.f, 0.f, 0.f, 0.f);
-                const float dot = warp_sum(ad.x * ad.w);
-                if (lane < LK && p.grad_logits)
-                    __stcs(p.grad_logits + sbase + lane, ad.x * (ad.w - dot));
-                // reference gradient: sum over this head's samples, then over heads
-                rx = warp_sum(rx);
-                ry = warp_sum(ry);
+        }
+        if constexpr (kFused) {
+            // Per item of the round, in the phase-1 layout (lane = seg * P + j
+            // holds sample j of item seg), segment sums over the item's samples:
+            //   softmax Jacobian  d z_j = A_j (dA_j - sum_i A_i dA_i)
+            //   reference point   d ref = sum_j d loc_j (box: also sum_j d loc_j * off_j)
+            __syncwarp();
+            const int64_t item = item0 + seg;
+            const bool act = jact && item < p.items;
+            const float4 ad = act ? smq[warp][seg][j] : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float2 dl = act ? sdl[warp][seg][j] : make_float2(0.f, 0.f);
+            const float dot = seg_sum<P>(ad.x * ad.w);
+            if (act && p.grad_logits) __stcs(p.grad_logits + item * LK + j, ad.x * (ad.w - dot));
+            const float rx = seg_sum<P>(dl.x), ry = seg_sum<P>(dl.y);
+            float rw = 0.f, rh = 0.f;
+            if (p.ref_dim == 4) {
+                rw = seg_sum<P>(dl.x * ad.y);
+                rh = seg_sum<P>(dl.y * ad.z);
+            }
+            // summed over the item's samples here, over its heads by the atomics
+            if (j == 0 && item < p.items && p.grad_ref) {
+                float *gr = p.grad_ref + (int64_t)fastdiv(p.dM, (unsigned)item) * p.ref_dim;
+                atomicAdd(gr, rx);
+                atomicAdd(gr + 1, ry);
                 if (p.ref_dim == 4) {
-                    rw = warp_sum(rw);
-                    rh = warp_sum(rh);
-                }
-                if (lane == 0 && p.grad_ref) {
-                    float *gr = p.grad_ref + nq * p.ref_dim;
-                    atomicAdd(gr, rx);
-                    atomicAdd(gr + 1, ry);
-                    if (p.ref_dim == 4) {
-                        atomicAdd(gr + 2, rw);
-                        atomicAdd(gr + 3, rh);
-                    }
+                    atomicAdd(gr + 2, rw);
+                    atomicAdd(gr + 3, rh);
                 }
             }
         }
