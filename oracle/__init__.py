@@ -189,10 +189,13 @@ def forward_fused(value, shapes, ref, off, logits):
     return forward(value, shapes, loc, a, loc_f32=True), loc, a
 
 
-def backward(value, shapes, loc, attn, grad_out, loc_f32: bool = True, with_mass=False):
+def backward(value, shapes, loc, attn, grad_out, loc_f32: bool = True, with_mass=False,
+             with_grad_value: bool = True):
     """Returns (grad_value [N,S,M,D], grad_loc like loc, grad_attn like attn),
     all float64; with_mass=True appends (grad_loc_mass, grad_attn_mass), the
-    sums of absolute terms that scale a finite-precision rounding bound."""
+    sums of absolute terms that scale a finite-precision rounding bound.
+    with_grad_value=False skips the scatter (grad_value is returned as None),
+    for value maps too large to mirror in fp64."""
     v, bf = _value_arg(value)
     shapes = np.ascontiguousarray(shapes, dtype=np.int64)
     starts, S = level_start_index(shapes)
@@ -201,13 +204,14 @@ def backward(value, shapes, loc, attn, grad_out, loc_f32: bool = True, with_mass
     a64 = np.ascontiguousarray(attn, dtype=np.float64)
     g64 = np.ascontiguousarray(grad_out, dtype=np.float64)
     d = dims_of(v, shapes, loc64.shape)
-    gv = np.empty(v.shape, dtype=np.float64)
+    gv = np.empty(v.shape, dtype=np.float64) if with_grad_value else None
     gl = np.empty(loc64.shape, dtype=np.float64)
     ga = np.empty(a64.shape, dtype=np.float64)
     glm = np.empty(loc64.shape, dtype=np.float64) if with_mass else None
     gam = np.empty(a64.shape, dtype=np.float64) if with_mass else None
     lib().ora_backward(_ptr(v), bf, _ptr(shapes), _ptr(starts), _ptr(loc64),
-                       1 if loc_f32 else 0, _ptr(a64), _ptr(g64), _ptr(gv),
+                       1 if loc_f32 else 0, _ptr(a64), _ptr(g64),
+                       None if gv is None else _ptr(gv),
                        _ptr(gl), _ptr(ga), None if glm is None else _ptr(glm),
                        None if gam is None else _ptr(gam), d)
     if with_mass:

@@ -323,7 +323,9 @@ void ora_locations_f64(const double *ref, const double *off, const int64_t *shap
  *   grad_loc_y[i]      = A_i * H * sum_j dw_j/dfy <v_j, g>
  * (dx/dloc_x = W by R1; dfx/dx = 1 by R6; outside corners have v_j = 0.)
  * grad_value [N,S,M,D] is overwritten.  Serial per (n, m): rows of different
- * (n, m) are disjoint, so the result is deterministic.
+ * (n, m) are disjoint, so the result is deterministic.  grad_value may be
+ * NULL: the per-sample gradients are then formed without the scatter (for
+ * value maps too large to mirror in fp64).
  *
  * grad_loc_mass / grad_attn_mass (may be NULL) receive the absolute mass of
  * each sum, the same expression with every term replaced by its absolute
@@ -338,7 +340,8 @@ void ora_backward(const void *value, int value_bf16, const int64_t *shapes,
                   double *grad_attn_mass, ora_dims d)
 {
     const int64_t N = d.N, Lq = d.Lq, S = d.S, M = d.M, D = d.D, L = d.L, K = d.K;
-    memset(grad_value, 0, sizeof(double) * (size_t)(N * S * M * D));
+    if (grad_value)
+        memset(grad_value, 0, sizeof(double) * (size_t)(N * S * M * D));
 #pragma omp parallel for schedule(static)
     for (int64_t nm = 0; nm < N * M; ++nm) {
         const int64_t n = nm / M, m = nm % M;
@@ -379,7 +382,8 @@ void ora_backward(const void *value, int value_bf16, const int64_t *shapes,
                                 const int64_t e = ((n * S + r) * M + m) * D + c;
                                 vg += value_at(value, value_bf16, e) * g[c];
                                 vg_abs += fabs(value_at(value, value_bf16, e) * g[c]);
-                                grad_value[e] += a * w * g[c];
+                                if (grad_value)
+                                    grad_value[e] += a * w * g[c];
                             }
                             dA += w * vg;
                             dfx += sx * wy * vg;

@@ -253,3 +253,70 @@ def make_random_problem(seed: int, N: int, Lq: int, M: int, D: int, K: int,
     d["logits"] = _normal(rng, (N, Lq, M, L, K))
     d["grad_out"] = _normal(rng, (N, Lq, M * D))
     return d
+
+
+def make_wide_batch_problem(seed: int, N: int, Lq: int, M: int, D: int, K: int,
+                            shapes) -> dict:
+    """A problem with many batch entries that share one value block: every
+    batch entry n reads value[n] = value_block[0], so the full map
+    (N x the block) can be laid out on the device by repetition while a
+    single block stays on the host.  Per-entry locations, reference points,
+    offsets, logits and grad_out are drawn for all N entries (as in
+    make_random_problem).  Used to reach value maps of close to 2^31
+    elements."""
+    rng = np.random.default_rng(seed)
+    L = len(shapes)
+    S = int(sum(h * w for h, w in shapes))
+    return {
+        "spatial_shapes": spatial_shapes_array(shapes),
+        "value_block": rng.uniform(-1.0, 1.0, size=(1, S, M, D)).astype(np.float32),
+        "sampling_locations": rng.uniform(-0.1, 1.1, size=(N, Lq, M, L, K, 2)).astype(np.float32),
+        "reference_points": rng.uniform(0.0, 1.0, size=(N, Lq, 2)).astype(np.float32),
+        "offsets": _normal(rng, (N, Lq, M, L, K, 2), 2.0),
+        "logits": _normal(rng, (N, Lq, M, L, K)),
+        "grad_out": _normal(rng, (N, Lq, M * D)),
+    }
+
+
+def make_windowed_problem(seed: int, shapes, windows, Lq: int, K: int, D: int) -> dict:
+    """One batch entry and one head over levels that may be huge.  Only
+    rectangular pixel windows of level 0 and every pixel of the other levels
+    carry values; every level-0 sample of query q lies inside window
+    q % len(windows), at least one and a half pixels from its edges, so all
+    four corners of its cell fall inside the window.  The samples of the
+    other levels are uniform over those levels.
+
+      windows   ((row0, col0, rows, cols), ...) on level 0, each at least 4x4
+    Returns the window rows as (level-0 pixel row index, values [.., D])
+    pairs plus the locations, logits and grad_out; the caller lays the rows
+    out in a zero map of S rows."""
+    rng = np.random.default_rng(seed)
+    L = len(shapes)
+    H0, W0 = shapes[0]
+    loc = np.empty((1, Lq, 1, L, K, 2), dtype=np.float32)
+    for q in range(Lq):
+        r0, c0, nr, nc = windows[q % len(windows)]
+        # pixel coordinates in [c0 + 1.5, c0 + nc - 2.5]: the cell and its
+        # right/lower neighbour stay inside the window
+        px = rng.uniform(c0 + 1.5, c0 + nc - 2.5, size=K)
+        py = rng.uniform(r0 + 1.5, r0 + nr - 2.5, size=K)
+        loc[0, q, 0, 0, :, 0] = ((px + 0.5) / W0).astype(np.float32)
+        loc[0, q, 0, 0, :, 1] = ((py + 0.5) / H0).astype(np.float32)
+        for lvl in range(1, L):
+            loc[0, q, 0, lvl] = rng.uniform(0.0, 1.0, size=(K, 2)).astype(np.float32)
+    rows, vals = [], []
+    for (r0, c0, nr, nc) in windows:
+        rr, cc = np.meshgrid(np.arange(r0, r0 + nr), np.arange(c0, c0 + nc), indexing="ij")
+        rows.append((rr * W0 + cc).ravel().astype(np.int64))
+        vals.append(rng.uniform(-1.0, 1.0, size=(nr * nc, D)).astype(np.float32))
+    other = int(sum(h * w for h, w in shapes[1:]))
+    return {
+        "spatial_shapes": spatial_shapes_array(shapes),
+        "window_rows": np.concatenate(rows),
+        "window_values": np.concatenate(vals),
+        "other_values": rng.uniform(-1.0, 1.0, size=(other, D)).astype(np.float32),
+        "sampling_locations": loc,
+        "logits": _normal(rng, (1, Lq, 1, L, K)),
+        "grad_out": _normal(rng, (1, Lq, D)),
+        "second_values": rng.uniform(-1.0, 1.0, size=(sum(len(r) for r in rows), D)).astype(np.float32),
+    }

@@ -256,3 +256,17 @@ def test_finite_differences_grouped_locations():
     assert checked >= 40
     # one group per head is the ungrouped problem
     assert np.array_equal(oracle.sum_groups(gl, 4), gl)
+
+
+def test_backward_without_grad_value_keeps_per_sample_gradients():
+    """with_grad_value=False only drops the scatter: the per-sample
+    gradients and their masses are the same numbers."""
+    d = wl.make_random_problem(5, N=2, Lq=7, M=2, D=8, K=3, shapes=((5, 6), (3, 2)))
+    A = oracle.softmax(d["logits"])
+    full = oracle.backward(d["value"], d["spatial_shapes"], d["sampling_locations"], A,
+                           d["grad_out"], with_mass=True)
+    part = oracle.backward(d["value"], d["spatial_shapes"], d["sampling_locations"], A,
+                           d["grad_out"], with_mass=True, with_grad_value=False)
+    assert part[0] is None
+    for a, b in zip(full[1:], part[1:]):
+        np.testing.assert_array_equal(a, b)
