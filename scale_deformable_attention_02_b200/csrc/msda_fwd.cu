@@ -463,20 +463,51 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
                     }
                 }
             }
-#pragma unroll
-            for (int o = R; o < 32; o <<= 1)
+            if constexpr (R * EPL == 32) {
+                // one element per lane: a butterfly reduce-scatter over the
+                // slot lanes of each chunk.  At xor distance o a lane keeps
+                // one half of its values (the upper half if bit o of its lane
+                // is set) and adds the partner's copy of that half, so after
+                // log2(32/R) steps it holds the finished element idx of its
+                // chunk (3 shuffles for 4-element lanes, 7 for 8, against 8
+                // and 24 for a full xor reduction)
+                float v[EPL];
 #pragma unroll
                 for (int i = 0; i < kNP; ++i) {
-                    acc[i].x += __shfl_xor_sync(kFull, acc[i].x, o);
-                    acc[i].y += __shfl_xor_sync(kFull, acc[i].y, o);
+                    v[2 * i] = acc[i].x;
+                    v[2 * i + 1] = acc[i].y;
                 }
-            if (slot == 0 && chunk_ok) {
-                float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D +
-                                                         chunk * EPL);
+                int idx = 0;
 #pragma unroll
-                for (int i = 0; i < kNP / 2; ++i)
-                    __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
-                                                acc[2 * i + 1].y));
+                for (int o = 16, n = EPL; o >= R; o >>= 1, n >>= 1) {
+                    const int half = n / 2;
+                    const bool up = (lane & o) != 0;
+#pragma unroll
+                    for (int i = 0; i < half; ++i) {
+                        const float send = up ? v[i] : v[i + half];
+                        const float keep = up ? v[i + half] : v[i];
+                        v[i] = keep + __shfl_xor_sync(kFull, send, o);
+                    }
+                    if (up) idx += half;
+                }
+                if (chunk_ok)
+                    __stcs(p.out + nq * (int64_t)MD + m * D + chunk * EPL + idx, v[0]);
+            } else {
+#pragma unroll
+                for (int o = R; o < 32; o <<= 1)
+#pragma unroll
+                    for (int i = 0; i < kNP; ++i) {
+                        acc[i].x += __shfl_xor_sync(kFull, acc[i].x, o);
+                        acc[i].y += __shfl_xor_sync(kFull, acc[i].y, o);
+                    }
+                if (slot == 0 && chunk_ok) {
+                    float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D +
+                                                             chunk * EPL);
+#pragma unroll
+                    for (int i = 0; i < kNP / 2; ++i)
+                        __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y,
+                                                    acc[2 * i + 1].x, acc[2 * i + 1].y));
+                }
             }
         }
         __syncwarp();  // the next round overwrites this warp's entries
@@ -887,10 +918,12 @@ cudaError_t launch_fwd_vt(const FwdParams &p, int R, cudaStream_t stream)
     // items of 17..32 samples, rows of at most eight 16-byte lanes
     if (LK >= MSDA_FWD_ITEM_MIN_LK && p.D % E16 == 0 && p.D / E16 <= 8)
         return launch_item_r<VT, E16, kFused>(p, p.D / E16, stream);
-    // fast path: lanes of four elements where a row needs at most eight of
-    // them (bf16: 8-byte loads, 5% faster on the encoder than 16-byte lanes),
-    // else 16-byte lanes
+    // fast path: bf16 rows of 32 elements take four 16-byte lanes (with the
+    // one-element-per-lane reduce-scatter: encoder bf16 forward 174 -> 166 us
+    // against 8-byte lanes); otherwise lanes of four elements where a row
+    // needs at most eight of them, else 16-byte lanes
     if (LK <= MSDA_FWD_FAST_MAX_LK) {
+        if (E16 == 8 && p.D == 32) return launch_fast_lanes<VT, E16, kFused>(p, 4, stream);
         if (p.D % 4 == 0 && p.D / 4 <= 8) return launch_fast_lanes<VT, 4, kFused>(p, p.D / 4, stream);
         if (E16 != 4 && p.D % E16 == 0 && p.D / E16 <= 8)
             return launch_fast_lanes<VT, E16, kFused>(p, p.D / E16, stream);
