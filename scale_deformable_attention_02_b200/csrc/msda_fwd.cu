@@ -318,6 +318,59 @@ struct LaneLoad<__nv_bfloat16, 4> {
 #define MSDA_FWD_PREFETCH 1  // load the next round's inputs during this round's gathers
 #endif
 
+// Sums each chunk's accumulators over the 32/R slot lanes that hold it and
+// stores the item's output row (evict-first).  Where the lanes hold 32
+// elements in all (R * EPL == 32) this is a butterfly reduce-scatter: at xor
+// distance o a lane keeps one half of its values (the upper half if bit o of
+// its lane is set) and adds the partner's copy of that half, so after
+// log2(32/R) steps it holds one finished element, idx, of its chunk, and the
+// warp stores the row with one coalesced instruction (3 shuffles for
+// 4-element lanes, 7 for 8, against 8 and 24 for a full xor reduction).
+// Other widths take the full xor reduction, and the slot-0 lanes store.
+template <int R, int EPL>
+__device__ __forceinline__ void store_row(float2 (&acc)[EPL / 2], int lane, int chunk,
+                                          bool chunk_ok, float *row)
+{
+    constexpr int kNP = EPL / 2;
+    if constexpr (R * EPL == 32) {
+        float v[EPL];
+#pragma unroll
+        for (int i = 0; i < kNP; ++i) {
+            v[2 * i] = acc[i].x;
+            v[2 * i + 1] = acc[i].y;
+        }
+        int idx = 0;
+#pragma unroll
+        for (int o = 16, n = EPL; o >= R; o >>= 1, n >>= 1) {
+            const int half = n / 2;
+            const bool up = (lane & o) != 0;
+#pragma unroll
+            for (int i = 0; i < half; ++i) {
+                const float send = up ? v[i] : v[i + half];
+                const float keep = up ? v[i + half] : v[i];
+                v[i] = keep + __shfl_xor_sync(kFull, send, o);
+            }
+            if (up) idx += half;
+        }
+        if (chunk_ok) __stcs(row + chunk * EPL + idx, v[0]);
+    } else {
+#pragma unroll
+        for (int o = R; o < 32; o <<= 1)
+#pragma unroll
+            for (int i = 0; i < kNP; ++i) {
+                acc[i].x += __shfl_xor_sync(kFull, acc[i].x, o);
+                acc[i].y += __shfl_xor_sync(kFull, acc[i].y, o);
+            }
+        if (lane < R && chunk_ok) {  // slot 0
+            float4 *dst = reinterpret_cast<float4 *>(row + chunk * EPL);
+#pragma unroll
+            for (int i = 0; i < kNP / 2; ++i)
+                __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
+                                            acc[2 * i + 1].y));
+        }
+    }
+}
+
 template <typename VT, int EPL, int R, int P, bool kFused>
 __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
     fwd_kernel(const __grid_constant__ FwdParams p)
@@ -463,52 +516,7 @@ __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)
                     }
                 }
             }
-            if constexpr (R * EPL == 32) {
-                // one element per lane: a butterfly reduce-scatter over the
-                // slot lanes of each chunk.  At xor distance o a lane keeps
-                // one half of its values (the upper half if bit o of its lane
-                // is set) and adds the partner's copy of that half, so after
-                // log2(32/R) steps it holds the finished element idx of its
-                // chunk (3 shuffles for 4-element lanes, 7 for 8, against 8
-                // and 24 for a full xor reduction)
-                float v[EPL];
-#pragma unroll
-                for (int i = 0; i < kNP; ++i) {
-                    v[2 * i] = acc[i].x;
-                    v[2 * i + 1] = acc[i].y;
-                }
-                int idx = 0;
-#pragma unroll
-                for (int o = 16, n = EPL; o >= R; o >>= 1, n >>= 1) {
-                    const int half = n / 2;
-                    const bool up = (lane & o) != 0;
-#pragma unroll
-                    for (int i = 0; i < half; ++i) {
-                        const float send = up ? v[i] : v[i + half];
-                        const float keep = up ? v[i + half] : v[i];
-                        v[i] = keep + __shfl_xor_sync(kFull, send, o);
-                    }
-                    if (up) idx += half;
-                }
-                if (chunk_ok)
-                    __stcs(p.out + nq * (int64_t)MD + m * D + chunk * EPL + idx, v[0]);
-            } else {
-#pragma unroll
-                for (int o = R; o < 32; o <<= 1)
-#pragma unroll
-                    for (int i = 0; i < kNP; ++i) {
-                        acc[i].x += __shfl_xor_sync(kFull, acc[i].x, o);
-                        acc[i].y += __shfl_xor_sync(kFull, acc[i].y, o);
-                    }
-                if (slot == 0 && chunk_ok) {
-                    float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D +
-                                                             chunk * EPL);
-#pragma unroll
-                    for (int i = 0; i < kNP / 2; ++i)
-                        __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y,
-                                                    acc[2 * i + 1].x, acc[2 * i + 1].y));
-                }
-            }
+            store_row<R, EPL>(acc, lane, chunk, chunk_ok, p.out + nq * (int64_t)MD + m * D);
         }
         __syncwarp();  // the next round overwrites this warp's entries
     }
@@ -805,20 +813,7 @@ __global__ void __launch_bounds__(kWarps * 32, item_min_ctas<VT>())
             }
         }
     }
-#pragma unroll
-    for (int o = R; o < 32; o <<= 1)
-#pragma unroll
-        for (int i = 0; i < kNP; ++i) {
-            acc[i].x += __shfl_xor_sync(kFull, acc[i].x, o);
-            acc[i].y += __shfl_xor_sync(kFull, acc[i].y, o);
-        }
-    if (slot == 0 && chunk_ok) {
-        float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D + chunk * EPL);
-#pragma unroll
-        for (int i = 0; i < kNP / 2; ++i)
-            __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
-                                        acc[2 * i + 1].y));
-    }
+    store_row<R, EPL>(acc, lane, chunk, chunk_ok, p.out + nq * (int64_t)MD + m * D);
 }
 
 template <typename VT, int EPL, int R, bool kFused>
