@@ -48,3 +48,21 @@ def test_touched_rows_replace_the_full_map():
     part = bench.algorithmic_bytes(w, "split", touched_rows=1000)
     rows = w.N * w.S * w.M
     assert full["fwd"] - part["fwd"] == (rows - 1000) * w.D * 4
+
+
+def test_kernel_source_hash_ignores_comments_only(tmp_path, monkeypatch):
+    """The recorded DRAM traffic is keyed by a hash of the kernels' device
+    code: a comment edit keeps it, a code edit changes it."""
+    import os
+    import shutil
+    src = os.path.join(bench.ROOT, "scale_deformable_attention_02_b200", "csrc")
+    dst = tmp_path / "scale_deformable_attention_02_b200" / "csrc"
+    shutil.copytree(src, dst)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    base = bench.kernel_source_hash()
+    f = dst / "msda_bwd.cu"
+    text = f.read_text()
+    f.write_text(text.replace("namespace msda {", "// a remark\nnamespace msda { /* another */", 1))
+    assert bench.kernel_source_hash() == base
+    f.write_text(text.replace("constexpr int kWarps = 8;", "constexpr int kWarps = 4;", 1))
+    assert bench.kernel_source_hash() != base
