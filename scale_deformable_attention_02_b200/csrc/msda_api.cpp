@@ -110,6 +110,8 @@ msda_status check_dims(msda_dtype dt, const int64_t *shapes, const int64_t *star
     if (!mul_le(d.N, smd, kGuard, &pr->n_value)) return MSDA_ERR_UNSUPPORTED;
     if (!mul_le(d.N, d.Lq, kGuard, &t) || !mul_le(t, d.M, kGuard, &pr->items))
         return MSDA_ERR_UNSUPPORTED;
+    // the kernels split item indices (n, q, m) in 32 bits
+    if (pr->items > kI32Max) return MSDA_ERR_UNSUPPORTED;
     if (!mul_le(pr->items, d.L * d.K * 2, kGuard, &t)) return MSDA_ERR_UNSUPPORTED;
     pr->samples = pr->items * d.L * d.K;
     pr->n_out = pr->items * d.D;
@@ -141,8 +143,8 @@ void set_dims(Params *p, const msda_dims &d, int64_t G, const Problem &pr)
     p->K = (int)d.K;
     p->G = (int)G;
     p->Hg = (int)(d.M / G);
-    // item indices N*Lq*M stay below 2^31 (element counts are capped at
-    // 2^31 - 1), so the kernels divide them in 32 bits
+    // item indices N*Lq*M stay below 2^31 (check_dims), so the kernels
+    // divide them in 32 bits
     p->dM = msda::make_fastdiv((unsigned)(d.M > 0 ? d.M : 1));
     p->dLq = msda::make_fastdiv((unsigned)(d.Lq > 0 ? d.Lq : 1));
     p->dHg = msda::make_fastdiv((unsigned)(p->Hg > 0 ? p->Hg : 1));
@@ -362,6 +364,20 @@ msda_status backward_impl(const void *value, msda_dtype value_dtype,
                         {grad_out, pr.n_out * 4}};
     if (any_alias(outs, 3, ins, 4)) return MSDA_ERR_ALIAS;
 
+    msda::BwdParams p;
+    memset(&p, 0, sizeof p);
+    p.value = value;
+    p.loc = sampling_locations;
+    p.attn = attention_weights;
+    p.grad_out = grad_out;
+    p.grad_value = grad_value;
+    p.grad_loc = grad_sampling_locations;
+    p.grad_attn = grad_attention_weights;
+    set_dims(&p, d, G, pr);
+    // before any device work, so that a failure here has launched nothing
+    // (a problem with no queries launches no kernel and needs no checks)
+    if (pr.n_out > 0 && (st = set_checks(&p, pr)) != MSDA_OK) return st;
+
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (pr.n_value > 0) {
         st = cuda_status(cudaMemsetAsync(grad_value, 0, (size_t)pr.n_value * 4, s));
@@ -373,18 +389,6 @@ msda_status backward_impl(const void *value, msda_dtype value_dtype,
         if (st != MSDA_OK) return st;
     }
     if (pr.n_out == 0) return MSDA_OK;
-
-    msda::BwdParams p;
-    memset(&p, 0, sizeof p);
-    p.value = value;
-    p.loc = sampling_locations;
-    p.attn = attention_weights;
-    p.grad_out = grad_out;
-    p.grad_value = grad_value;
-    p.grad_loc = grad_sampling_locations;
-    p.grad_attn = grad_attention_weights;
-    set_dims(&p, d, G, pr);
-    if ((st = set_checks(&p, pr)) != MSDA_OK) return st;
     return launched(msda::launch_backward(p, value_dtype == MSDA_BF16, pr.lanes, s), s);
 }
 
@@ -422,6 +426,23 @@ msda_status backward_fused_impl(const void *value, msda_dtype value_dtype,
                         {grad_out, pr.n_out * 4}};
     if (any_alias(outs, 4, ins, 5)) return MSDA_ERR_ALIAS;
 
+    msda::BwdParams p;
+    memset(&p, 0, sizeof p);
+    p.value = value;
+    p.ref = reference_points;
+    p.ref_dim = reference_dim;
+    p.off = offsets;
+    p.logits = logits;
+    p.grad_out = grad_out;
+    p.grad_value = grad_value;
+    p.grad_ref = grad_reference_points;
+    p.grad_off = grad_offsets;
+    p.grad_logits = grad_logits;
+    set_dims(&p, d, G, pr);
+    // before any device work, so that a failure here has launched nothing
+    // (a problem with no queries launches no kernel and needs no checks)
+    if (pr.n_out > 0 && (st = set_checks(&p, pr)) != MSDA_OK) return st;
+
     const cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (pr.n_value > 0) {
         st = cuda_status(cudaMemsetAsync(grad_value, 0, (size_t)pr.n_value * 4, s));
@@ -437,21 +458,6 @@ msda_status backward_fused_impl(const void *value, msda_dtype value_dtype,
         if (st != MSDA_OK) return st;
     }
     if (pr.n_out == 0) return MSDA_OK;
-
-    msda::BwdParams p;
-    memset(&p, 0, sizeof p);
-    p.value = value;
-    p.ref = reference_points;
-    p.ref_dim = reference_dim;
-    p.off = offsets;
-    p.logits = logits;
-    p.grad_out = grad_out;
-    p.grad_value = grad_value;
-    p.grad_ref = grad_reference_points;
-    p.grad_off = grad_offsets;
-    p.grad_logits = grad_logits;
-    set_dims(&p, d, G, pr);
-    if ((st = set_checks(&p, pr)) != MSDA_OK) return st;
     return launched(msda::launch_backward_fused(p, value_dtype == MSDA_BF16, pr.lanes, s), s);
 }
 

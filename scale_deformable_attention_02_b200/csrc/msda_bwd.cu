@@ -13,7 +13,7 @@
 //   * bwd_kernel (value rows of at most 128 bytes): a group of R lanes owns
 //     whole samples and sums their four corners inside each lane, so only
 //     the R chunk lanes need combining (see its comment).  Persistent CTAs
-//     sweep contiguous item ranges.
+//     whose warps take rounds of items grid-stride.
 //   * bwd_kernel_wide (rows wider than 128 bytes): one warp per item; lane j
 //     finds sample j's cell and stores per-corner (row offset, w, dw/dfx,
 //     dw/dfy) in shared memory; min(32, 4R) lanes work on one sample, and the

@@ -4,8 +4,6 @@
 // the default build.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "msda_internal.h"
 
 namespace msda {
@@ -18,17 +16,12 @@ __device__ __align__(16) unsigned long long g_check_word[2];
 
 unsigned long long *check_word()
 {
-    static std::mutex mu;
-    static unsigned long long *cache[64] = {};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!cache[dev]) {
-        void *ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_check_word) != cudaSuccess) return nullptr;
-        cache[dev] = static_cast<unsigned long long *>(ptr);
-    }
-    return cache[dev];
+    // Looked up on every call (this build is for checking, not timing): the
+    // address stays valid for the current device's context, including a
+    // context created again after cudaDeviceReset.
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_check_word) != cudaSuccess) return nullptr;
+    return static_cast<unsigned long long *>(ptr);
 }
 #endif
 

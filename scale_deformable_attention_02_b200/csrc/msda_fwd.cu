@@ -8,17 +8,24 @@
 // D elements.  A (pixel, head) row is split into 16-byte chunks and R lanes
 // cover one row, so a warp instruction gathers 32/R whole rows with 16 bytes
 // per lane (fp32, D = 32: R = 8; bf16, D = 32: R = 4); lanes accumulate their
-// chunk in fp32 with packed FMA (`__ffma2_rn`).  Two kernels:
-//   * fwd_kernel (rows of at most 128 bytes): a group of R lanes owns whole
-//     samples; every lane forms its corner addresses and weights in registers
-//     (see its comment).
-//   * fwd_kernel_wide (wider rows): lane j of an item's P-lane segment forms
-//     sample j's cell and writes four (row address, weight) entries to shared
-//     memory; the warp then walks the (sample, corner) pairs.
-// Both run persistent CTAs that sweep contiguous item ranges (neighbouring
-// queries sample neighbouring pixels, so rows are reused from L1), issue a
-// batch of gathers before consuming any, and send corners outside the level
-// to a zero row instead of branching.
+// chunk in fp32 with packed FMA (`__ffma2_rn`).  Four kernels:
+//   * fwd_kernel (rows of at most eight lanes, at most 32 samples per item;
+//     items of 17..32 samples over 16-byte lanes go to fwd_kernel_item):
+//     persistent CTAs whose warps take rounds of 32/P items grid-stride
+//     (round r of CTA b starts at item (r * gridDim.x + b) * 8 * 32/P).
+//     Lane j of an item's P-lane segment forms sample j's weight, location
+//     and cell and writes four 8-byte (row offset, weight) corner entries to
+//     shared memory; the warp then gathers the entries' rows, several
+//     instructions in flight, and reduces the slot sums with a
+//     reduce-scatter (see its comment).
+//   * fwd_kernel_item (17..32 samples per item): one warp per item, a plain
+//     grid over the items, the same entries and reduction.
+//   * fwd_kernel_long (more than 32 samples): one warp per item and round,
+//     samples taken in blocks of 32.
+//   * fwd_kernel_wide (rows wider than eight lanes): each CTA sweeps one
+//     contiguous item range with the same entries.
+// A corner outside the level has no entry (row -1 or a zero row) and adds
+// nothing.
 // Single-use data (locations, weights, logits, offsets, outputs) is read and
 // written with evict-first hints so that the value map, which every sample
 // gathers from, keeps the L2.  The gather is the whole cost ("Deformable

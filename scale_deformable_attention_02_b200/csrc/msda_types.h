@@ -28,8 +28,8 @@ struct Levels {
 //   m' = floor(2^32 (2^l - d) / d) + 1, which fits in 32 bits
 //   t  = floor(m' n / 2^32)
 //   n / d = (t + ((n - t) >> min(l, 1))) >> max(l - 1, 0)   for every n < 2^32.
-// The kernels index items (n, q, m) of at most 2^31 - 1 entries, so 32 bits
-// hold every dividend.
+// The host rejects problems of 2^31 or more items (n, q, m), so 32 bits hold
+// every dividend.
 struct FastDiv {
     unsigned d;   // the divisor
     unsigned m;   // m'

@@ -190,6 +190,11 @@ def test_forward_argument_errors(lib):
     # int32 row offsets: S*M*D must stay below 2^31
     huge = Prob(M=8, D=32, shapes=((4096, 2049),))
     assert fwd(lib, huge) == UNSUP
+    # 32-bit item indices: N*Lq*M must stay below 2^31 (here exactly 2^31)
+    many = Prob(N=2, Lq=1 << 29, M=2)
+    assert fwd(lib, many) == UNSUP
+    assert lib.msda_backward(fake(0), 0, many.sp(), many.st(), fake(1), fake(2), fake(3),
+                             fake(4), None, None, many.dims, None) == UNSUP
 
 
 def test_empty_problems_are_no_ops(lib):

@@ -22,7 +22,7 @@ from scale_deformable_attention_02_b200 import (MsdaError, checked_library, last
                                                 msda_forward, msda_forward_fused)
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import F32, GRAD, assert_close, host, to_dev
+from gpu_util import F32, GRAD, PLAIN, assert_close, host, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -110,8 +110,8 @@ def test_checked_build_default_bound_matches_oracle(case):
     assert_close(host(outs["out"]), out, **F32, what="checked forward")
     assert_close(host(outs["fout"]), fo, **F32, what="checked fused forward")
     assert_close(host(outs["gv"]), ogv, **GRAD, what="checked grad_value")
-    assert_close(host(outs["gl"]), ogl, **GRAD, what="checked grad_loc", mass=mgl)
-    assert_close(host(outs["ga"]), oga, **GRAD, what="checked grad_attn", mass=mga)
+    assert_close(host(outs["gl"]), ogl, **PLAIN, what="checked grad_loc", mass=mgl)
+    assert_close(host(outs["ga"]), oga, **PLAIN, what="checked grad_attn", mass=mga)
 
 
 def _zero_beyond(value: np.ndarray, limit: int) -> np.ndarray:
@@ -165,8 +165,8 @@ def test_checked_build_skips_and_reports_beyond_lowered_bound(case):
     assert not gv.reshape(-1)[limit:].any(), "a scatter beyond the bound was made"
     assert_close(gv.reshape(-1)[:limit], ogv.reshape(-1)[:limit], **GRAD,
                  what="grad_value below the bound")
-    assert_close(host(outs["gl"]), ogl, **GRAD, what="grad_loc, lowered bound", mass=mgl)
-    assert_close(host(outs["ga"]), oga, **GRAD, what="grad_attn, lowered bound", mass=mga)
+    assert_close(host(outs["gl"]), ogl, **PLAIN, what="grad_loc, lowered bound", mass=mgl)
+    assert_close(host(outs["ga"]), oga, **PLAIN, what="grad_attn, lowered bound", mass=mga)
     # the word was cleared: the next call with the default bound is clean, and
     # the thread's last report is still the backward's
     with checked_library():

@@ -13,7 +13,8 @@ from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fus
                                                 msda_forward, msda_forward_fused)
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import F32, GRAD, KAPPA, U32, assert_bits_equal, assert_close, host, to_dev
+from gpu_util import (F32, GRAD, KAPPA, PLAIN, U32, assert_bits_equal, assert_close, grad_tol,
+                      host, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -62,9 +63,9 @@ def test_grouped_forward_and_backward(case):
     ogv, ogl, oga, mgl, mga = oracle.backward(d["value"], sh, loc_h, A, d["grad_out"],
                                               with_mass=True)
     assert_close(host(gv), ogv, **GRAD, what="grouped grad_value")
-    assert_close(host(ga), oga, **GRAD, what="grouped grad_attn", mass=mga)
+    assert_close(host(ga), oga, **PLAIN, what="grouped grad_attn", mass=mga)
     # a group's location gradient adds its heads' gradients (atomically, any order)
-    assert_close(host(gl), oracle.sum_groups(ogl, G), **GRAD, what="grouped grad_loc",
+    assert_close(host(gl), oracle.sum_groups(ogl, G), **grad_tol(G, M), what="grouped grad_loc",
                  mass=oracle.sum_groups(mgl + np.abs(ogl), G))
 
 
@@ -100,9 +101,9 @@ def test_grouped_fused_forward_and_backward(case):
     mz = (Af * (mga.reshape(Af.shape) + mz_head)).reshape(A.shape)
     mref = (mgl + np.abs(ogl)).sum(axis=(2, 3, 4))
     assert_close(host(gv), ogv, **GRAD, what="grouped fused grad_value")
-    assert_close(host(go), oracle.sum_groups(ogo, G), **GRAD, what="grouped grad_offsets",
-                 mass=oracle.sum_groups(mgo, G))
-    assert_close(host(gz), ogz, **GRAD, what="grouped grad_logits", mass=mz)
+    assert_close(host(go), oracle.sum_groups(ogo, G), **grad_tol(G, M),
+                 what="grouped grad_offsets", mass=oracle.sum_groups(mgo, G))
+    assert_close(host(gz), ogz, **PLAIN, what="grouped grad_logits", mass=mz)
     assert_close(host(gr), ogr, **GRAD, what="grouped grad_reference", mass=mref)
 
 

@@ -28,7 +28,7 @@ from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fus
                                                 msda_forward, msda_forward_fused)
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import F32, GRAD, KAPPA, U32, assert_bits_equal, assert_close, host, to_dev
+from gpu_util import F32, GRAD, KAPPA, PLAIN, U32, assert_bits_equal, assert_close, host, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -78,8 +78,8 @@ def test_wide_batch_at_the_element_limit():
         ogv, ogl, oga, mgl, mga = oracle.backward(block, sh, loc[sl], A[sl], g[sl],
                                                   with_mass=True)
         assert_close(host(gv[sl]), ogv, **GRAD, what=f"{what} grad_value")
-        assert_close(host(gl[sl]), ogl, **GRAD, what=f"{what} grad_loc", mass=mgl)
-        assert_close(host(ga[sl]), oga, **GRAD, what=f"{what} grad_attn", mass=mga)
+        assert_close(host(gl[sl]), ogl, **PLAIN, what=f"{what} grad_loc", mass=mgl)
+        assert_close(host(ga[sl]), oga, **PLAIN, what=f"{what} grad_attn", mass=mga)
         # fused backward: the oracle's backward at its own locations and
         # weights, then its chain rule (bounds as in the fused-backward tests)
         oA64 = oracle.softmax(d["logits"][sl])
@@ -94,8 +94,8 @@ def test_wide_batch_at_the_element_limit():
         mz_head = (Af * (fmga.reshape(Af.shape) + np.abs(fga_o.reshape(Af.shape)))).sum(-1, keepdims=True)
         mz = (Af * (fmga.reshape(Af.shape) + mz_head)).reshape(oA64.shape)
         assert_close(host(fgv[sl]), fgv_o, **GRAD, what=f"{what} fused grad_value")
-        assert_close(host(fgo[sl]), ogo, **GRAD, what=f"{what} grad_offsets", mass=mgo)
-        assert_close(host(fgz[sl]), ogz, **GRAD, what=f"{what} grad_logits", mass=mz)
+        assert_close(host(fgo[sl]), ogo, **PLAIN, what=f"{what} grad_offsets", mass=mgo)
+        assert_close(host(fgz[sl]), ogz, **PLAIN, what=f"{what} grad_logits", mass=mz)
         assert_close(host(fgr[sl]), ogr, **GRAD, what=f"{what} grad_reference", mass=mref)
 
 
@@ -129,8 +129,8 @@ def test_huge_level_at_the_element_limit():
     gv, gl, ga = msda_backward(value, sh, None, to_dev(loc), to_dev(A), to_dev(g))
     _, ogl, oga, mgl, mga = oracle.backward(value_h, sh, loc, A, g, with_mass=True,
                                             with_grad_value=False)
-    assert_close(host(gl), ogl, **GRAD, what="grad_loc", mass=mgl)
-    assert_close(host(ga), oga, **GRAD, what="grad_attn", mass=mga)
+    assert_close(host(gl), ogl, **PLAIN, what="grad_loc", mass=mgl)
+    assert_close(host(ga), oga, **PLAIN, what="grad_attn", mass=mga)
     del value
     # grad_value: zero outside the windows and the small level ...
     held = torch.from_numpy(np.concatenate([rows, np.arange(start1, S)])).to("cuda")

@@ -2,8 +2,11 @@
 points, the pixel offsets and the logits) against the oracle's backward
 followed by its chain rule (pinned by finite differences on the CPU).
 
-Bounds: GRAD (1e-4 relative, 1e-5 absolute) plus the fp32 rounding bound of
-each chained quantity, built from the oracle's absolute masses:
+Bounds: PLAIN (1e-5 relative, 1e-6 absolute) for the offsets and logits,
+which the kernel writes once per sample; GRAD (1e-4 relative, 1e-5 absolute)
+for grad_value and the reference points, which are summed with atomics; each
+plus the fp32 rounding bound of the chained quantity, built from the oracle's
+absolute masses:
   offsets   point: mass(d loc) / W_l     box: mass(d loc) * (w, h)
   logits    A_s (m_s + sum_j A_j m_j + sum_j A_j |dA_j|)  with m = mass(dA)
   reference sum over the query's samples of mass(d loc) (+ |d loc|, for the
@@ -16,7 +19,7 @@ import oracle
 from scale_deformable_attention_02_b200 import msda_backward_fused, msda_forward_fused
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import GRAD, KAPPA, U32, assert_close, host, to_dev
+from gpu_util import GRAD, KAPPA, PLAIN, U32, assert_close, host, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -55,8 +58,8 @@ def _check(d, ref, off, logits, box: bool):
     mz_head = (Af * (mga.reshape(Af.shape) + np.abs(oga.reshape(Af.shape)))).sum(-1, keepdims=True)
     mz = (Af * (mga.reshape(Af.shape) + mz_head)).reshape(A.shape)
     assert_close(host(gv), ogv, **GRAD, what="grad_value")
-    assert_close(host(go), ogo, **GRAD, what="grad_offsets", mass=mgo)
-    assert_close(host(gz), ogz, **GRAD, what="grad_logits", mass=mz)
+    assert_close(host(go), ogo, **PLAIN, what="grad_offsets", mass=mgo)
+    assert_close(host(gz), ogz, **PLAIN, what="grad_logits", mass=mz)
     assert_close(host(gr), ogr, **GRAD, what="grad_reference", mass=mref)
 
 

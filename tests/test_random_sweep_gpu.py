@@ -13,7 +13,8 @@ from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fus
                                                 msda_forward, msda_forward_fused)
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import F32, GRAD, KAPPA, U32, assert_bits_equal, assert_close, host, to_dev
+from gpu_util import (F32, GRAD, KAPPA, PLAIN, U32, assert_bits_equal, assert_close, grad_tol,
+                      host, to_dev)
 
 pytestmark = pytest.mark.gpu
 
@@ -72,8 +73,8 @@ def test_random_shape(c):
     ogv, ogl, oga, mgl, mga = oracle.backward(d["value"], sh, loc_h, A, d["grad_out"],
                                               with_mass=True)
     assert_close(host(gv), ogv, **GRAD, what="grad_value")
-    assert_close(host(ga), oga, **GRAD, what="grad_attn", mass=mga)
-    assert_close(host(gl), oracle.sum_groups(ogl, G), **GRAD, what="grad_loc",
+    assert_close(host(ga), oga, **PLAIN, what="grad_attn", mass=mga)
+    assert_close(host(gl), oracle.sum_groups(ogl, G), **grad_tol(G, M), what="grad_loc",
                  mass=oracle.sum_groups(mgl + np.abs(ogl), G))
     # fused: point or box references, per-group offsets
     if c["box"]:
@@ -125,7 +126,7 @@ def test_random_shape(c):
                                                                                 keepdims=True)
     mz = (Af * (mga.reshape(Af.shape) + mz_head)).reshape(A64.shape)
     assert_close(host(gv), ogv, **GRAD, what="fused grad_value")
-    assert_close(host(go), oracle.sum_groups(ogo, G), **GRAD, what="fused grad_offsets",
-                 mass=oracle.sum_groups(mgo, G))
-    assert_close(host(gz), ogz, **GRAD, what="fused grad_logits", mass=mz)
+    assert_close(host(go), oracle.sum_groups(ogo, G), **grad_tol(G, M),
+                 what="fused grad_offsets", mass=oracle.sum_groups(mgo, G))
+    assert_close(host(gz), ogz, **PLAIN, what="fused grad_logits", mass=mz)
     assert_close(host(gr), ogr, **GRAD, what="fused grad_reference", mass=mref)
