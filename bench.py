@@ -73,6 +73,17 @@ def parse_args(argv=None):
                     help="capture the forward and the backward as two CUDA graphs and time "
                          "their replays (the launch-latency path for small problems such "
                          "as the decoder)")
+    ap.add_argument("--schedule", choices=["tiled", "untiled"], default=None,
+                    help="tiled: tile plan + msda_tiled.h calls (default, except the decoder); "
+                         "untiled: the msda.h calls")
+    ap.add_argument("--halo", type=int, default=None,
+                    help="window halo of the tiled schedule, pixels (default per workload)")
+    ap.add_argument("--ctas-per-sm", type=int, default=None,
+                    help="resident CTAs the tiled windows are sized for (default per workload)")
+    ap.add_argument("--also", default="encoder_bf16,stress",
+                    help="comma-separated workloads timed briefly after the main one and "
+                         "reported under 'also' (rank 0, one GPU); empty for none")
+    ap.add_argument("--also-steps", type=int, default=5)
     ap.add_argument("--step", choices=["split", "fused"], default="split",
                     help="split: fused forward writing locations and weights, then "
                          "msda_backward (grad value, locations, weights); fused: fused "
@@ -133,10 +144,10 @@ def algorithmic_bytes(w: wl.Workload, step: str = "split", touched_rows=None) ->
 
 
 def kernel_source_hash() -> str:
-    """sha256 of the forward and backward kernels' device code: msda_fwd.cu,
-    msda_bwd.cu, msda_common.cuh, msda_types.h and the FwdParams / BwdParams
-    structs, with comments and blank space removed, so that a counter taken on
-    those kernels stays valid across edits that do not touch them."""
+    """sha256 of the forward and backward kernels' device code: the kernel
+    sources and device headers and the launch-parameter structs, with comments
+    and blank space removed, so that a counter taken on those kernels stays
+    valid across edits that do not touch them."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "scale_deformable_attention_02_b200", "csrc")
 
@@ -145,12 +156,14 @@ def kernel_source_hash() -> str:
         text = re.sub(r"//[^\n]*", " ", text)
         return " ".join(text.split())
 
-    for f in ("msda_fwd.cu", "msda_bwd.cu", "msda_common.cuh", "msda_types.h"):
+    for f in ("msda_fwd.cu", "msda_bwd.cu", "msda_fwd_tiled.cu", "msda_bwd_tiled.cu",
+              "msda_tile_plan.cu", "msda_common.cuh", "msda_rows.cuh", "msda_tile.cuh",
+              "msda_tma.cuh", "msda_types.h"):
         with open(os.path.join(csrc, f), encoding="utf-8") as fh:
             h.update(f.encode() + b"\0" + norm(fh.read()).encode())
     with open(os.path.join(csrc, "msda_internal.h"), encoding="utf-8") as fh:
         internal = norm(fh.read())
-    for name in ("FwdParams", "BwdParams"):
+    for name in ("FwdParams", "BwdParams", "TileView", "FwdTiledParams", "BwdTiledParams"):
         m = re.search(r"struct " + name + r" \{.*?\};", internal)
         h.update(name.encode() + b"\0" + (m.group(0) if m else "").encode())
     return h.hexdigest()
@@ -255,12 +268,175 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------
+# Window halo of the tiled schedule per workload: about twice the standard
+# deviation of the workload's offsets (the window-hit replay in the design doc), at
+# least 3 pixels; the compass offsets reach K = 4 pixels.
+TILE_HALO = {"encoder": 3, "encoder_bf16": 3, "encoder_compass": 4, "stress": 8, "decoder": 4,
+             "tiny": 1}
+# Resident CTAs per SM the tiled windows are sized for.
+TILE_CTAS = {"stress": 1}
+# Workloads whose default schedule is untiled: the decoder's 300 queries per
+# image are spread over the whole map, so cells would hold one or two queries.
+UNTILED_DEFAULT = {"decoder", "tiny"}
+
+
+class Steps:
+    """Device tensors of one workload and its forward and backward calls.
+    `schedule` tiled: the step rebuilds the tile plan from the reference
+    points (msda_tile_plan_build), then runs the tiled forward and backward;
+    untiled: the msda.h calls.  `step` split: the fused forward writes the
+    locations and weights, msda_backward reads them; fused: the forward
+    writes only out, msda_backward_fused recomputes them."""
+
+    def __init__(self, torch, device, w, inp, step, schedule, halo=None, ctas=None):
+        import scale_deformable_attention_02_b200 as m
+        self.m, self.w, self.step, self.schedule = m, w, step, schedule
+        self.sh = inp["spatial_shapes"]
+        self.starts, _ = m.msda_level_start_index(self.sh)
+
+        def dev_tensor(a):
+            a = np.ascontiguousarray(a)
+            if a.dtype == np.uint16:
+                return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+            return torch.from_numpy(a).to(device)
+
+        self.value = dev_tensor(inp["value"])
+        self.ref = dev_tensor(inp["reference_points"])
+        self.off = dev_tensor(inp["offsets"])
+        self.logits = dev_tensor(inp["logits"])
+        self.gout = dev_tensor(inp["grad_out"])
+        self.out = torch.empty((w.N, w.queries, w.M * w.D), device=device)
+        self.loc = torch.empty_like(self.off)
+        self.attn = torch.empty_like(self.logits)
+        self.gval = torch.empty((w.N, w.S, w.M, w.D), device=device)
+        self.gloc = torch.empty_like(self.off)
+        self.gattn = torch.empty_like(self.logits)
+        self.gref = torch.empty_like(self.ref)
+        self.plan = None
+        if schedule == "tiled":
+            self.halo = TILE_HALO.get(w.name, 3) if halo is None else halo
+            self.ctas = TILE_CTAS.get(w.name, 2) if ctas is None else ctas
+            self.plan = m.msda_tile_plan(self.value, self.sh, self.starts, self.ref, K=w.K,
+                                         halo=self.halo, ctas_per_sm=self.ctas)
+        # our kernels per step: (plan build,) forward, backward
+        self.launches = 3 if schedule == "tiled" else 2
+
+    def describe(self) -> dict:
+        if self.plan is None:
+            return {"schedule": "untiled (msda.h calls)"}
+        gx, gy = self.plan.grid
+        return {"schedule": "tiled (msda_tiled.h): the tile plan is rebuilt from the reference "
+                            "points inside every timed forward",
+                "halo_px": self.halo, "ctas_per_sm": self.ctas, "grid": [gx, gy],
+                "windows": self.plan.windows, "window_kb": self.plan.desc.window_bytes / 1024}
+
+    def kernel_names(self) -> dict:
+        if self.plan is not None:
+            f = ("tile_plan_kernel + fwd_tiled_kernel (msda_tile_plan_build + "
+                 "msda_forward_fused_tiled)")
+            b = ("memset + bwd_tiled_kernel (msda_backward_fused_tiled)" if self.step == "fused"
+                 else "memset + bwd_tiled_kernel (msda_backward_tiled)")
+        else:
+            f = "fwd_kernel (msda_forward_fused)"
+            b = ("memset + bwd_kernel (msda_backward_fused)" if self.step == "fused"
+                 else "memset + bwd_kernel (msda_backward)")
+        return {"fwd": f, "bwd": b}
+
+    # stream=None: the current stream (the capture stream while a graph records)
+    def fwd(self, st, t=None):
+        m, t = self.m, t or self
+        extra = {} if self.step == "fused" else {"sampling_locations_out": t.loc,
+                                                  "attention_weights_out": t.attn}
+        if self.plan is not None:
+            m.msda_tile_plan_rebuild(self.plan, t.ref, buffer=getattr(t, "plan_buf", None),
+                                     stream=st)
+            plan = self.plan if not hasattr(t, "plan_buf") else \
+                m.TilePlan(self.plan.desc, t.plan_buf)
+            m.msda_forward_fused_tiled(t.value, self.sh, self.starts, t.ref, t.off, t.logits,
+                                       plan, out=t.out, stream=st, **extra)
+        else:
+            m.msda_forward_fused(t.value, self.sh, self.starts, t.ref, t.off, t.logits,
+                                 out=t.out, stream=st, **extra)
+
+    def bwd(self, st, t=None):
+        m, t = self.m, t or self
+        sh, starts = self.sh, self.starts
+        plan = None
+        if self.plan is not None:
+            plan = self.plan if not hasattr(t, "plan_buf") else \
+                m.TilePlan(self.plan.desc, t.plan_buf)
+        if self.step == "fused":
+            kw = dict(grad_value=t.gval, grad_reference_points=t.gref, grad_offsets=t.gloc,
+                      grad_logits=t.gattn, stream=st)
+            if plan is not None:
+                m.msda_backward_fused_tiled(t.value, sh, starts, t.ref, t.off, t.logits, t.gout,
+                                            plan, **kw)
+            else:
+                m.msda_backward_fused(t.value, sh, starts, t.ref, t.off, t.logits, t.gout, **kw)
+        else:
+            kw = dict(grad_value=t.gval, grad_sampling_locations=t.gloc,
+                      grad_attention_weights=t.gattn, stream=st)
+            if plan is not None:
+                m.msda_backward_tiled(t.value, sh, starts, t.loc, t.attn, t.gout, plan, **kw)
+            else:
+                m.msda_backward(t.value, sh, starts, t.loc, t.attn, t.gout, **kw)
+
+
+def time_steps(torch, steps, stream, flush, K, warmup, clocks=None):
+    """K timed steps after `warmup` untimed ones, each after an L2 flush:
+    per-step (fwd, bwd, step) milliseconds from CUDA events on `stream`."""
+    for _ in range(warmup):
+        flush.zero_()
+        steps.fwd(stream)
+        steps.bwd(stream)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.start()
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record(stream)
+        steps.fwd(stream)
+        ev[i][1].record(stream)
+        steps.bwd(stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.stop()
+    return ([ev[i][0].elapsed_time(ev[i][1]) for i in range(K)],
+            [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)],
+            [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)])
+
+
+def sub_record(torch, device, name, args, flush, peak, peak_kind):
+    """Device timing of another workload in the same run (a few steps): the
+    forward and backward times, queries/s, HBM fractions and clocks."""
+    w = wl.WORKLOADS[name]
+    inp = wl.make_inputs(w)
+    sched = "untiled" if name in UNTILED_DEFAULT or args.schedule == "untiled" else "tiled"
+    st = Steps(torch, device, w, inp, "split", sched)
+    del inp
+    stream = torch.cuda.current_stream(device)
+    clocks = ClockSampler(_pci_bus_id(torch, device), _nvml_index(device.index or 0))
+    f, b, s = time_steps(torch, st, stream, flush, args.also_steps, 3, clocks)
+    ab = algorithmic_bytes(w, "split")
+    ms_f, ms_b, ms_s = statistics.fmean(f), statistics.fmean(b), statistics.fmean(s)
+    rec = {"workload": WORKLOAD_TEXT[name], "value_dtype": w.value_dtype, "steps": len(s),
+           "warmup": 3, "ms_per_step": ms_s, "queries_per_s": w.N * w.queries / (ms_s / 1e3),
+           "fwd_ms": ms_f, "bwd_ms": ms_b,
+           "fwd_algorithmic_bytes": ab["fwd"], "bwd_algorithmic_bytes": ab["bwd"],
+           "fwd_frac_of_" + peak_kind: ab["fwd"] / (ms_f / 1e3) / 1e9 / peak,
+           "bwd_frac_of_" + peak_kind: ab["bwd"] / (ms_b / 1e3) / 1e9 / peak,
+           "kernels": st.kernel_names(), "clocks": clocks.summary(), **st.describe()}
+    del st
+    torch.cuda.empty_cache()
+    return rec
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
-
-    from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fused,
-                                                    msda_forward_fused)
 
     world, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -270,103 +446,48 @@ def run_ours(args):
                                 device_id=device)
     w = rank_workload(args.workload, rank)
     inp = wl.make_inputs(w)
-    sh = inp["spatial_shapes"]
-
-    def dev_tensor(a):
-        a = np.ascontiguousarray(a)
-        if a.dtype == np.uint16:
-            return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
-        return torch.from_numpy(a).to(device)
-
-    value = dev_tensor(inp["value"])
-    ref = dev_tensor(inp["reference_points"])
-    off = dev_tensor(inp["offsets"])
-    logits = dev_tensor(inp["logits"])
-    gout = dev_tensor(inp["grad_out"])
-    out = torch.empty((w.N, w.queries, w.M * w.D), device=device)
-    loc = torch.empty_like(off)
-    attn = torch.empty_like(logits)
-    gval = torch.empty((w.N, w.S, w.M, w.D), device=device)
-    gloc = torch.empty_like(off)
-    gattn = torch.empty_like(logits)
-    starts, _ = __import__("scale_deformable_attention_02_b200").msda_level_start_index(sh)
+    schedule = args.schedule or ("untiled" if args.workload in UNTILED_DEFAULT else "tiled")
+    st = Steps(torch, device, w, inp, args.step, schedule, args.halo, args.ctas_per_sm)
+    sched_desc = st.describe()
+    sh, starts = st.sh, st.starts
+    value, ref, off, logits = st.value, st.ref, st.off, st.logits
     stream = torch.cuda.current_stream(device)
 
-    gref = torch.empty_like(ref)
-    fused = args.step == "fused"
-
-    # stream=None: the current stream (the capture stream while a graph records)
-    def fwd_call(st):
-        if fused:
-            msda_forward_fused(value, sh, starts, ref, off, logits, out=out, stream=st)
-        else:
-            msda_forward_fused(value, sh, starts, ref, off, logits, out=out,
-                               sampling_locations_out=loc, attention_weights_out=attn,
-                               stream=st)
-
-    def bwd_call(st):
-        if fused:
-            msda_backward_fused(value, sh, starts, ref, off, logits, gout, grad_value=gval,
-                                grad_reference_points=gref, grad_offsets=gloc,
-                                grad_logits=gattn, stream=st)
-        else:
-            msda_backward(value, sh, starts, loc, attn, gout, grad_value=gval,
-                          grad_sampling_locations=gloc, grad_attention_weights=gattn,
-                          stream=st)
-
     graphs = []
+    timed = st
     if args.graph:
         side = torch.cuda.Stream(device)
         side.wait_stream(stream)
         with torch.cuda.stream(side):  # first launches (occupancy queries) off the capture
-            fwd_call(None)
-            bwd_call(None)
+            st.fwd(None)
+            st.bwd(None)
         stream.wait_stream(side)
         torch.cuda.synchronize()
         gf, gb = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(gf):
-            fwd_call(None)
+            st.fwd(None)
         with torch.cuda.graph(gb):
-            bwd_call(None)
+            st.bwd(None)
         graphs = [gf, gb]
-        step, step_bwd = gf.replay, gb.replay
-    else:
-        def step():
-            fwd_call(stream)
 
-        def step_bwd():
-            bwd_call(stream)
+        class Replay:
+            def fwd(self, s):
+                gf.replay()
+
+            def bwd(self, s):
+                gb.replay()
+        timed = Replay()
 
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush = torch.empty(max(2 * l2, 64 << 20), dtype=torch.uint8, device=device)
 
-    for _ in range(args.warmup):
-        flush.zero_()
-        step()
-        step_bwd()
-    torch.cuda.synchronize()
-
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     clocks = ClockSampler(_pci_bus_id(torch, device), _nvml_index(local))
     if world > 1:
         dist.barrier()
-    torch.cuda.synchronize()
-    clocks.start()
-    for i in range(K):
-        flush.zero_()
-        ev[i][0].record(stream)
-        step()
-        ev[i][1].record(stream)
-        step_bwd()
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
-    clocks.stop()
+    fwd_ms, bwd_ms, step_ms = time_steps(torch, timed, stream, flush, K, args.warmup, clocks)
     if world > 1:
         dist.barrier()
-    fwd_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
-    bwd_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    step_ms = [ev[i][0].elapsed_time(ev[i][2]) for i in range(K)]
     ms_step, ms_fwd, ms_bwd = max_over_ranks(
         [statistics.fmean(step_ms), statistics.fmean(fwd_ms), statistics.fmean(bwd_ms)],
         world, device)
@@ -376,8 +497,7 @@ def run_ours(args):
     # ---- end to end through the binding with host buffers -----------------
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value,
-                      queries)
+        e2e = run_e2e(args, torch, dist, world, device, stream, inp, w, st)
 
     # ---- roofline of the dominant launch ----------------------------------
     offs = corner_rows(torch, w, sh, starts, value, ref, off, logits)
@@ -387,25 +507,24 @@ def run_ours(args):
     dom = "bwd" if ms_bwd >= ms_fwd else "fwd"
     dom_ms = ms_bwd if dom == "bwd" else ms_fwd
     achieved = ab[dom] / (dom_ms / 1e3) / 1e9
-    bwd_name = ("memset + bwd_kernel (msda_backward_fused)" if args.step == "fused"
-                else "memset + bwd_kernel (msda_backward)")
+    names = st.kernel_names()
     kernels = {
-        "fwd": {"kernel": "fwd_kernel (msda_forward_fused)", "ms": ms_fwd,
-                "algorithmic_bytes": ab["fwd"],
+        "fwd": {"kernel": names["fwd"], "ms": ms_fwd, "algorithmic_bytes": ab["fwd"],
                 "GB_s": ab["fwd"] / (ms_fwd / 1e3) / 1e9},
-        "bwd": {"kernel": bwd_name, "ms": ms_bwd,
-                "algorithmic_bytes": ab["bwd"],
+        "bwd": {"kernel": names["bwd"], "ms": ms_bwd, "algorithmic_bytes": ab["bwd"],
                 "GB_s": ab["bwd"] / (ms_bwd / 1e3) / 1e9},
     }
     for k in kernels.values():
         k["frac_of_" + peak_kind] = k["GB_s"] / peak
+    tkey = args.workload if args.step == "split" else args.workload + "/fused"
+    if schedule == "untiled":
+        tkey += "/untiled"
     roofline = {
         "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
         "frac": achieved / peak, "frac_of_nominal_8000": achieved / 8000.0,
         "value_rows_touched": touched, "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)"
         if peak_kind == "measured" else "fallback 6.65 TB/s",
-        "traffic": read_traffic(args.workload if args.step == "split" else
-                                args.workload + "/fused", dom),
+        "traffic": read_traffic(tkey, dom),
         "kernel": kernels[dom]["kernel"],
         "algorithmic_bytes_per_launch": ab[dom],
     }
@@ -418,9 +537,17 @@ def run_ours(args):
             kernels["bwd"]["frac_of_row_floor"] = floors["gather_reduce_us"] / (ms_bwd * 1e3)
     del offs
 
+    also = []
+    if rank == 0 and world == 1 and args.also:
+        del st, inp
+        torch.cuda.empty_cache()
+        for name in args.also.split(","):
+            if name and name != args.workload:
+                also.append(sub_record(torch, device, name, args, flush, peak, peak_kind))
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, inp)
+        cpu = cpu_baseline(w, wl.make_inputs(w))
 
     if rank == 0:
         line = {
@@ -450,14 +577,16 @@ def run_ours(args):
                 "l2": "flushed before every timed step (memset of 2x L2, outside the events)",
                 "launch": ("two CUDA graph replays per step (forward graph, backward graph)"
                            if args.graph else "eager launches through the binding"),
+                **sched_desc,
             },
             "effective_GB_s": (ab["fwd"] + ab["bwd"]) / (ms_step / 1e3) / 1e9,
             "kernels": kernels,
             "roofline": roofline,
             "row_floors": floors,
+            "also": also,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": 2 * K,
+            "gpu_launches": launches_per_step(schedule) * K,
             "clocks": clocks.summary(),
             "impl": "ours",
         }
@@ -465,6 +594,12 @@ def run_ours(args):
     del graphs
     if world > 1:
         dist.destroy_process_group()
+
+
+def launches_per_step(schedule: str) -> int:
+    """Our kernels in one step: (the tile plan's sort,) the forward and the
+    backward; the backward's zero-fill is a runtime memset, not counted."""
+    return 3 if schedule == "tiled" else 2
 
 
 def corner_rows(torch, w, sh, starts, value, ref, off, logits):
@@ -544,17 +679,17 @@ def _nvml_index(local: int) -> int:
         return local
 
 
-def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_dev, queries):
+def run_e2e(args, torch, dist, world, device, stream, inp, w, st):
     """The same step through the public binding, starting from pinned host
-    buffers: every step copies its inputs host -> device, runs the fused
-    forward and the backward, and copies its results (out and the gradients)
-    device -> host, all inside the timed events.  Steps are pipelined over
-    two device buffer sets and three streams (copy in, compute, copy out), so
-    step i+1's upload and step i-1's download overlap step i's kernels."""
-    from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fused,
-                                                    msda_forward_fused)
+    buffers: every step copies its inputs host -> device, runs the step's
+    calls (the tile plan's sort, the forward, the backward), and copies its
+    results (out and the gradients) device -> host, all inside the timed
+    events.  Steps are pipelined over two device buffer sets and three streams
+    (copy in, compute, copy out), so step i+1's upload and step i-1's download
+    overlap step i's kernels."""
     fused = args.step == "fused"
     nbuf = 2
+    queries = w.N * w.queries
 
     def pinned(a):
         a = np.ascontiguousarray(a)
@@ -568,60 +703,53 @@ def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_
     if fused:
         res_shapes["grad_ref"] = tuple(inp["reference_points"].shape)
     h_out = {k: torch.empty(s, dtype=torch.float32).pin_memory() for k, s in res_shapes.items()}
-    bufs = []
-    for _ in range(nbuf):
-        bufs.append({
-            "in": {k: torch.empty(h_in[k].shape, dtype=h_in[k].dtype, device=device)
-                   for k in names},
-            "out": {k: torch.empty(s, dtype=torch.float32, device=device)
-                    for k, s in res_shapes.items()},
-            "loc": torch.empty(tuple(inp["offsets"].shape), device=device),
-            "attn": torch.empty(tuple(inp["logits"].shape), device=device),
-            "loaded": torch.cuda.Event(), "computed": torch.cuda.Event(),
-            "stored": torch.cuda.Event(), "used": False,
-        })
-    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
-    s_comp = stream
     bf16 = w.value_dtype == "bf16"
 
-    def compute(b):
-        d_in, d_out = b["in"], b["out"]
-        v = d_in["value"].view(torch.bfloat16) if bf16 else d_in["value"]
-        if fused:
-            msda_forward_fused(v, sh, starts, d_in["reference_points"], d_in["offsets"],
-                               d_in["logits"], out=d_out["out"], stream=s_comp)
-            msda_backward_fused(v, sh, starts, d_in["reference_points"], d_in["offsets"],
-                                d_in["logits"], d_in["grad_out"], grad_value=d_out["grad_value"],
-                                grad_reference_points=d_out["grad_ref"],
-                                grad_offsets=d_out["grad_loc"], grad_logits=d_out["grad_attn"],
-                                stream=s_comp)
-        else:
-            msda_forward_fused(v, sh, starts, d_in["reference_points"], d_in["offsets"],
-                               d_in["logits"], out=d_out["out"], sampling_locations_out=b["loc"],
-                               attention_weights_out=b["attn"], stream=s_comp)
-            msda_backward(v, sh, starts, b["loc"], b["attn"], d_in["grad_out"],
-                          grad_value=d_out["grad_value"], grad_sampling_locations=d_out["grad_loc"],
-                          grad_attention_weights=d_out["grad_attn"], stream=s_comp)
+    class Set:
+        """One device buffer set, named as Steps names its tensors."""
+
+    bufs = []
+    for _ in range(nbuf):
+        t = Set()
+        t.inp = {k: torch.empty(h_in[k].shape, dtype=h_in[k].dtype, device=device)
+                 for k in names}
+        t.res = {k: torch.empty(s, dtype=torch.float32, device=device)
+                 for k, s in res_shapes.items()}
+        t.value = t.inp["value"].view(torch.bfloat16) if bf16 else t.inp["value"]
+        t.ref, t.off, t.logits, t.gout = (t.inp[k] for k in names[1:])
+        t.out, t.gval, t.gloc, t.gattn = (t.res[k] for k in ("out", "grad_value", "grad_loc",
+                                                              "grad_attn"))
+        t.gref = t.res.get("grad_ref")
+        t.loc = torch.empty(tuple(inp["offsets"].shape), device=device)
+        t.attn = torch.empty(tuple(inp["logits"].shape), device=device)
+        if st.plan is not None:
+            t.plan_buf = torch.empty_like(st.plan.buffer)
+        t.loaded, t.computed, t.stored = (torch.cuda.Event() for _ in range(3))
+        t.used = False
+        bufs.append(t)
+    s_in, s_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    s_comp = stream
 
     def step(i):
         b = bufs[i % nbuf]
-        if b["used"]:
-            s_in.wait_event(b["computed"])    # step i-2 has read this input set
+        if b.used:
+            s_in.wait_event(b.computed)    # step i-2 has read this input set
         with torch.cuda.stream(s_in):
             for k in names:
-                b["in"][k].copy_(h_in[k], non_blocking=True)
-        b["loaded"].record(s_in)
-        s_comp.wait_event(b["loaded"])
-        if b["used"]:
-            s_comp.wait_event(b["stored"])    # step i-2's results have left this set
-        compute(b)
-        b["computed"].record(s_comp)
-        s_out.wait_event(b["computed"])
+                b.inp[k].copy_(h_in[k], non_blocking=True)
+        b.loaded.record(s_in)
+        s_comp.wait_event(b.loaded)
+        if b.used:
+            s_comp.wait_event(b.stored)    # step i-2's results have left this set
+        st.fwd(s_comp, b)
+        st.bwd(s_comp, b)
+        b.computed.record(s_comp)
+        s_out.wait_event(b.computed)
         with torch.cuda.stream(s_out):
             for k in res_shapes:
-                h_out[k].copy_(b["out"][k], non_blocking=True)
-        b["stored"].record(s_out)
-        b["used"] = True
+                h_out[k].copy_(b.res[k], non_blocking=True)
+        b.stored.record(s_out)
+        b.used = True
 
     for i in range(2 * nbuf):
         step(i)
@@ -660,11 +788,11 @@ def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_
             if do_in:
                 with torch.cuda.stream(s_in):
                     for k in names:
-                        b["in"][k].copy_(h_in[k], non_blocking=True)
+                        b.inp[k].copy_(h_in[k], non_blocking=True)
             if do_out:
                 with torch.cuda.stream(s_out):
                     for k in res_shapes:
-                        h_out[k].copy_(b["out"][k], non_blocking=True)
+                        h_out[k].copy_(b.res[k], non_blocking=True)
         s_in.wait_stream(s_out)
         c1.record(s_in)
         torch.cuda.synchronize()
@@ -678,9 +806,8 @@ def run_e2e(args, torch, dist, world, device, stream, inp, w, sh, starts, value_
             "copy_floor": floor, "frac_of_copy_floor": both_ms / ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n,
             "pipelining": f"{nbuf} device buffer sets; copy-in, compute and copy-out streams",
-            "api": "scale_deformable_attention_02_b200.msda_forward_fused + "
-                   + ("msda_backward_fused" if fused else "msda_backward")
-                   + " on pinned host buffers copied in and out every step"}
+            "api": "scale_deformable_attention_02_b200: " + " + ".join(st.kernel_names().values())
+                   + ", on pinned host buffers copied in and out every step"}
 
 
 # ---------------------------------------------------------------------------

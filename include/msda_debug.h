@@ -78,6 +78,16 @@ MSDA_API msda_status msda_debug_row_traffic(int mode, const void *value, msda_dt
                                             float *sink, int64_t sink_len, int depth, int ctas,
                                             msda_stream_t stream);
 
+/*
+ * Bounded waits of the tiled kernels (msda_tiled.h) that ran out on the
+ * current device since the last call: a tiled kernel waits for its tensor
+ * copies with a bounded number of tries, and if a wait ever ran out it would
+ * count it here and stop instead of spinning.  Synchronises the current
+ * device, reads the count into *count and clears it.
+ * Errors: MSDA_ERR_NULL, MSDA_ERR_CUDA.
+ */
+MSDA_API msda_status msda_debug_tiled_stalls(int64_t *count);
+
 #ifdef __cplusplus
 }
 #endif

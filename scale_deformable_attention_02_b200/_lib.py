@@ -1,5 +1,5 @@
-"""ctypes view of libmsda.so (the C ABI in include/msda.h and
-include/msda_debug.h) and of its bounds-checked build libmsda_checked.so
+"""ctypes view of libmsda.so (the C ABI in include/msda.h, include/msda_tiled.h
+and include/msda_debug.h) and of its bounds-checked build libmsda_checked.so
 (plus include/msda_checked.h).  No fallback: if a library is missing or does
 not load, every call raises."""
 from __future__ import annotations
@@ -31,6 +31,20 @@ class Dims(ctypes.Structure):
     _fields_ = [(k, ctypes.c_int64) for k in ("N", "Lq", "S", "M", "D", "L", "K")]
 
 
+TILE_MAX_LEVELS = 8
+I32 = ctypes.c_int32
+
+
+class TilePlan(ctypes.Structure):
+    """msda_tile_plan (include/msda_tiled.h)."""
+    _fields_ = [("N", ctypes.c_int64), ("Lq", ctypes.c_int64), ("S", ctypes.c_int64),
+                ("L", ctypes.c_int64), ("D", ctypes.c_int64), ("value_dtype", I32),
+                ("halo", I32), ("grid_x", I32), ("grid_y", I32), ("ctas_per_sm", I32),
+                ("reserved", I32), ("shapes", ctypes.c_int64 * (2 * TILE_MAX_LEVELS)),
+                ("window_w", I32 * TILE_MAX_LEVELS), ("window_h", I32 * TILE_MAX_LEVELS),
+                ("window_bytes", ctypes.c_int64), ("device_bytes", ctypes.c_int64)]
+
+
 SIGNATURES = {
     "msda_status_string": (ctypes.c_char_p, [INT]),
     "msda_abi_version": (INT, []),
@@ -45,8 +59,16 @@ SIGNATURES = {
     "msda_backward_grouped": (INT, [P, INT, P, P, P, P, P, P, P, P, Dims, I64, P]),
     "msda_backward_fused_grouped": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, P, P, Dims, I64,
                                           P]),
+    "msda_tile_plan_init": (INT, [INT, P, P, Dims, INT, INT, P]),
+    "msda_tile_plan_build": (INT, [P, P, INT, P, P]),
+    "msda_forward_tiled": (INT, [P, INT, P, P, P, P, P, Dims, P, P, P]),
+    "msda_forward_fused_tiled": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, Dims, P, P, P]),
+    "msda_backward_tiled": (INT, [P, INT, P, P, P, P, P, P, P, P, Dims, P, P, P]),
+    "msda_backward_fused_tiled": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, P, P, Dims, P, P,
+                                        P]),
     "msda_debug_sample_points": (INT, [P, P, P, Dims, P, P, P, P, P, P, P]),
     "msda_debug_row_traffic": (INT, [INT, P, INT, P, I64, P, I64, P, I64, INT, INT, P]),
+    "msda_debug_tiled_stalls": (INT, [P]),
 }
 
 # Only in libmsda_checked.so (include/msda_checked.h).

@@ -344,6 +344,225 @@ def msda_backward_fused(value: torch.Tensor, spatial_shapes, level_start_index,
     return grad_value, grad_reference_points, grad_offsets, grad_logits
 
 
+class TilePlan:
+    """A tile plan (include/msda_tiled.h): the host description `desc` (an
+    msda_tile_plan) and the device buffer `buffer` that msda_tile_plan_build
+    filled.  Valid while the reference points it was built from do not
+    change."""
+
+    def __init__(self, desc, buffer: torch.Tensor):
+        self.desc = desc
+        self.buffer = buffer
+
+    @property
+    def grid(self) -> tuple[int, int]:
+        return self.desc.grid_x, self.desc.grid_y
+
+    @property
+    def windows(self) -> list[tuple[int, int]]:
+        return [(self.desc.window_w[i], self.desc.window_h[i]) for i in range(self.desc.L)]
+
+
+def msda_tile_plan(value: torch.Tensor, spatial_shapes, level_start_index,
+                   reference_points: torch.Tensor, K: int, M: int | None = None,
+                   halo: int = 4, ctas_per_sm: int = 0, stream=None) -> TilePlan:
+    """Describe (msda_tile_plan_init), allocate and build (msda_tile_plan_build)
+    the tile plan of a problem: value [N,S,M,D] gives N, S, D, M and the value
+    dtype, reference_points [N,Lq,2|4] gives Lq and the points to sort."""
+    dev = value.device
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    if value.dim() != 4:
+        raise ValueError("value must be [N, S, M, D]")
+    N, S, Mv, D = value.shape
+    rdim = reference_points.shape[-1] if reference_points.dim() == 3 else -1
+    if rdim not in (2, 4):
+        raise ValueError("reference_points must be [N, Lq, 2] or [N, Lq, 4]")
+    Lq = reference_points.shape[1]
+    _need(reference_points, "reference_points", (N, Lq, rdim), dev)
+    d = _lib.Dims(N, Lq, S, Mv if M is None else M, D, shapes.shape[0], K)
+    desc = _lib.TilePlan()
+    _check(_lib.load().msda_tile_plan_init(_value_dtype(value), _hptr(shapes), _hptr(starts), d,
+                                           int(halo), int(ctas_per_sm), ctypes.byref(desc)),
+           "msda_tile_plan_init")
+    buf = torch.empty(max(int(desc.device_bytes), 16), device=dev, dtype=torch.uint8)
+    _check(_lib.load().msda_tile_plan_build(ctypes.byref(desc), _dptr(reference_points),
+                                            int(rdim), _dptr(buf), _stream_handle(dev, stream)),
+           "msda_tile_plan_build")
+    return TilePlan(desc, buf)
+
+
+def msda_tile_plan_rebuild(plan: TilePlan, reference_points: torch.Tensor,
+                           buffer: torch.Tensor | None = None, stream=None) -> None:
+    """Sort `reference_points` into the plan's cells again (msda_tile_plan_build),
+    into the plan's own buffer or into `buffer` (another uint8 device tensor
+    of at least plan.desc.device_bytes)."""
+    buf = plan.buffer if buffer is None else buffer
+    dev = buf.device
+    rdim = reference_points.shape[-1] if reference_points.dim() == 3 else -1
+    if rdim not in (2, 4):
+        raise ValueError("reference_points must be [N, Lq, 2] or [N, Lq, 4]")
+    _need(reference_points, "reference_points", (plan.desc.N, plan.desc.Lq, rdim), dev)
+    if buf.numel() < plan.desc.device_bytes or buf.dtype != torch.uint8:
+        raise ValueError("the plan buffer must be uint8 of at least plan.desc.device_bytes")
+    _check(_lib.load().msda_tile_plan_build(ctypes.byref(plan.desc), _dptr(reference_points),
+                                            int(rdim), _dptr(buf), _stream_handle(dev, stream)),
+           "msda_tile_plan_build")
+
+
+def msda_forward_tiled(value: torch.Tensor, spatial_shapes, level_start_index,
+                       sampling_locations: torch.Tensor, attention_weights: torch.Tensor,
+                       plan: TilePlan, out: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """msda_forward on a tile plan (the same result, cell by cell with the
+    value windows in shared memory)."""
+    dev = value.device
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    d = _value_dims(value, shapes, tuple(attention_weights.shape))
+    _need(sampling_locations, "sampling_locations", (d.N, d.Lq, d.M, d.L, d.K, 2), dev)
+    _need(attention_weights, "attention_weights", (d.N, d.Lq, d.M, d.L, d.K), dev)
+    if not value.is_contiguous():
+        raise ValueError("value must be contiguous")
+    if out is None:
+        out = torch.empty((d.N, d.Lq, d.M * d.D), device=dev, dtype=torch.float32)
+    _need(out, "out", (d.N, d.Lq, d.M * d.D), dev)
+    _check(_lib.load().msda_forward_tiled(
+        _dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
+        _dptr(sampling_locations), _dptr(attention_weights), _dptr(out), d,
+        ctypes.byref(plan.desc), _dptr(plan.buffer), _stream_handle(dev, stream)),
+        "msda_forward_tiled")
+    return out
+
+
+def msda_forward_fused_tiled(value: torch.Tensor, spatial_shapes, level_start_index,
+                             reference_points: torch.Tensor, offsets: torch.Tensor,
+                             logits: torch.Tensor, plan: TilePlan,
+                             out: torch.Tensor | None = None,
+                             sampling_locations_out: torch.Tensor | None = None,
+                             attention_weights_out: torch.Tensor | None = None,
+                             return_sampling: bool = False, stream=None):
+    """msda_forward_fused on a tile plan."""
+    dev = value.device
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    d = _value_dims(value, shapes, tuple(logits.shape))
+    rdim = reference_points.shape[-1] if reference_points.dim() == 3 else -1
+    if rdim not in (2, 4):
+        raise ValueError("reference_points must be [N, Lq, 2] or [N, Lq, 4]")
+    _need(reference_points, "reference_points", (d.N, d.Lq, rdim), dev)
+    _need(offsets, "offsets", (d.N, d.Lq, d.M, d.L, d.K, 2), dev)
+    _need(logits, "logits", (d.N, d.Lq, d.M, d.L, d.K), dev)
+    if not value.is_contiguous():
+        raise ValueError("value must be contiguous")
+    if out is None:
+        out = torch.empty((d.N, d.Lq, d.M * d.D), device=dev, dtype=torch.float32)
+    _need(out, "out", (d.N, d.Lq, d.M * d.D), dev)
+    if return_sampling:
+        if sampling_locations_out is None:
+            sampling_locations_out = torch.empty_like(offsets)
+        if attention_weights_out is None:
+            attention_weights_out = torch.empty_like(logits)
+    if sampling_locations_out is not None:
+        _need(sampling_locations_out, "sampling_locations_out", tuple(offsets.shape), dev)
+    if attention_weights_out is not None:
+        _need(attention_weights_out, "attention_weights_out", tuple(logits.shape), dev)
+    _check(_lib.load().msda_forward_fused_tiled(
+        _dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
+        _dptr(reference_points), int(rdim), _dptr(offsets), _dptr(logits), _dptr(out),
+        _dptr(sampling_locations_out), _dptr(attention_weights_out), d,
+        ctypes.byref(plan.desc), _dptr(plan.buffer), _stream_handle(dev, stream)),
+        "msda_forward_fused_tiled")
+    if return_sampling:
+        return out, sampling_locations_out, attention_weights_out
+    return out
+
+
+def msda_backward_tiled(value: torch.Tensor, spatial_shapes, level_start_index,
+                        sampling_locations: torch.Tensor, attention_weights: torch.Tensor,
+                        grad_out: torch.Tensor, plan: TilePlan,
+                        grad_value: torch.Tensor | None = None,
+                        grad_sampling_locations: torch.Tensor | None = None,
+                        grad_attention_weights: torch.Tensor | None = None,
+                        need_sampling_grad: bool = True, need_weight_grad: bool = True,
+                        stream=None):
+    """msda_backward on a tile plan.  Returns (grad_value, grad_loc or None,
+    grad_attn or None)."""
+    dev = value.device
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    d = _value_dims(value, shapes, tuple(attention_weights.shape))
+    _need(sampling_locations, "sampling_locations", (d.N, d.Lq, d.M, d.L, d.K, 2), dev)
+    _need(attention_weights, "attention_weights", (d.N, d.Lq, d.M, d.L, d.K), dev)
+    _need(grad_out, "grad_out", (d.N, d.Lq, d.M * d.D), dev)
+    if not value.is_contiguous():
+        raise ValueError("value must be contiguous")
+    if grad_value is None:
+        grad_value = torch.empty(tuple(value.shape), device=dev, dtype=torch.float32)
+    _need(grad_value, "grad_value", tuple(value.shape), dev)
+    if grad_sampling_locations is None and need_sampling_grad:
+        grad_sampling_locations = torch.empty_like(sampling_locations)
+    if grad_attention_weights is None and need_weight_grad:
+        grad_attention_weights = torch.empty_like(attention_weights)
+    if grad_sampling_locations is not None:
+        _need(grad_sampling_locations, "grad_sampling_locations",
+              tuple(sampling_locations.shape), dev)
+    if grad_attention_weights is not None:
+        _need(grad_attention_weights, "grad_attention_weights",
+              tuple(attention_weights.shape), dev)
+    _check(_lib.load().msda_backward_tiled(
+        _dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
+        _dptr(sampling_locations), _dptr(attention_weights), _dptr(grad_out), _dptr(grad_value),
+        _dptr(grad_sampling_locations), _dptr(grad_attention_weights), d,
+        ctypes.byref(plan.desc), _dptr(plan.buffer), _stream_handle(dev, stream)),
+        "msda_backward_tiled")
+    return grad_value, grad_sampling_locations, grad_attention_weights
+
+
+def msda_backward_fused_tiled(value: torch.Tensor, spatial_shapes, level_start_index,
+                              reference_points: torch.Tensor, offsets: torch.Tensor,
+                              logits: torch.Tensor, grad_out: torch.Tensor, plan: TilePlan,
+                              grad_value: torch.Tensor | None = None,
+                              grad_reference_points: torch.Tensor | None = None,
+                              grad_offsets: torch.Tensor | None = None,
+                              grad_logits: torch.Tensor | None = None,
+                              need_reference_grad: bool = True, need_offset_grad: bool = True,
+                              need_logit_grad: bool = True, stream=None):
+    """msda_backward_fused on a tile plan.  Returns (grad_value,
+    grad_reference_points or None, grad_offsets or None, grad_logits or None)."""
+    dev = value.device
+    shapes, starts = _levels(spatial_shapes, level_start_index)
+    d = _value_dims(value, shapes, tuple(logits.shape))
+    rdim = reference_points.shape[-1] if reference_points.dim() == 3 else -1
+    if rdim not in (2, 4):
+        raise ValueError("reference_points must be [N, Lq, 2] or [N, Lq, 4]")
+    _need(reference_points, "reference_points", (d.N, d.Lq, rdim), dev)
+    _need(offsets, "offsets", (d.N, d.Lq, d.M, d.L, d.K, 2), dev)
+    _need(logits, "logits", (d.N, d.Lq, d.M, d.L, d.K), dev)
+    _need(grad_out, "grad_out", (d.N, d.Lq, d.M * d.D), dev)
+    if not value.is_contiguous():
+        raise ValueError("value must be contiguous")
+    if grad_value is None:
+        grad_value = torch.empty(tuple(value.shape), device=dev, dtype=torch.float32)
+    _need(grad_value, "grad_value", tuple(value.shape), dev)
+    if grad_reference_points is None and need_reference_grad:
+        grad_reference_points = torch.empty_like(reference_points)
+    if grad_offsets is None and need_offset_grad:
+        grad_offsets = torch.empty_like(offsets)
+    if grad_logits is None and need_logit_grad:
+        grad_logits = torch.empty_like(logits)
+    if grad_reference_points is not None:
+        _need(grad_reference_points, "grad_reference_points", tuple(reference_points.shape), dev)
+    if grad_offsets is not None:
+        _need(grad_offsets, "grad_offsets", tuple(offsets.shape), dev)
+    if grad_logits is not None:
+        _need(grad_logits, "grad_logits", tuple(logits.shape), dev)
+    _check(_lib.load().msda_backward_fused_tiled(
+        _dptr(value), _value_dtype(value), _hptr(shapes), _hptr(starts),
+        _dptr(reference_points), int(rdim), _dptr(offsets), _dptr(logits), _dptr(grad_out),
+        _dptr(grad_value), _dptr(grad_reference_points), _dptr(grad_offsets),
+        _dptr(grad_logits), d, ctypes.byref(plan.desc), _dptr(plan.buffer),
+        _stream_handle(dev, stream)),
+        "msda_backward_fused_tiled")
+    return grad_value, grad_reference_points, grad_offsets, grad_logits
+
+
 def msda_debug_sample_points(spatial_shapes, level_start_index,
                              sampling_locations: torch.Tensor, stream=None) -> dict:
     """Per-sample cell record computed by the kernels' own cell arithmetic."""
@@ -399,3 +618,11 @@ def msda_debug_row_traffic(mode: int, rows: torch.Tensor, value: torch.Tensor | 
         _dptr(sink), 0 if sink is None else sink.numel(), int(depth), int(ctas),
         _stream_handle(dev, stream)),
         "msda_debug_row_traffic")
+
+
+def msda_debug_tiled_stalls() -> int:
+    """Bounded waits of the tiled kernels that ran out since the last call
+    (synchronises the device; include/msda_debug.h)."""
+    c = ctypes.c_int64(0)
+    _check(_lib.load().msda_debug_tiled_stalls(ctypes.byref(c)), "msda_debug_tiled_stalls")
+    return int(c.value)

@@ -10,6 +10,7 @@
 
 #include "msda.h"
 #include "msda_debug.h"
+#include "msda_api_util.h"
 #include "msda_internal.h"
 #ifdef MSDA_CHECKED
 #include "msda_checked.h"
@@ -19,10 +20,14 @@ namespace {
 
 using msda::Levels;
 using msda::kMaxLK;
+using namespace msda::api;
 
-constexpr int kAbiVersion = 10100;  // 1.1.0: MSDA_ERR_DEVICE_CHECK, msda_backward_fused
-constexpr int64_t kI32Max = 2147483647LL;
-constexpr int64_t kGuard = (int64_t)1 << 62;
+constexpr int kAbiVersion = 10200;  // 1.2.0: tiled entry points (msda_tiled.h)
+
+}  // namespace
+
+namespace msda {
+namespace api {
 
 thread_local int g_last_cuda_error = 0;
 
@@ -35,11 +40,6 @@ bool mul_le(int64_t a, int64_t b, int64_t limit, int64_t *out)
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
-
-struct Span {
-    const void *p;
-    int64_t bytes;
-};
 
 bool overlap(Span a, Span b)
 {
@@ -60,19 +60,6 @@ bool any_alias(const Span *outs, int nout, const Span *ins, int nin)
     }
     return false;
 }
-
-// Validated problem: element counts and launch-side metadata.
-struct Problem {
-    int64_t items;    // N*Lq*M
-    int64_t samples;  // N*Lq*M*L*K: per-head tensors (weights, logits)
-    int64_t lsamples; // N*Lq*G*L*K: per-group tensors (locations, offsets)
-    int64_t n_value;  // N*S*M*D
-    int64_t n_out;    // N*Lq*M*D
-    int esz;          // value element size
-    int nchunks;      // 16-byte chunks per value row
-    int lanes;        // lanes per row: next power of two >= nchunks
-    Levels lv;
-};
 
 // Dims, level metadata and size limits (no pointers).
 msda_status check_dims(msda_dtype dt, const int64_t *shapes, const int64_t *starts,
@@ -131,27 +118,6 @@ msda_status check_groups(const msda_dims &d, int64_t G, Problem *pr)
     return MSDA_OK;
 }
 
-template <class Params>
-void set_dims(Params *p, const msda_dims &d, int64_t G, const Problem &pr)
-{
-    p->items = pr.items;
-    p->Lq = (int)d.Lq;
-    p->S = (int)d.S;
-    p->M = (int)d.M;
-    p->D = (int)d.D;
-    p->L = (int)d.L;
-    p->K = (int)d.K;
-    p->G = (int)G;
-    p->Hg = (int)(d.M / G);
-    // item indices N*Lq*M stay below 2^31 (check_dims), so the kernels
-    // divide them in 32 bits
-    p->dM = msda::make_fastdiv((unsigned)(d.M > 0 ? d.M : 1));
-    p->dLq = msda::make_fastdiv((unsigned)(d.Lq > 0 ? d.Lq : 1));
-    p->dHg = msda::make_fastdiv((unsigned)(p->Hg > 0 ? p->Hg : 1));
-    p->nchunks = pr.nchunks;
-    p->lv = pr.lv;
-}
-
 msda_status cuda_status(cudaError_t e)
 {
     if (e == cudaSuccess) return MSDA_OK;
@@ -164,25 +130,6 @@ std::atomic<int64_t> g_check_limit{-1};
 thread_local int64_t g_violation_count = 0;
 thread_local int64_t g_violation_first = -1;
 #endif
-
-// The bounds-check fields of a launch: the value map's element count (or the
-// lowered test limit) and the device word.  Nothing in the default build.
-template <class Params>
-msda_status set_checks(Params *p, const Problem &pr)
-{
-    p->check_limit = pr.n_value;
-    p->check = nullptr;
-#ifdef MSDA_CHECKED
-    const int64_t lim = g_check_limit.load();
-    if (lim >= 0 && lim < p->check_limit) p->check_limit = lim;
-    p->check = msda::check_word();
-    if (!p->check) {
-        const cudaError_t e = cudaGetLastError();
-        return cuda_status(e != cudaSuccess ? e : cudaErrorUnknown);
-    }
-#endif
-    return MSDA_OK;
-}
 
 // Status of a launch.  The bounds-checked build also waits for the stream,
 // reads the device word, and clears it if the kernel recorded a violation.
@@ -207,7 +154,8 @@ msda_status launched(cudaError_t e, cudaStream_t s)
 #endif
 }
 
-}  // namespace
+}  // namespace api
+}  // namespace msda
 
 extern "C" {
 

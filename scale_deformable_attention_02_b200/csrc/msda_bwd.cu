@@ -22,6 +22,7 @@
 // Both scatter A w_j g with one vector `red.global.add.v4.f32` per 16 bytes.
 #include "msda_common.cuh"
 #include "msda_internal.h"
+#include "msda_rows.cuh"
 
 namespace msda {
 namespace {
@@ -54,27 +55,6 @@ __device__ __forceinline__ void reduce_scatter(float (&v)[kNV], int lane)
             v[i] = keep + __shfl_xor_sync(kFull, send, o);
         }
         reduce_scatter<o, h>(v, lane);
-    }
-}
-
-// Butterfly reduce-scatter of the first CNT values of v over aligned groups
-// of SPAN lanes (CNT a multiple of SPAN): afterwards lane b = lane % SPAN holds
-// in v[0, CNT/SPAN) the group totals of values b*CNT/SPAN ... (b+1)*CNT/SPAN - 1.
-template <int SPAN, int CNT, int N>
-__device__ __forceinline__ void reduce_scatter_n(float (&v)[N], int lane)
-{
-    static_assert(CNT <= N && CNT % SPAN == 0, "reduce-scatter shape");
-    if constexpr (SPAN > 1) {
-        constexpr int o = SPAN / 2;
-        constexpr int h = CNT / 2;
-        const bool upper = (lane & o) != 0;
-#pragma unroll
-        for (int i = 0; i < h; ++i) {
-            const float send = upper ? v[i] : v[i + h];
-            const float keep = upper ? v[i + h] : v[i];
-            v[i] = keep + __shfl_xor_sync(kFull, send, o);
-        }
-        reduce_scatter_n<o, h, N>(v, lane);  // the kept half now sits in v[0, h)
     }
 }
 
@@ -326,46 +306,6 @@ __global__ void __launch_bounds__(kWarps * 32)
         }
     }
 }
-
-// Four consecutive value elements of one lane, widened to fp32: a 16-byte
-// load for fp32, an 8-byte load for bf16.  The backward's fast path gives
-// every lane four elements so that R = D/4 lanes cover a row of the fp32
-// gradient and one vector reduction instruction updates whole 128-byte
-// gradient rows, whatever the value dtype.
-template <typename VT>
-struct Lane4;
-
-template <>
-struct Lane4<float> {
-    using Raw = uint4;
-    __device__ __forceinline__ static Raw load(const float *p)
-    {
-        return __ldg(reinterpret_cast<const uint4 *>(p));
-    }
-    __device__ __forceinline__ static void widen(const Raw &r, float (&v)[4])
-    {
-        v[0] = __uint_as_float(r.x);
-        v[1] = __uint_as_float(r.y);
-        v[2] = __uint_as_float(r.z);
-        v[3] = __uint_as_float(r.w);
-    }
-};
-
-template <>
-struct Lane4<__nv_bfloat16> {
-    using Raw = uint2;
-    __device__ __forceinline__ static Raw load(const __nv_bfloat16 *p)
-    {
-        return __ldg(reinterpret_cast<const uint2 *>(p));
-    }
-    __device__ __forceinline__ static void widen(const Raw &r, float (&v)[4])
-    {
-        v[0] = __uint_as_float(r.x << 16);
-        v[1] = __uint_as_float(r.x & 0xffff0000u);
-        v[2] = __uint_as_float(r.y << 16);
-        v[3] = __uint_as_float(r.y & 0xffff0000u);
-    }
-};
 
 // Fast path for D <= 32 (R = D/4 <= 8 lanes per row, four elements per lane).
 //

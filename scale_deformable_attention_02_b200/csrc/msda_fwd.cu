@@ -33,6 +33,7 @@
 // access); there is no dense contraction, so no tensor-core path.
 #include "msda_common.cuh"
 #include "msda_internal.h"
+#include "msda_rows.cuh"
 
 namespace msda {
 namespace {
@@ -249,55 +250,6 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
     }
 }
 
-// EPL consecutive value elements of one lane (16 or 8 bytes), widened to
-// float pairs when consumed.
-template <typename VT, int EPL>
-struct LaneLoad;
-
-template <>
-struct LaneLoad<float, 4> {
-    using Raw = uint4;
-    __device__ __forceinline__ static Raw load(const float *p)
-    {
-        return __ldg(reinterpret_cast<const uint4 *>(p));
-    }
-    __device__ __forceinline__ static void widen(const Raw &r, float2 (&v)[2])
-    {
-        v[0] = make_float2(__uint_as_float(r.x), __uint_as_float(r.y));
-        v[1] = make_float2(__uint_as_float(r.z), __uint_as_float(r.w));
-    }
-};
-
-template <>
-struct LaneLoad<__nv_bfloat16, 8> {
-    using Raw = uint4;
-    __device__ __forceinline__ static Raw load(const __nv_bfloat16 *p)
-    {
-        return __ldg(reinterpret_cast<const uint4 *>(p));
-    }
-    __device__ __forceinline__ static void widen(const Raw &r, float2 (&v)[4])
-    {
-        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)  // exact widening: bf16 bits become the high half
-            v[i] = make_float2(__uint_as_float(w[i] << 16), __uint_as_float(w[i] & 0xffff0000u));
-    }
-};
-
-template <>
-struct LaneLoad<__nv_bfloat16, 4> {
-    using Raw = uint2;
-    __device__ __forceinline__ static Raw load(const __nv_bfloat16 *p)
-    {
-        return __ldg(reinterpret_cast<const uint2 *>(p));
-    }
-    __device__ __forceinline__ static void widen(const Raw &r, float2 (&v)[2])
-    {
-        v[0] = make_float2(__uint_as_float(r.x << 16), __uint_as_float(r.x & 0xffff0000u));
-        v[1] = make_float2(__uint_as_float(r.y << 16), __uint_as_float(r.y & 0xffff0000u));
-    }
-};
-
 // ---------------------------------------------------------------------------
 // Fast path for value rows of at most 128 bytes (R <= 8 lanes per row).
 //
@@ -324,59 +276,6 @@ struct LaneLoad<__nv_bfloat16, 4> {
 #ifndef MSDA_FWD_PREFETCH
 #define MSDA_FWD_PREFETCH 1  // load the next round's inputs during this round's gathers
 #endif
-
-// Sums each chunk's accumulators over the 32/R slot lanes that hold it and
-// stores the item's output row (evict-first).  Where the lanes hold 32
-// elements in all (R * EPL == 32) this is a butterfly reduce-scatter: at xor
-// distance o a lane keeps one half of its values (the upper half if bit o of
-// its lane is set) and adds the partner's copy of that half, so after
-// log2(32/R) steps it holds one finished element, idx, of its chunk, and the
-// warp stores the row with one coalesced instruction (3 shuffles for
-// 4-element lanes, 7 for 8, against 8 and 24 for a full xor reduction).
-// Other widths take the full xor reduction, and the slot-0 lanes store.
-template <int R, int EPL>
-__device__ __forceinline__ void store_row(float2 (&acc)[EPL / 2], int lane, int chunk,
-                                          bool chunk_ok, float *row)
-{
-    constexpr int kNP = EPL / 2;
-    if constexpr (R * EPL == 32) {
-        float v[EPL];
-#pragma unroll
-        for (int i = 0; i < kNP; ++i) {
-            v[2 * i] = acc[i].x;
-            v[2 * i + 1] = acc[i].y;
-        }
-        int idx = 0;
-#pragma unroll
-        for (int o = 16, n = EPL; o >= R; o >>= 1, n >>= 1) {
-            const int half = n / 2;
-            const bool up = (lane & o) != 0;
-#pragma unroll
-            for (int i = 0; i < half; ++i) {
-                const float send = up ? v[i] : v[i + half];
-                const float keep = up ? v[i + half] : v[i];
-                v[i] = keep + __shfl_xor_sync(kFull, send, o);
-            }
-            if (up) idx += half;
-        }
-        if (chunk_ok) __stcs(row + chunk * EPL + idx, v[0]);
-    } else {
-#pragma unroll
-        for (int o = R; o < 32; o <<= 1)
-#pragma unroll
-            for (int i = 0; i < kNP; ++i) {
-                acc[i].x += __shfl_xor_sync(kFull, acc[i].x, o);
-                acc[i].y += __shfl_xor_sync(kFull, acc[i].y, o);
-            }
-        if (lane < R && chunk_ok) {  // slot 0
-            float4 *dst = reinterpret_cast<float4 *>(row + chunk * EPL);
-#pragma unroll
-            for (int i = 0; i < kNP / 2; ++i)
-                __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
-                                            acc[2 * i + 1].y));
-        }
-    }
-}
 
 template <typename VT, int EPL, int R, int P, bool kFused>
 __global__ void __launch_bounds__(kWarps * 32, MSDA_FWD_MIN_CTAS)

@@ -2,6 +2,7 @@
 // the kernels.  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -113,5 +114,69 @@ cudaError_t launch_row_traffic(TrafficParams p, int mode, int depth, int ctas,
 // address.
 unsigned long long *check_word();
 #endif
+
+// ---------------------------------------------------------------------------
+// Tiled kernels (msda_tiled.h): a tile plan sorts each batch entry's queries
+// into the cells of a gx x gy grid over the unit square; a work unit is one
+// (batch entry, cell, head) and stages the head's value window around the
+// cell on every level into shared memory.
+// ---------------------------------------------------------------------------
+constexpr int kTileLevels = 8;     // levels a tiled call takes
+constexpr int kTileMaxCells = 8192;
+
+// Device view of a plan and the unit schedule.  Checked on the host: the plan
+// matches the call's dims; windows are 0 (level not staged) or at least 2 x 2
+// pixels and at most 256 x 256.
+struct TileView {
+    const int *cell_start;  // [N][G + 1]: first sorted query of every cell
+    const int *perm;        // [N][Lq]: queries sorted by cell
+    int gx, gy, G, halo;
+    FastDiv dG;              // division by G
+    int ww[kTileLevels];     // window width and height per level, pixels
+    int wh[kTileLevels];
+    int soff[kTileLevels];   // byte offset of the level's window in dynamic shared memory
+    unsigned window_tx;      // bytes the windows of one unit bring in
+    int units;               // N * G * M
+    unsigned *stall;         // device word: waits that ran out (never expected)
+};
+
+// Tensor maps first: each CUtensorMap is 64-byte aligned.
+struct FwdTiledParams {
+    CUtensorMap maps[kTileLevels];  // value of level l as a 5-d tensor (D, M, W_l, H_l, N)
+    FwdParams f;
+    TileView t;
+};
+
+// The tiled backward also keeps, per chunk of up to T queries of a cell, the
+// chunk's grad_out rows, one record per sample inside its window, the records
+// sorted by window pixel, and the pixels' record ranges.  Byte offsets into
+// dynamic shared memory, after the windows.
+struct BwdTiledParams {
+    CUtensorMap maps[kTileLevels];
+    BwdParams b;
+    TileView t;
+    int T;                     // queries per chunk
+    int keys;                  // window pixels of all levels
+    int roff[kTileLevels + 1]; // first key of each level's window; roff[L] = keys
+    int off_g, off_rec, off_sorted, off_start, off_cursor;
+};
+
+struct TilePlanParams {
+    const float *ref;  // [N, Lq, ref_dim]
+    int ref_dim;
+    int N, Lq, gx, gy;
+    int *cell_start;   // [N][gx*gy + 1]
+    int *perm;         // [N][Lq]
+};
+
+cudaError_t launch_tile_plan(const TilePlanParams &p, cudaStream_t stream);
+cudaError_t launch_forward_tiled(const FwdTiledParams &p, bool bf16, bool fused,
+                                 int ctas_per_sm, int dyn_smem, cudaStream_t stream);
+cudaError_t launch_backward_tiled(const BwdTiledParams &p, bool bf16, bool fused, int dyn_smem,
+                                  cudaStream_t stream);
+// Static shared memory of the tiled backward kernel for these dims, or < 0.
+int backward_tiled_static_smem(bool bf16, bool fused, int D, int LK);
+// The device word that counts bounded waits that ran out, or nullptr.
+unsigned *stall_word();
 
 }  // namespace msda

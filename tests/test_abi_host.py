@@ -20,7 +20,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 OK, NULL, SHAPE, LEVELS, DTYPE, ALIGN, ALIAS, UNSUP = range(8)
 
-PRODUCT_HEADERS = ("msda.h", "msda_debug.h")
+PRODUCT_HEADERS = ("msda.h", "msda_tiled.h", "msda_debug.h")
 CHECKED_HEADERS = PRODUCT_HEADERS + ("msda_checked.h",)
 
 
@@ -74,7 +74,7 @@ def test_library_exports_nothing_else(path, headers):
 def test_status_strings_and_version(lib):
     for code, name in _lib.STATUS_NAMES.items():
         assert lib.msda_status_string(code).decode().startswith(name)
-    assert lib.msda_abi_version() == 10100
+    assert lib.msda_abi_version() == 10200
 
 
 def test_checked_build_host_calls():

@@ -1,8 +1,8 @@
 """bench.py keeps its output contract: one JSON line with the metric, the
 whole-job value, the timing bookkeeping, the roofline of the dominant launch
 (HBM fraction and the row-traffic floor), the end-to-end figure with its
-host<->device bytes, the clock record and the launch count.  A short run on
-the decoder workload (a few seconds of GPU time)."""
+host<->device bytes, the clock record, the launch count and the sub-records
+of other workloads.  Short runs (a few seconds of GPU time each)."""
 import json
 import os
 import subprocess
@@ -33,7 +33,7 @@ def _run(*args):
 
 def test_bench_json_contract():
     d = _run("--workload", "decoder", "--steps", "5", "--warmup", "3", "--e2e-steps", "2",
-             "--no-cpu-baseline")
+             "--no-cpu-baseline", "--also", "")
     for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
               "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
               "roofline", "e2e", "gpu_launches", "clocks", "impl"):
@@ -59,6 +59,22 @@ def test_bench_json_contract():
 
 def test_bench_graph_and_fused_step():
     d = _run("--workload", "decoder", "--steps", "5", "--warmup", "3", "--graph", "--step",
-             "fused", "--no-e2e", "--no-cpu-baseline", "--no-floors")
+             "fused", "--no-e2e", "--no-cpu-baseline", "--no-floors", "--also", "")
     assert d["value"] > 0 and "graph" in d["config"]["launch"]
     assert "msda_backward_fused" in d["kernels"]["bwd"]["kernel"]
+
+
+def test_bench_tiled_schedule_and_sub_records():
+    """The default schedule of the encoder is tiled: the plan's sort, the
+    tiled forward and the tiled backward are three launches per step; the
+    e2e leg runs the same calls; a sub-record times another workload."""
+    d = _run("--workload", "encoder", "--steps", "4", "--warmup", "3", "--e2e-steps", "2",
+             "--no-cpu-baseline", "--no-floors", "--also", "encoder_bf16", "--also-steps", "3")
+    assert d["config"]["schedule"].startswith("tiled")
+    assert d["gpu_launches"] == 3 * d["steps"]
+    assert "fwd_tiled_kernel" in d["kernels"]["fwd"]["kernel"]
+    assert "bwd_tiled_kernel" in d["kernels"]["bwd"]["kernel"]
+    assert d["e2e"]["value"] > 0 and "tiled" in d["e2e"]["api"]
+    (sub,) = d["also"]
+    assert "bf16" in sub["workload"] and sub["fwd_ms"] > 0 and sub["bwd_ms"] > 0
+    assert sub["queries_per_s"] > 0 and set(sub["clocks"]) >= {"sm_mhz", "reasons"}
