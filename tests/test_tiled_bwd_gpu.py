@@ -8,8 +8,9 @@ same order as the untiled kernel (a window corner outside the level reads
 zero and adds nothing), so the location, weight, offset and logit gradients
 equal the untiled ones bit for bit.  The value gradient is summed in another
 order (per window pixel on the chip, then one reduction per pixel), so it is
-compared within the atomics tolerance; so is the reference-point gradient,
-which the M heads add with atomics."""
+compared within the atomics tolerance.  The reference-point gradient, which
+the M heads add with atomics, is compared with the oracle's, with its
+rounding mass (its heads' terms can cancel)."""
 import numpy as np
 import pytest
 import torch
@@ -95,7 +96,6 @@ def _check_fused(d, halo, cps, value=None, n_sel=None):
     torch.cuda.synchronize()
     assert torch.equal(go, ugo), "tiled grad_offsets differ from the untiled ones"
     assert torch.equal(gz, ugz), "tiled grad_logits differ from the untiled ones"
-    assert_close(host(gr), host(ugr), **GRAD, what="tiled vs untiled grad_reference")
     assert_close(host(gv), host(ugv), **GRAD, what="tiled vs untiled grad_value")
     sel = range(d["logits"].shape[0]) if n_sel is None else n_sel
     for n in sel:
