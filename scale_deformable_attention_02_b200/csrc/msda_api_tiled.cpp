@@ -28,7 +28,7 @@ constexpr int64_t kSmemPerCtaMax = 232448;
 constexpr int64_t kSmemReserved = 1024;
 // Static shared memory of the tiled kernels (corner entries, barrier) and
 // the 128 bytes that align the windows, bound.
-constexpr int64_t kTiledStatic = 12 * 1024;
+constexpr int64_t kTiledStatic = 14 * 1024;
 constexpr int kMaxHalo = 64;
 // Work units (batch entry, cell, head) per resident CTA the grid aims for.
 constexpr int64_t kUnitsPerCta = 4;
@@ -251,17 +251,20 @@ bool backward_layout(msda::BwdTiledParams *p, const msda_tile_plan *pl, const ms
     if (keys >= (1 << 16)) return false;  // records keep the pixel in 16 bits
     p->keys = keys;
     for (int T = 512; T >= 32; T -= 32) {
+        // the chunk's sorted (query, coefficient) entries, four per sample at
+        // most, take the windows' place after phase A
+        if ((int64_t)T * LK * 4 * 8 > pl->window_bytes) continue;
         int64_t off = round_up(pl->window_bytes, 128);
         p->off_g = (int)off;
         off = round_up(off + (int64_t)T * d.D * 4, 16);
         p->off_rec = (int)off;
         off = round_up(off + (int64_t)T * LK * 16, 16);
-        p->off_sorted = (int)off;
-        off = round_up(off + (int64_t)T * LK * 2, 16);
         p->off_start = (int)off;
         off = round_up(off + (int64_t)(keys + 1) * 4, 16);
         p->off_cursor = (int)off;
-        off = round_up(off + (int64_t)keys * 4, 16) + 128;  // + the window base alignment
+        off = round_up(off + (int64_t)keys * 4, 16);
+        p->off_queue = (int)off;
+        off = round_up(off + (int64_t)T * 4, 16) + 128;  // + the window base alignment
         if (off + stat <= kSmemPerCtaMax) {
             p->T = T;
             *dyn = (int)off;

@@ -24,13 +24,15 @@
 //      (window pixel of its first corner, query, A, fx, fy), counted per
 //      pixel; any other sample reads global memory and adds A w_j g to
 //      grad_value directly, as bwd_kernel does;
-//   3. a counting sort orders the records by pixel (prefix sum of the
-//      counts, then one placement pass);
-//   4. phase B: R lanes take one window pixel, walk the records of the four
-//      cells that have it as a corner, sum A w_j g over them in registers and
-//      add the row to grad_value with one vector reduction per 16 bytes.
-//      Each touched pixel is reduced into L2 once per chunk instead of once
-//      per (sample, corner).
+//   3. a counting sort orders the contributions A w_j g by target pixel:
+//      phase A counted one per corner inside its level; after a prefix sum of
+//      the counts, one pass places a (query, A w_j) entry per corner, in the
+//      shared memory of the windows, which the chunk no longer reads;
+//   4. phase B: R lanes take one window pixel, walk its run of entries, sum
+//      A w_j g in registers and add the row to grad_value with one vector
+//      reduction per 16 bytes.  Each touched pixel is reduced into L2 once
+//      per chunk instead of once per (sample, corner).  The next chunk (of
+//      the same cell, or of the next one) copies the windows in again.
 // No shared-memory atomics touch floating point: the only shared atomics
 // are the integer counts and placements of the sort.
 #include "msda_common.cuh"
@@ -109,9 +111,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char *const win = dyn_raw + ((128u - (smem_addr(dyn_raw) & 127u)) & 127u);
     float *const sgo = reinterpret_cast<float *>(win + tp.off_g);        // [T][D] grad_out rows
     int4 *const rec = reinterpret_cast<int4 *>(win + tp.off_rec);        // [T][L*K] records
-    unsigned short *const sorted = reinterpret_cast<unsigned short *>(win + tp.off_sorted);
     int *const kstart = reinterpret_cast<int *>(win + tp.off_start);     // [keys + 1]
     int *const kcur = reinterpret_cast<int *>(win + tp.off_cursor);      // [keys]
+    int *const squeue = reinterpret_cast<int *>(win + tp.off_queue);     // [T] the chunk's queries
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
@@ -167,10 +169,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         for (int cb = q0; cb < q1; cb += tp.T) {
             const int cnt = min(tp.T, q1 - cb);
-            const bool first = cb == q0;
-            __syncthreads();  // the previous chunk is done with shared memory
-            if (first && tid == 0) {
-                fence_proxy_async_smem();
+            // the previous chunk is done with shared memory; its entries (written
+            // through the generic proxy) are ordered before the tensor copies
+            fence_proxy_async_smem();
+            __syncthreads();
+            if (tid == 0) {  // every chunk: the previous chunk's entries overwrote the windows
                 mbar_arrive_expect_tx(&bar, t.window_tx);
                 for (int l = 0; l < p.L; ++l) {
                     if (t.ww[l] == 0) continue;
@@ -179,16 +182,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tma_load_5d(win + t.soff[l], &tp.maps[l], 0, m, ox, oy, (int)n, &bar);
                 }
             }
-            // the chunk's grad_out rows, and zero pixel counts
+            // the chunk's queries (clamped: a stale plan is slow, never out of
+            // bounds) and grad_out rows, and zero pixel counts
             for (int i = tid / R; i < cnt; i += kThreads / R) {
-                if (!chunk_ok) continue;
                 const int q = min(max(__ldg(pl + cb + i), 0), p.Lq - 1);
+                if (chunk == 0) squeue[i] = q;
+                if (!chunk_ok) continue;
                 const float4 gq = __ldcs(reinterpret_cast<const float4 *>(
                     p.grad_out + (nbase + q) * MD + m * D + chunk * kVec));
                 *reinterpret_cast<float4 *>(sgo + i * D + chunk * kVec) = gq;
             }
             for (int k = tid; k <= tp.keys; k += kThreads) kstart[k] = 0;
-            if (first) {
+            {
                 const bool ok = mbar_wait(&bar, parity);
                 parity ^= 1u;
                 if (__syncthreads_or(!ok)) {
@@ -197,38 +202,56 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_wait(&bar, parity ^ 1u);
                     return;
                 }
-            } else {
-                __syncthreads();
             }
 
             // ---- phase A: dA, dloc; records of the in-window samples --------
+            // this lane's sample inputs in the round starting at item i0:
+            // (logit, off) fused, (attn, loc) unfused
+            float pa = 0.f, pb = 0.f, pc = 0.f;
+            auto fetch = [&](int i0) {
+                const int ii = i0 + seg;
+                pa = pb = pc = 0.f;
+                if (jact && ii < cnt) {
+                    const int64_t si = ((nbase + squeue[ii]) * M + m) * LK + j;
+                    if constexpr (kFused) {
+                        pa = __ldcs(p.logits + si);
+                        const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + si);
+                        pb = o.x;
+                        pc = o.y;
+                    } else {
+                        const float2 tl = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
+                        pb = tl.x;
+                        pc = tl.y;
+                        pa = __ldcs(p.attn + si);
+                    }
+                }
+            };
+            fetch(warp * kItems);
             for (int i0 = warp * kItems; i0 < cnt; i0 += kWarps * kItems) {
                 const int ii = i0 + seg;
                 const bool iact = ii < cnt;
                 const bool act = jact && iact;
-                const int q = iact ? min(max(__ldg(pl + cb + ii), 0), p.Lq - 1) : 0;
+                const int q = iact ? squeue[ii] : 0;
                 {
                     const int64_t nq = nbase + q;
-                    const int64_t si = (nq * M + m) * LK + j;
                     float lx = 0.f, ly = 0.f, a = 0.f;
                     if constexpr (kFused) {
-                        const float2 o = act ? __ldcs(reinterpret_cast<const float2 *>(p.off) + si)
-                                             : make_float2(0.f, 0.f);
                         // the fused forward's softmax and location map, bit for bit
-                        a = seg_softmax<P>(act ? __ldcs(p.logits + si) : 0.f, act);
+                        a = seg_softmax<P>(pa, act);
                         if (act) {
                             const float2 loc =
-                                msda_fused_location(p.ref, p.ref_dim, nq, o.x, o.y, H, W);
+                                msda_fused_location(p.ref, p.ref_dim, nq, pb, pc, H, W);
                             lx = loc.x;
                             ly = loc.y;
                         }
-                        smq[warp][seg][j] = make_float4(act ? a : 0.f, o.x, o.y, 0.f);
+                        smq[warp][seg][j] = make_float4(act ? a : 0.f, act ? pb : 0.f,
+                                                        act ? pc : 0.f, 0.f);
                     } else if (act) {
-                        const float2 tl = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
-                        lx = tl.x;
-                        ly = tl.y;
-                        a = __ldcs(p.attn + si);
+                        lx = pb;
+                        ly = pc;
+                        a = pa;
                     }
+                    fetch(i0 + kWarps * kItems);  // loads while this round gathers
                     int2 e[4] = {{-1, 0}, {-1, 0}, {-1, 0}, {-1, 0}};
                     float4 sr = make_float4(0.f, 0.f, 0.f, 0.f);
                     int4 pr = make_int4(-1, 0, 0, 0);
@@ -248,7 +271,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                             const int key = kbase + uy * ww + ux;
                             pr = make_int4(key | (ii << 16), __float_as_int(a),
                                            __float_as_int(fx), __float_as_int(fy));
-                            atomicAdd(&kstart[key], 1);
+                            // one value-gradient contribution per corner inside the level
+#pragma unroll
+                            for (int cc = 0; cc < 4; ++cc) {
+                                const int xx = x0 + (cc & 1), yy = y0 + (cc >> 1);
+                                if (xx >= 0 && xx < W && yy >= 0 && yy < H)
+                                    atomicAdd(&kstart[key + (cc >> 1) * ww + (cc & 1)], 1);
+                            }
                         } else {
 #pragma unroll
                             for (int cc = 0; cc < 4; ++cc) {
@@ -396,52 +425,63 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             __syncthreads();
 
-            // ---- counting sort of the records by window pixel --------------
+            // ---- counting sort of the contributions by window pixel --------
+            // Each in-window sample adds A w_j g to the pixel of each corner j
+            // inside its level.  The windows are no longer read in this chunk,
+            // so the sorted (query, A w_j) entries take their place.
             cta_exclusive_scan(kstart, tp.keys, warp_tot);
             for (int k = tid; k < tp.keys; k += kThreads) kcur[k] = kstart[k];
             __syncthreads();
+            int2 *const cent = reinterpret_cast<int2 *>(win);
             for (int r = tid; r < cnt * LK; r += kThreads) {
-                const int x = rec[r].x;
-                if (x >= 0) sorted[atomicAdd(&kcur[x & 0xffff], 1)] = (unsigned short)r;
+                const int4 rr = rec[r];
+                if (rr.x < 0) continue;
+                const int key = rr.x & 0xffff, ii = rr.x >> 16;
+                int l = 0;
+                while (l + 1 < p.L && key >= tp.roff[l + 1]) ++l;
+                const int wwl = t.ww[l];
+                const int loc = key - tp.roff[l];
+                const int uy = loc / wwl, ux = loc - uy * wwl;
+                const int x0 = window_origin(ccx, t.gx, p.lv.W[l], t.halo, wwl) + ux;
+                const int y0 = window_origin(ccy, t.gy, p.lv.H[l], t.halo, t.wh[l]) + uy;
+                const float a = __int_as_float(rr.y);
+                const float fx = __int_as_float(rr.z), fy = __int_as_float(rr.w);
+                const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+                const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int xx = x0 + (cc & 1), yy = y0 + (cc >> 1);
+                    if (xx < 0 || xx >= p.lv.W[l] || yy < 0 || yy >= p.lv.H[l]) continue;
+                    const int pos = atomicAdd(&kcur[key + (cc >> 1) * wwl + (cc & 1)], 1);
+                    cent[pos] = make_int2(ii, __float_as_int(a * w[cc]));
+                }
             }
             __syncthreads();
 
             // ---- phase B: one vector reduction per touched window pixel ----
             for (int pix = tid / R; pix < tp.keys; pix += kThreads / R) {
+                const int r0 = kstart[pix], r1 = kstart[pix + 1];
+                if (r0 == r1 || !chunk_ok) continue;
+                float acc[kVec] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
+                for (int idx = r0; idx < r1; ++idx) {
+                    const int2 e = cent[idx];
+                    const float coef = __int_as_float(e.y);
+                    const float4 g4 =
+                        *reinterpret_cast<const float4 *>(sgo + e.x * D + lane_elem);
+                    acc[0] = fmaf(coef, g4.x, acc[0]);
+                    acc[1] = fmaf(coef, g4.y, acc[1]);
+                    acc[2] = fmaf(coef, g4.z, acc[2]);
+                    acc[3] = fmaf(coef, g4.w, acc[3]);
+                }
                 int l = 0;
                 while (l + 1 < p.L && pix >= tp.roff[l + 1]) ++l;
-                const int wwl = t.ww[l];
+                const int wwl = t.ww[l], Wl = p.lv.W[l];
                 const int loc = pix - tp.roff[l];
                 const int py = loc / wwl, px = loc - py * wwl;
-                float acc[kVec] = {0.f, 0.f, 0.f, 0.f};
-                bool any = false;
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int dx = cc & 1, dy = cc >> 1;
-                    if (px < dx || py < dy) continue;
-                    const int k = pix - dy * wwl - dx;  // the cell with this pixel as corner cc
-                    const int r1 = kstart[k + 1];
-                    for (int idx = kstart[k]; idx < r1; ++idx) {
-                        const int4 rr = rec[sorted[idx]];
-                        const float a = __int_as_float(rr.y);
-                        const float fx = __int_as_float(rr.z), fy = __int_as_float(rr.w);
-                        const float wy = dy ? fy : __fsub_rn(1.f, fy);
-                        const float wx = dx ? fx : __fsub_rn(1.f, fx);
-                        const float coef = a * (wy * wx);
-                        const float4 g4 = *reinterpret_cast<const float4 *>(
-                            sgo + (rr.x >> 16) * D + lane_elem);
-                        acc[0] = fmaf(coef, g4.x, acc[0]);
-                        acc[1] = fmaf(coef, g4.y, acc[1]);
-                        acc[2] = fmaf(coef, g4.z, acc[2]);
-                        acc[3] = fmaf(coef, g4.w, acc[3]);
-                        any = true;
-                    }
-                }
-                if (!any || !chunk_ok) continue;
-                const int Hl = p.lv.H[l], Wl = p.lv.W[l];
                 const int gx = window_origin(ccx, t.gx, Wl, t.halo, wwl) + px;
-                const int gy = window_origin(ccy, t.gy, Hl, t.halo, t.wh[l]) + py;
-                if (gx < 0 || gx >= Wl || gy < 0 || gy >= Hl) continue;  // the zero border
+                const int gy = window_origin(ccy, t.gy, p.lv.H[l], t.halo, t.wh[l]) + py;
+                // gx, gy lie inside the level: only corners inside it were placed
                 const int64_t off = (int64_t)(p.lv.start[l] + gy * Wl + gx) * MD;
                 if (!msda_in_map(p.check, p.check_limit, mapoff + off + chunk * kVec, kVec))
                     continue;  // bounds-checked build: dropped and reported

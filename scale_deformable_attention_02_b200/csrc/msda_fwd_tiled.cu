@@ -36,9 +36,8 @@ namespace {
 
 constexpr int kWarps = 8;
 
-#ifndef MSDA_TILED_BATCH
-#define MSDA_TILED_BATCH 4  // corner-row groups loaded before the first is used
-#endif
+constexpr int kQueueQ = 512;  // queries of a cell taken per chunk (their order in shared memory)
+
 
 template <typename VT, int EPL, int R, int P, bool kFused, int kMinCtas>
 __global__ void __launch_bounds__(kWarps * 32, kMinCtas)
@@ -50,13 +49,9 @@ __global__ void __launch_bounds__(kWarps * 32, kMinCtas)
     const TileView &t = tp.t;
     constexpr int kSlots = 32 / R;   // (sample, corner) pairs per warp instruction
     constexpr int kItems = 32 / P;   // items per warp round
-    constexpr int kStride = P + 2;   // = 2 mod 8 for P >= 8: conflict-free entries
     constexpr int kNP = EPL / 2;
-    constexpr int kB0 = MSDA_TILED_BATCH;
-    constexpr int kB = kB0 * kSlots <= 4 * P ? kB0 : (4 * P) / kSlots;
-    static_assert(kB >= 1 && (4 * P) % (kB * kSlots) == 0, "a batch must tile the entries");
-    static_assert(kSlots % 4 == 0, "a warp instruction covers whole samples");
-    __shared__ int2 ent[kWarps][kItems][4 * kStride];  // (row offset, weight)
+    __shared__ int4 srec[kWarps][kItems][P];  // one record per sample
+    __shared__ int squeue[kQueueQ];           // the chunk's queries
     __shared__ __align__(8) uint64_t bar;
     extern __shared__ __align__(128) unsigned char win_raw[];
     // tensor copies land on 128-byte boundaries (the launch adds 128 bytes)
@@ -101,50 +96,81 @@ __global__ void __launch_bounds__(kWarps * 32, kMinCtas)
         if (q1 == q0) continue;  // the same for every thread of the CTA
         const int cy = c / t.gx, cx = c - cy * t.gx;
 
-        __syncthreads();  // every warp is done with the previous unit's windows
-        if (threadIdx.x == 0) {
-            fence_proxy_async_smem();
-            mbar_arrive_expect_tx(&bar, t.window_tx);
-            for (int l = 0; l < p.L; ++l) {
-                if (t.ww[l] == 0) continue;
-                const int ox = window_origin(cx, t.gx, p.lv.W[l], t.halo, t.ww[l]);
-                const int oy = window_origin(cy, t.gy, p.lv.H[l], t.halo, t.wh[l]);
-                tma_load_5d(win + t.soff[l], &tp.maps[l], 0, m, ox, oy, (int)n, &bar);
-            }
-        }
         // this lane's level window (its origin; the extent test below)
         const int wx0 = ww ? window_origin(cx, t.gx, W, t.halo, ww) : 0;
         const int wy0 = ww ? window_origin(cy, t.gy, H, t.halo, wh) : 0;
-        const bool ok = mbar_wait(&bar, parity);
-        parity ^= 1u;
-        if (__syncthreads_or(!ok)) {
-            // never expected: record it, give the copies a second bound, stop
-            if (threadIdx.x == 0 && t.stall) atomicAdd(t.stall, 1u);
-            mbar_wait(&bar, parity ^ 1u);
-            return;
-        }
-
         const int count = q1 - q0;
         const int *pl = t.perm + (int64_t)n * p.Lq + q0;
         const int64_t nbase = (int64_t)n * p.Lq;
         const int64_t vbe = ((int64_t)n * p.S * M + m) * (int64_t)D + lane_elem;
         const VT *vb = static_cast<const VT *>(p.value) + vbe;
 
-        for (int i0 = warp * kItems; i0 < count; i0 += kWarps * kItems) {
+        // this lane's sample inputs in the round starting at item i0 of the
+        // chunk: (logit, off) fused, (attn, loc) unfused
+        float pa = 0.f, pb = 0.f, pc = 0.f;
+        auto fetch = [&](int i0, int ccount) {
+            const int ii = i0 + seg;
+            pa = pb = pc = 0.f;
+            if (jact && ii < ccount) {
+                const int64_t si = ((nbase + squeue[ii]) * M + m) * LK + j;
+                if constexpr (kFused) {
+                    pa = __ldcs(p.logits + si);
+                    const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + si);
+                    pb = o.x;
+                    pc = o.y;
+                } else {
+                    const float2 tl = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
+                    pb = tl.x;
+                    pc = tl.y;
+                    pa = __ldcs(p.attn + si);
+                }
+            }
+        };
+
+        for (int cb = 0; cb < count; cb += kQueueQ) {
+            const int ccount = min(kQueueQ, count - cb);
+            const bool first = cb == 0;
+            fence_proxy_async_smem();  // this thread's window reads before the next copies
+            __syncthreads();  // every warp is done with the windows and the queue
+            if (first && threadIdx.x == 0) {
+                mbar_arrive_expect_tx(&bar, t.window_tx);
+                for (int l = 0; l < p.L; ++l) {
+                    if (t.ww[l] == 0) continue;
+                    const int ox = window_origin(cx, t.gx, p.lv.W[l], t.halo, t.ww[l]);
+                    const int oy = window_origin(cy, t.gy, p.lv.H[l], t.halo, t.wh[l]);
+                    tma_load_5d(win + t.soff[l], &tp.maps[l], 0, m, ox, oy, (int)n, &bar);
+                }
+            }
+            // the chunk's queries, clamped: a stale plan is slow, never out of bounds
+            for (int i = threadIdx.x; i < ccount; i += kWarps * 32)
+                squeue[i] = min(max(__ldg(pl + cb + i), 0), p.Lq - 1);
+            __syncthreads();
+            fetch(warp * kItems, ccount);  // in flight while the windows arrive
+            if (first) {
+                const bool ok = mbar_wait(&bar, parity);
+                parity ^= 1u;
+                if (__syncthreads_or(!ok)) {
+                    // never expected: record it, give the copies a second bound, stop
+                    if (threadIdx.x == 0 && t.stall) atomicAdd(t.stall, 1u);
+                    mbar_wait(&bar, parity ^ 1u);
+                    return;
+                }
+            }
+
+        for (int i0 = warp * kItems; i0 < ccount; i0 += kWarps * kItems) {
             // ---- phase 1: sample j of item i0 + seg ------------------------
             const int ii = i0 + seg;
-            const bool iact = ii < count;
+            const bool iact = ii < ccount;
             const bool act = jact && iact;
-            const int q = iact ? min(max(__ldg(pl + ii), 0), p.Lq - 1) : 0;
+            const int q = iact ? squeue[ii] : 0;
             const int64_t nq = nbase + q;
             const int64_t item = nq * M + m;
             const int64_t si = item * LK + j;
             float lx = 0.f, ly = 0.f, a = 0.f;
             if constexpr (kFused) {
-                a = seg_softmax<P>(act ? __ldcs(p.logits + si) : 0.f, act);
+                a = seg_softmax<P>(pa, act);
                 if (act) {
-                    const float2 o = __ldcs(reinterpret_cast<const float2 *>(p.off) + si);
-                    const float2 loc = msda_fused_location(p.ref, p.ref_dim, nq, o.x, o.y, H, W);
+                    const float2 loc = msda_fused_location(p.ref, p.ref_dim, nq, pb, pc, H, W);
                     lx = loc.x;
                     ly = loc.y;
                     if (p.loc_out)
@@ -152,81 +178,90 @@ __global__ void __launch_bounds__(kWarps * 32, kMinCtas)
                     if (p.attn_out) __stcs(p.attn_out + si, a);
                 }
             } else if (act) {
-                const float2 tl = __ldcs(reinterpret_cast<const float2 *>(p.loc) + si);
-                lx = tl.x;
-                ly = tl.y;
-                a = __ldcs(p.attn + si);
+                lx = pb;
+                ly = pc;
+                a = pa;
             }
+            fetch(i0 + kWarps * kItems, ccount);  // loads while this round gathers
             {
-                int2 e[4] = {{-1, 0}, {-1, 0}, {-1, 0}, {-1, 0}};
+                // one record per sample: (window row offset and row step, or the
+                // cell for a global read, or none; A; fx; fy)
+                int4 rc = make_int4(-1, 0, 0, 0);
                 float x, y, fx, fy;
                 int x0, y0;
                 if (act && msda_cell(lx, ly, H, W, x, y, x0, y0, fx, fy)) {
-                    const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
-                    const float w[4] = {hy * hx, hy * fx, fy * hx, fy * fx};
                     const int ux = x0 - wx0, uy = y0 - wy0;
-                    if (ux >= 0 && ux <= ww - 2 && uy >= 0 && uy <= wh - 2) {
+                    int code;
+                    if (ux >= 0 && ux <= ww - 2 && uy >= 0 && uy <= wh - 2)
                         // all four corners in the window (corners outside the
                         // level read its zero fill)
-                        const int b = soff + (uy * ww + ux) * rowb;
-                        const int step[4] = {0, rowb, ww * rowb, (ww + 1) * rowb};
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc)
-                            e[cc] = make_int2(shared_entry(b + step[cc]),
-                                              __float_as_int(w[cc] * a));
-                    } else {
-#pragma unroll
-                        for (int cc = 0; cc < 4; ++cc) {
-                            const int r = msda_row(start, H, W, y0 + (cc >> 1), x0 + (cc & 1));
-                            if (r >= 0) e[cc] = make_int2(r * MD, __float_as_int(w[cc] * a));
-                        }
-                    }
+                        code = window_record(soff + (uy * ww + ux) * rowb, ww * rowb);
+                    else
+                        code = global_record(x0, y0, W);
+                    rc = make_int4(code, __float_as_int(a), __float_as_int(fx), __float_as_int(fy));
                 }
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) ent[warp][seg][cc * kStride + j] = e[cc];
+                srec[warp][seg][j] = rc;
             }
             __syncwarp();
 
             // ---- phase 2: gather, item by item ----------------------------
+            // slot s walks samples s, s + kSlots, ...; for each it reads the
+            // sample's record once and its four corner rows (16 bytes a lane)
 #pragma unroll 1
             for (int it = 0; it < kItems; ++it) {
                 const int qi = __shfl_sync(kFull, q, it * P);
-                if (i0 + it >= count) break;  // uniform
-                const int2 *enl = ent[warp][it] + (slot & 3) * kStride + (slot >> 2);
+                if (i0 + it >= ccount) break;  // uniform
                 float2 acc[kNP];
 #pragma unroll
                 for (int i = 0; i < kNP; ++i) acc[i] = make_float2(0.f, 0.f);
-                for (int s0 = 0; s0 < LK; s0 += kB * (kSlots / 4)) {
-                    int2 e[kB];
-                    Raw raw[kB];
+                const int4 *rs = srec[warp][it];
+#pragma unroll 2
+                for (int smp = slot; smp < LK; smp += kSlots) {
+                    const int4 rc = rs[smp];
+                    if (rc.x == -1) continue;
+                    const float a = __int_as_float(rc.y);
+                    const float fx = __int_as_float(rc.z), fy = __int_as_float(rc.w);
+                    const float hx = __fsub_rn(1.f, fx), hy = __fsub_rn(1.f, fy);
+                    const float w[4] = {(hy * hx) * a, (hy * fx) * a, (fy * hx) * a, (fy * fx) * a};
+                    Raw raw[4];
+                    bool has[4] = {true, true, true, true};
+                    if (rc.x >= 0) {
+                        const unsigned char *pb = wlane + (rc.x & kRecOffMask);
+                        const int step = (rc.x >> kRecOffBits) << 4;
+                        raw[0] = *reinterpret_cast<const Raw *>(pb);
+                        raw[1] = *reinterpret_cast<const Raw *>(pb + rowb);
+                        raw[2] = *reinterpret_cast<const Raw *>(pb + step);
+                        raw[3] = *reinterpret_cast<const Raw *>(pb + step + rowb);
+                    } else {
+                        // outside the window: this sample's level, its cell, global rows
+                        const int l = smp / K;
+                        const int Hl = p.lv.H[l], Wl = p.lv.W[l];
+                        const int cell = -2 - rc.x;
+                        const int cy0 = cell / (Wl + 1) - 1, cx0 = cell % (Wl + 1) - 1;
 #pragma unroll
-                    for (int b = 0; b < kB; ++b) {
-                        e[b] = enl[s0 + b * (kSlots / 4)];
-                        if (e[b].x <= -2) {
-                            raw[b] = *reinterpret_cast<const Raw *>(wlane + (-2 - e[b].x));
-                        } else if (e[b].x >= 0) {
-                            if (!msda_in_map(p.check, p.check_limit, vbe + e[b].x, EPL))
-                                e[b].x = -1;  // bounds-checked build: skipped, reads as zero
-                            else
-                                raw[b] = LL::load(vb + e[b].x);
+                        for (int cc = 0; cc < 4; ++cc) {
+                            const int r = msda_row(p.lv.start[l], Hl, Wl, cy0 + (cc >> 1),
+                                                   cx0 + (cc & 1));
+                            has[cc] = r >= 0 && msda_in_map(p.check, p.check_limit,
+                                                            vbe + (int64_t)r * MD, EPL);
+                            if (has[cc]) raw[cc] = LL::load(vb + (int64_t)r * MD);
                         }
                     }
 #pragma unroll
-                    for (int b = 0; b < kB; ++b) {
-                        if (e[b].x != -1) {
-                            float2 v[kNP];
-                            LL::widen(raw[b], v);
-                            const float wb = __int_as_float(e[b].y);
-                            const float2 w2 = make_float2(wb, wb);
+                    for (int cc = 0; cc < 4; ++cc) {
+                        if (!has[cc]) continue;
+                        float2 v[kNP];
+                        LL::widen(raw[cc], v);
+                        const float2 w2 = make_float2(w[cc], w[cc]);
 #pragma unroll
-                            for (int i = 0; i < kNP; ++i) acc[i] = __ffma2_rn(w2, v[i], acc[i]);
-                        }
+                        for (int i = 0; i < kNP; ++i) acc[i] = __ffma2_rn(w2, v[i], acc[i]);
                     }
                 }
                 store_row<R, EPL>(acc, lane, chunk, chunk_ok,
                                   p.out + (nbase + qi) * (int64_t)MD + m * D);
             }
             __syncwarp();  // the next round overwrites this warp's entries
+        }
         }
     }
     __syncthreads();

@@ -148,9 +148,10 @@ struct FwdTiledParams {
 };
 
 // The tiled backward also keeps, per chunk of up to T queries of a cell, the
-// chunk's grad_out rows, one record per sample inside its window, the records
-// sorted by window pixel, and the pixels' record ranges.  Byte offsets into
-// dynamic shared memory, after the windows.
+// chunk's grad_out rows, one record per sample inside its window, the pixels'
+// contribution counts (then run starts) and placement cursors, and the
+// chunk's queries.  Byte offsets into dynamic shared memory, after the
+// windows, whose space then holds the sorted contributions.
 struct BwdTiledParams {
     CUtensorMap maps[kTileLevels];
     BwdParams b;
@@ -158,7 +159,7 @@ struct BwdTiledParams {
     int T;                     // queries per chunk
     int keys;                  // window pixels of all levels
     int roff[kTileLevels + 1]; // first key of each level's window; roff[L] = keys
-    int off_g, off_rec, off_sorted, off_start, off_cursor;
+    int off_g, off_rec, off_start, off_cursor, off_queue;
 };
 
 struct TilePlanParams {

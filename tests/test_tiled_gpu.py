@@ -5,9 +5,9 @@ depend on the schedule:
 
   * against the oracle, element by element, with the tolerances of the
     untiled calls (fp32 1e-5 / 1e-6; the fused locations bit for bit);
-  * against the untiled call on the same inputs: for items of at most 16
-    samples the tiled forward sums every item's corner terms in the untiled
-    kernel's order, so the outputs are equal;
+  * against the untiled call on the same inputs, within the fp32 tolerance
+    (the tiled kernel sums an item's corner terms in another order), with the
+    locations and weights of the fused call bit for bit;
   * the plan itself against a CPU count of the reference points' cells.
 
 The plans cover coarse and fine grids (one to three resident CTAs per SM),
@@ -105,8 +105,7 @@ def test_tiled_encoder_fused_forward(name, halo, cps):
     assert_bits_equal(host(loc), oloc, what=f"{name} tiled loc")
     assert_close(host(a), oA, **F32, what=f"{name} tiled softmax")
     assert_close(host(out), ora, **F32, what=f"{name} tiled out")
-    # 16 samples per item: the untiled kernel's summation order, so equal
-    assert torch.equal(out, uout), f"{name}: tiled and untiled forward differ"
+    assert_close(host(out), host(uout), **F32, what=f"{name} tiled vs untiled")
     assert torch.equal(loc, uloc) and torch.equal(a, ua)
 
 
@@ -180,18 +179,14 @@ def test_tiled_random_problems(case):
     _loc_equal(host(loc), oloc, "tiled fused loc")
     assert_close(host(a), oA, **F32, what="tiled fused softmax")
     assert_close(host(out), ora, **F32, what="tiled fused out")
-    LK = len(shapes) * K
-    if LK <= 16:
-        assert torch.equal(out, uout), "tiled and untiled fused forward differ"
-    else:
-        assert_close(host(out), host(uout), **F32, what="tiled vs untiled")
+    assert_close(host(out), host(uout), **F32, what="tiled vs untiled")
     # the unfused tiled call on the oracle's locations and weights
     A = oA.astype(np.float32)
     t_out = msda_forward_tiled(value, sh, None, to_dev(oloc), to_dev(A), plan)
     assert_close(host(t_out), oracle.forward(d["value"], sh, oloc, A), **F32,
                  what="tiled unfused out")
-    if LK <= 16:
-        assert torch.equal(t_out, msda_forward(value, sh, None, to_dev(oloc), to_dev(A)))
+    assert_close(host(t_out), host(msda_forward(value, sh, None, to_dev(oloc), to_dev(A))),
+                 **F32, what="tiled vs untiled unfused")
 
 
 def test_tiled_all_queries_in_one_cell():
@@ -203,7 +198,7 @@ def test_tiled_all_queries_in_one_cell():
     sh = d["spatial_shapes"]
     plan, (out, loc, a), (uout, _, _) = _fused_both(d, 3, 2)
     _check_plan(plan, d["reference_points"])
-    assert torch.equal(out, uout)
+    assert_close(host(out), host(uout), **F32, what="one-cell tiled vs untiled")
     ora, _, _ = oracle.forward_fused(d["value"], sh, d["reference_points"], d["offsets"],
                                      d["logits"])
     assert_close(host(out), ora, **F32, what="one-cell out")

@@ -44,7 +44,7 @@ def _init(lib, sh, st, d, dtype=0, halo=3, cps=2):
 
 def _budget(cps):
     per_cta = min(233472 // cps - 1024, 232448)
-    return per_cta - 12 * 1024
+    return per_cta - 14 * 1024
 
 
 @pytest.mark.parametrize("name,dtype,halo,cps", [("encoder", 0, 3, 2), ("encoder", 0, 4, 1),
