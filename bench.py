@@ -74,8 +74,8 @@ def parse_args(argv=None):
                          "their replays (the launch-latency path for small problems such "
                          "as the decoder)")
     ap.add_argument("--schedule", choices=["tiled", "untiled"], default=None,
-                    help="tiled: tile plan + msda_tiled.h calls (default, except the decoder); "
-                         "untiled: the msda.h calls")
+                    help="untiled: the msda.h calls (default); tiled: tile plan + msda_tiled.h "
+                         "calls")
     ap.add_argument("--halo", type=int, default=None,
                     help="window halo of the tiled schedule, pixels (default per workload)")
     ap.add_argument("--ctas-per-sm", type=int, default=None,
@@ -275,9 +275,12 @@ TILE_HALO = {"encoder": 3, "encoder_bf16": 3, "encoder_compass": 4, "stress": 8,
              "tiny": 1}
 # Resident CTAs per SM the tiled windows are sized for.
 TILE_CTAS = {"stress": 1}
-# Workloads whose default schedule is untiled: the decoder's 300 queries per
-# image are spread over the whole map, so cells would hold one or two queries.
-UNTILED_DEFAULT = {"decoder", "tiny"}
+# Default schedule: untiled (the msda.h calls).  The tiled schedule
+# (msda_tiled.h) stages value windows in shared memory and cuts the L2->SM
+# bytes and the L2 reductions, but measured slower on B200 for every workload
+# here (encoder fp32: forward 202 against 163 us, backward 693 against
+# 439 us); it stays selectable with --schedule tiled.
+DEFAULT_SCHEDULE = "untiled"
 
 
 class Steps:
@@ -414,7 +417,7 @@ def sub_record(torch, device, name, args, flush, peak, peak_kind):
     forward and backward times, queries/s, HBM fractions and clocks."""
     w = wl.WORKLOADS[name]
     inp = wl.make_inputs(w)
-    sched = "untiled" if name in UNTILED_DEFAULT or args.schedule == "untiled" else "tiled"
+    sched = args.schedule or DEFAULT_SCHEDULE
     st = Steps(torch, device, w, inp, "split", sched)
     del inp
     stream = torch.cuda.current_stream(device)
@@ -446,7 +449,7 @@ def run_ours(args):
                                 device_id=device)
     w = rank_workload(args.workload, rank)
     inp = wl.make_inputs(w)
-    schedule = args.schedule or ("untiled" if args.workload in UNTILED_DEFAULT else "tiled")
+    schedule = args.schedule or DEFAULT_SCHEDULE
     st = Steps(torch, device, w, inp, args.step, schedule, args.halo, args.ctas_per_sm)
     sched_desc = st.describe()
     sh, starts = st.sh, st.starts

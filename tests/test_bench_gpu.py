@@ -42,7 +42,7 @@ def test_bench_json_contract():
     assert d["higher_is_better"] is True and d["scaling"] == "weak" and d["impl"] == "ours"
     assert d["value"] > 0 and d["ms_per_step"] > 0
     assert d["gpu_launches"] == 2 * d["steps"]
-    assert "workload" in d["config"]
+    assert "workload" in d["config"] and d["config"]["schedule"].startswith("untiled")
     r = d["roofline"]
     for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
         assert k in r, k
@@ -65,11 +65,12 @@ def test_bench_graph_and_fused_step():
 
 
 def test_bench_tiled_schedule_and_sub_records():
-    """The default schedule of the encoder is tiled: the plan's sort, the
-    tiled forward and the tiled backward are three launches per step; the
-    e2e leg runs the same calls; a sub-record times another workload."""
-    d = _run("--workload", "encoder", "--steps", "4", "--warmup", "3", "--e2e-steps", "2",
-             "--no-cpu-baseline", "--no-floors", "--also", "encoder_bf16", "--also-steps", "3")
+    """With --schedule tiled the plan's sort, the tiled forward and the tiled
+    backward are three launches per step; the e2e leg runs the same calls; a
+    sub-record times another workload on the same schedule."""
+    d = _run("--workload", "encoder", "--schedule", "tiled", "--steps", "4", "--warmup", "3",
+             "--e2e-steps", "2", "--no-cpu-baseline", "--no-floors", "--also", "encoder_bf16",
+             "--also-steps", "3")
     assert d["config"]["schedule"].startswith("tiled")
     assert d["gpu_launches"] == 3 * d["steps"]
     assert "fwd_tiled_kernel" in d["kernels"]["fwd"]["kernel"]
