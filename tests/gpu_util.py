@@ -48,8 +48,31 @@ def host(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu").numpy()
 
 
-def assert_close(gpu, ora, rtol, atol, what="", mass=None):
-    """|gpu - ora| <= atol + rtol*|ora| (+ KAPPA * 2^-24 * mass if given)."""
+def value_grad_terms(value, shapes, loc, attn, grad_out):
+    """(terms, mass) of every grad_value element: terms is the number of
+    (sample, corner) contributions it sums, counted from the oracle's corner
+    rows; mass is the sum of their absolute values, which is the oracle's
+    grad_value for |attention weights| and |grad_out| (corner weights are not
+    negative).  A sum of n terms formed in any order is within
+    n * 2^-24 * mass of the exact sum, whatever the order of the atomics."""
+    import oracle
+    N, Lq, M, L, K, _ = loc.shape
+    S, D = value.shape[1], value.shape[3]
+    rows = oracle.sample_points(loc, shapes)["rows"].reshape(N, Lq, M, L * K * 4)
+    n = np.arange(N).reshape(N, 1, 1, 1)
+    m = np.arange(M).reshape(1, 1, M, 1)
+    ok = rows >= 0
+    idx = ((n * S + rows) * M + m)[ok]
+    cnt = np.bincount(idx, minlength=N * S * M).reshape(N, S, M, 1)
+    terms = np.broadcast_to(cnt, (N, S, M, D)).astype(np.float64)
+    mass = oracle.backward(value, shapes, loc, np.abs(np.asarray(attn, np.float64)),
+                           np.abs(np.asarray(grad_out, np.float64)))[0]
+    return terms, mass
+
+
+def assert_close(gpu, ora, rtol, atol, what="", mass=None, terms=None):
+    """|gpu - ora| <= atol + rtol*|ora| (+ KAPPA * 2^-24 * mass if given, or
+    terms * 2^-24 * mass with a per-element term count)."""
     g = np.asarray(gpu, dtype=np.float64)
     o = np.asarray(ora, dtype=np.float64)
     assert g.shape == o.shape, (what, g.shape, o.shape)
@@ -60,7 +83,8 @@ def assert_close(gpu, ora, rtol, atol, what="", mass=None):
     err = np.abs(g - o)
     bound = atol + rtol * np.abs(o)
     if mass is not None:
-        bound = bound + KAPPA * U32 * np.where(fin, np.asarray(mass, dtype=np.float64), 0.0)
+        k = KAPPA if terms is None else np.asarray(terms, dtype=np.float64)
+        bound = bound + k * U32 * np.where(fin, np.asarray(mass, dtype=np.float64), 0.0)
     bad = err > bound
     if bad.any():
         i = np.unravel_index(np.argmax(err - bound), err.shape)

@@ -22,7 +22,7 @@ from scale_deformable_attention_02_b200 import (MsdaError, checked_library, last
                                                 msda_forward, msda_forward_fused)
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import F32, GRAD, PLAIN, assert_close, host, to_dev
+from gpu_util import F32, GRAD, PLAIN, assert_close, host, to_dev, value_grad_terms
 
 pytestmark = pytest.mark.gpu
 
@@ -109,7 +109,9 @@ def test_checked_build_default_bound_matches_oracle(case):
     # bf16 value bits are widened exactly on both sides: the fp32 bound holds
     assert_close(host(outs["out"]), out, **F32, what="checked forward")
     assert_close(host(outs["fout"]), fo, **F32, what="checked fused forward")
-    assert_close(host(outs["gv"]), ogv, **GRAD, what="checked grad_value")
+    tv, mv = value_grad_terms(d["value"], d["spatial_shapes"], d["sampling_locations"], A,
+                              d["grad_out"])
+    assert_close(host(outs["gv"]), ogv, **GRAD, what="checked grad_value", mass=mv, terms=tv)
     assert_close(host(outs["gl"]), ogl, **PLAIN, what="checked grad_loc", mass=mgl)
     assert_close(host(outs["ga"]), oga, **PLAIN, what="checked grad_attn", mass=mga)
 

@@ -12,7 +12,7 @@ from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fus
                                                 msda_forward_fused)
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import F32, GRAD, assert_close, host, to_dev
+from gpu_util import F32, GRAD, assert_close, host, to_dev, value_grad_terms
 
 pytestmark = pytest.mark.gpu
 
@@ -73,5 +73,7 @@ def test_decoder_step_in_cuda_graph(fused_bwd):
         oloc = oracle.locations_f32(d["reference_points"], d["offsets"], sh)
         A = oracle.softmax(d["logits"]).astype(np.float32)
         ogv, _, _ = oracle.backward(d["value"], sh, oloc, A, d["grad_out"])
-        assert_close(host(gv), ogv, **GRAD, what="graph grad_value vs oracle")
+        tv, mv = value_grad_terms(d["value"], sh, oloc, A, d["grad_out"])
+        assert_close(host(gv), ogv, **GRAD, what="graph grad_value vs oracle", mass=mv,
+                     terms=tv)
     del graph

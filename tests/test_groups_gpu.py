@@ -14,7 +14,7 @@ from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fus
 from scale_deformable_attention_02_b200 import workloads as wl
 
 from gpu_util import (F32, GRAD, KAPPA, PLAIN, U32, assert_bits_equal, assert_close, grad_tol,
-                      host, to_dev)
+                      host, to_dev, value_grad_terms)
 
 pytestmark = pytest.mark.gpu
 
@@ -62,7 +62,8 @@ def test_grouped_forward_and_backward(case):
                                to_dev(d["grad_out"]), groups=G)
     ogv, ogl, oga, mgl, mga = oracle.backward(d["value"], sh, loc_h, A, d["grad_out"],
                                               with_mass=True)
-    assert_close(host(gv), ogv, **GRAD, what="grouped grad_value")
+    tv, mv = value_grad_terms(d["value"], sh, loc_h, A, d["grad_out"])
+    assert_close(host(gv), ogv, **GRAD, what="grouped grad_value", mass=mv, terms=tv)
     assert_close(host(ga), oga, **PLAIN, what="grouped grad_attn", mass=mga)
     # a group's location gradient adds its heads' gradients (atomically, any order)
     assert_close(host(gl), oracle.sum_groups(ogl, G), **grad_tol(G, M), what="grouped grad_loc",
@@ -100,7 +101,8 @@ def test_grouped_fused_forward_and_backward(case):
                                                                                 keepdims=True)
     mz = (Af * (mga.reshape(Af.shape) + mz_head)).reshape(A.shape)
     mref = (mgl + np.abs(ogl)).sum(axis=(2, 3, 4))
-    assert_close(host(gv), ogv, **GRAD, what="grouped fused grad_value")
+    tv, mv = value_grad_terms(d["value"], sh, loc, A, g)
+    assert_close(host(gv), ogv, **GRAD, what="grouped fused grad_value", mass=mv, terms=tv)
     assert_close(host(go), oracle.sum_groups(ogo, G), **grad_tol(G, M),
                  what="grouped grad_offsets", mass=oracle.sum_groups(mgo, G))
     assert_close(host(gz), ogz, **PLAIN, what="grouped grad_logits", mass=mz)

@@ -28,7 +28,8 @@ from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fus
                                                 msda_forward, msda_forward_fused)
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import F32, GRAD, KAPPA, PLAIN, U32, assert_bits_equal, assert_close, host, to_dev
+from gpu_util import (F32, GRAD, KAPPA, PLAIN, U32, assert_bits_equal, assert_close, host,
+                      to_dev, value_grad_terms)
 
 pytestmark = pytest.mark.gpu
 
@@ -77,7 +78,8 @@ def test_wide_batch_at_the_element_limit():
         assert_close(host(fo[sl]), ora, **F32, what=f"{what} fused out")
         ogv, ogl, oga, mgl, mga = oracle.backward(block, sh, loc[sl], A[sl], g[sl],
                                                   with_mass=True)
-        assert_close(host(gv[sl]), ogv, **GRAD, what=f"{what} grad_value")
+        tv, mv = value_grad_terms(block, sh, loc[sl], A[sl], g[sl])
+        assert_close(host(gv[sl]), ogv, **GRAD, what=f"{what} grad_value", mass=mv, terms=tv)
         assert_close(host(gl[sl]), ogl, **PLAIN, what=f"{what} grad_loc", mass=mgl)
         assert_close(host(ga[sl]), oga, **PLAIN, what=f"{what} grad_attn", mass=mga)
         # fused backward: the oracle's backward at its own locations and
@@ -93,7 +95,9 @@ def test_wide_batch_at_the_element_limit():
         Af = oA64.reshape(oA64.shape[:3] + (-1,))
         mz_head = (Af * (fmga.reshape(Af.shape) + np.abs(fga_o.reshape(Af.shape)))).sum(-1, keepdims=True)
         mz = (Af * (fmga.reshape(Af.shape) + mz_head)).reshape(oA64.shape)
-        assert_close(host(fgv[sl]), fgv_o, **GRAD, what=f"{what} fused grad_value")
+        tv, mv = value_grad_terms(block, sh, oloc, oA64, g[sl])
+        assert_close(host(fgv[sl]), fgv_o, **GRAD, what=f"{what} fused grad_value", mass=mv,
+                     terms=tv)
         assert_close(host(fgo[sl]), ogo, **PLAIN, what=f"{what} grad_offsets", mass=mgo)
         assert_close(host(fgz[sl]), ogz, **PLAIN, what=f"{what} grad_logits", mass=mz)
         assert_close(host(fgr[sl]), ogr, **GRAD, what=f"{what} grad_reference", mass=mref)

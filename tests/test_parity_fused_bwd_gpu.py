@@ -19,7 +19,7 @@ import oracle
 from scale_deformable_attention_02_b200 import msda_backward_fused, msda_forward_fused
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import GRAD, KAPPA, PLAIN, U32, assert_close, host, to_dev
+from gpu_util import GRAD, KAPPA, PLAIN, U32, assert_close, host, to_dev, value_grad_terms
 
 pytestmark = pytest.mark.gpu
 
@@ -57,7 +57,8 @@ def _check(d, ref, off, logits, box: bool):
     Af = A.reshape(A.shape[:3] + (LK,))
     mz_head = (Af * (mga.reshape(Af.shape) + np.abs(oga.reshape(Af.shape)))).sum(-1, keepdims=True)
     mz = (Af * (mga.reshape(Af.shape) + mz_head)).reshape(A.shape)
-    assert_close(host(gv), ogv, **GRAD, what="grad_value")
+    tv, mv = value_grad_terms(d["value"], sh, loc, A, g)
+    assert_close(host(gv), ogv, **GRAD, what="grad_value", mass=mv, terms=tv)
     assert_close(host(go), ogo, **PLAIN, what="grad_offsets", mass=mgo)
     assert_close(host(gz), ogz, **PLAIN, what="grad_logits", mass=mz)
     assert_close(host(gr), ogr, **GRAD, what="grad_reference", mass=mref)

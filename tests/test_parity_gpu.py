@@ -19,7 +19,8 @@ from scale_deformable_attention_02_b200 import (msda_backward, msda_debug_sample
                                                 msda_forward, msda_forward_fused)
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import F32, GRAD, PLAIN, assert_bits_equal, assert_close, host, to_dev
+from gpu_util import (F32, GRAD, PLAIN, assert_bits_equal, assert_close, host, to_dev,
+                      value_grad_terms)
 
 pytestmark = pytest.mark.gpu
 
@@ -56,7 +57,8 @@ def test_tiny_forward_backward():
                                to_dev(d["grad_out"]))
     ogv, ogl, oga, mgl, mga = oracle.backward(d["value"], sh, loc, A, d["grad_out"],
                                               with_mass=True)
-    assert_close(host(gv), ogv, **GRAD, what="tiny grad_value")
+    tv, mv = value_grad_terms(d["value"], sh, loc, A, d["grad_out"])
+    assert_close(host(gv), ogv, **GRAD, what="tiny grad_value", mass=mv, terms=tv)
     assert_close(host(gl), ogl, **PLAIN, what="tiny grad_loc", mass=mgl)
     assert_close(host(ga), oga, **PLAIN, what="tiny grad_attn", mass=mga)
 
@@ -151,7 +153,8 @@ def test_encoder_compass_fused_forward_and_backward():
                                to_dev(d["grad_out"]))
     ogv, ogl, oga, mgl, mga = oracle.backward(d["value"], sh, oloc, A, d["grad_out"],
                                               with_mass=True)
-    assert_close(host(gv), ogv, **GRAD, what="compass grad_value")
+    tv, mv = value_grad_terms(d["value"], sh, oloc, A, d["grad_out"])
+    assert_close(host(gv), ogv, **GRAD, what="compass grad_value", mass=mv, terms=tv)
     assert_close(host(gl), ogl, **PLAIN, what="compass grad_loc", mass=mgl)
     assert_close(host(ga), oga, **PLAIN, what="compass grad_attn", mass=mga)
 
@@ -188,7 +191,8 @@ def test_encoder_backward():
                                to_dev(d["grad_out"]))
     ogv, ogl, oga, mgl, mga = oracle.backward(d["value"], sh, loc, A, d["grad_out"],
                                               with_mass=True)
-    assert_close(host(gv), ogv, **GRAD, what="encoder grad_value")
+    tv, mv = value_grad_terms(d["value"], sh, loc, A, d["grad_out"])
+    assert_close(host(gv), ogv, **GRAD, what="encoder grad_value", mass=mv, terms=tv)
     assert_close(host(gl), ogl, **PLAIN, what="encoder grad_loc", mass=mgl)
     assert_close(host(ga), oga, **PLAIN, what="encoder grad_attn", mass=mga)
 
@@ -230,7 +234,9 @@ def test_stress_forward_backward():
         # gradients are linear in the weight
         ogv, ogl, oga, mgl, mga = oracle.backward(v, sh, oloc, A32, d["grad_out"][sl],
                                                   with_mass=True)
-        assert_close(host(gv[sl]), ogv, **GRAD, what=f"stress grad_value n={n}")
+        tv, mv = value_grad_terms(v, sh, oloc, A32, d["grad_out"][sl])
+        assert_close(host(gv[sl]), ogv, **GRAD, what=f"stress grad_value n={n}", mass=mv,
+                     terms=tv)
         assert_close(host(gl[sl]), ogl, **PLAIN, what=f"stress grad_loc n={n}", mass=mgl)
         assert_close(host(ga[sl]), oga, **PLAIN, what=f"stress grad_attn n={n}", mass=mga)
     # at least the pushed 5% of the samples leave their level
@@ -299,7 +305,8 @@ def test_random_problems(case):
     gv, gl, ga = msda_backward(value, sh, None, to_dev(loc), to_dev(A), to_dev(d["grad_out"]))
     ogv, ogl, oga, mgl, mga = oracle.backward(d["value"], sh, loc, A, d["grad_out"],
                                               with_mass=True)
-    assert_close(host(gv), ogv, **GRAD, what="grad_value")
+    tv, mv = value_grad_terms(d["value"], sh, loc, A, d["grad_out"])
+    assert_close(host(gv), ogv, **GRAD, what="grad_value", mass=mv, terms=tv)
     assert_close(host(gl), ogl, **PLAIN, what="grad_loc", mass=mgl)
     assert_close(host(ga), oga, **PLAIN, what="grad_attn", mass=mga)
 
@@ -343,7 +350,8 @@ def test_out_of_range_and_non_finite_locations():
                                to_dev(d["grad_out"]))
     ogv, ogl, oga, mgl, mga = oracle.backward(d["value"], sh, loc, A, d["grad_out"],
                                               with_mass=True)
-    assert_close(host(gv), ogv, **GRAD, what="edge grad_value")
+    tv, mv = value_grad_terms(d["value"], sh, loc, A, d["grad_out"])
+    assert_close(host(gv), ogv, **GRAD, what="edge grad_value", mass=mv, terms=tv)
     assert_close(host(gl), ogl, **PLAIN, what="edge grad_loc", mass=mgl)
     assert_close(host(ga), oga, **PLAIN, what="edge grad_attn", mass=mga)
 

@@ -14,7 +14,7 @@ from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fus
 from scale_deformable_attention_02_b200 import workloads as wl
 
 from gpu_util import (F32, GRAD, KAPPA, PLAIN, U32, assert_bits_equal, assert_close, grad_tol,
-                      host, to_dev)
+                      host, to_dev, value_grad_terms)
 
 pytestmark = pytest.mark.gpu
 
@@ -72,7 +72,8 @@ def test_random_shape(c):
                                groups=groups)
     ogv, ogl, oga, mgl, mga = oracle.backward(d["value"], sh, loc_h, A, d["grad_out"],
                                               with_mass=True)
-    assert_close(host(gv), ogv, **GRAD, what="grad_value")
+    tv, mv = value_grad_terms(d["value"], sh, loc_h, A, d["grad_out"])
+    assert_close(host(gv), ogv, **GRAD, what="grad_value", mass=mv, terms=tv)
     assert_close(host(ga), oga, **PLAIN, what="grad_attn", mass=mga)
     assert_close(host(gl), oracle.sum_groups(ogl, G), **grad_tol(G, M), what="grad_loc",
                  mass=oracle.sum_groups(mgl + np.abs(ogl), G))
@@ -125,7 +126,8 @@ def test_random_shape(c):
     mz_head = (Af * (mga.reshape(Af.shape) + np.abs(oga.reshape(Af.shape)))).sum(-1,
                                                                                 keepdims=True)
     mz = (Af * (mga.reshape(Af.shape) + mz_head)).reshape(A64.shape)
-    assert_close(host(gv), ogv, **GRAD, what="fused grad_value")
+    tv, mv = value_grad_terms(d["value"], sh, oloc, A64, d["grad_out"])
+    assert_close(host(gv), ogv, **GRAD, what="fused grad_value", mass=mv, terms=tv)
     assert_close(host(go), oracle.sum_groups(ogo, G), **grad_tol(G, M),
                  what="fused grad_offsets", mass=oracle.sum_groups(mgo, G))
     assert_close(host(gz), ogz, **PLAIN, what="fused grad_logits", mass=mz)

@@ -21,7 +21,7 @@ from scale_deformable_attention_02_b200 import (msda_backward, msda_backward_fus
                                                 msda_debug_tiled_stalls, msda_tile_plan)
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import GRAD, PLAIN, assert_close, host, to_dev
+from gpu_util import GRAD, PLAIN, assert_close, host, to_dev, value_grad_terms
 from test_tiled_gpu import CASES, _check_plan, _refs
 
 pytestmark = pytest.mark.gpu
@@ -69,7 +69,9 @@ def _check_unfused(d, halo, cps, value=None, n_sel=None):
     # per-sample gradients: the untiled kernel's arithmetic, bit for bit
     assert torch.equal(gl, ugl), "tiled grad_loc differs from the untiled one"
     assert torch.equal(ga, uga), "tiled grad_attn differs from the untiled one"
-    assert_close(host(gv), host(ugv), **GRAD, what="tiled vs untiled grad_value")
+    tv, mv = value_grad_terms(d["value"], sh, loc, A, d["grad_out"])
+    assert_close(host(gv), host(ugv), **GRAD, what="tiled vs untiled grad_value", mass=2 * mv,
+                 terms=tv)
     sel = range(d["logits"].shape[0]) if n_sel is None else n_sel
     for n in sel:
         s = slice(n, n + 1)
@@ -78,7 +80,10 @@ def _check_unfused(d, halo, cps, value=None, n_sel=None):
                                                   np.ascontiguousarray(A[s]),
                                                   np.ascontiguousarray(d["grad_out"][s]),
                                                   with_mass=True)
-        assert_close(host(gv[s]), ogv, **GRAD, what=f"tiled grad_value n={n}")
+        tv, mv = value_grad_terms(v, sh, np.ascontiguousarray(loc[s]), np.ascontiguousarray(A[s]),
+                                  np.ascontiguousarray(d["grad_out"][s]))
+        assert_close(host(gv[s]), ogv, **GRAD, what=f"tiled grad_value n={n}", mass=mv,
+                     terms=tv)
         assert_close(host(gl[s]), ogl, **PLAIN, what=f"tiled grad_loc n={n}", mass=mgl)
         assert_close(host(ga[s]), oga, **PLAIN, what=f"tiled grad_attn n={n}", mass=mga)
     return plan
@@ -96,7 +101,10 @@ def _check_fused(d, halo, cps, value=None, n_sel=None):
     torch.cuda.synchronize()
     assert torch.equal(go, ugo), "tiled grad_offsets differ from the untiled ones"
     assert torch.equal(gz, ugz), "tiled grad_logits differ from the untiled ones"
-    assert_close(host(gv), host(ugv), **GRAD, what="tiled vs untiled grad_value")
+    lf = oracle.locations_f32(d["reference_points"], d["offsets"], sh)
+    tv, mv = value_grad_terms(d["value"], sh, lf, oracle.softmax(d["logits"]), d["grad_out"])
+    assert_close(host(gv), host(ugv), **GRAD, what="tiled vs untiled grad_value", mass=2 * mv,
+                 terms=tv)
     sel = range(d["logits"].shape[0]) if n_sel is None else n_sel
     for n in sel:
         s = slice(n, n + 1)
@@ -108,7 +116,9 @@ def _check_fused(d, halo, cps, value=None, n_sel=None):
                                                   A.astype(np.float32), g_, with_mass=True)
         ogr, ogo, ogz = oracle.fused_chain(ogl, oga, A, sh)
         mgo, mz, mref = _fused_masses(sh, mgl, ogl, mga, oga, A)
-        assert_close(host(gv[s]), ogv, **GRAD, what=f"tiled fused grad_value n={n}")
+        tv, mv = value_grad_terms(np.ascontiguousarray(d["value"][s]), sh, loc, A, g_)
+        assert_close(host(gv[s]), ogv, **GRAD, what=f"tiled fused grad_value n={n}", mass=mv,
+                     terms=tv)
         assert_close(host(go[s]), ogo, **PLAIN, what=f"tiled grad_offsets n={n}", mass=mgo)
         assert_close(host(gz[s]), ogz, **PLAIN, what=f"tiled grad_logits n={n}", mass=mz)
         assert_close(host(gr[s]), ogr, **GRAD, what=f"tiled grad_reference n={n}", mass=mref)
