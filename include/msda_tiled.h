@@ -158,6 +158,38 @@ MSDA_API msda_status msda_backward_fused_tiled(const void *value, msda_dtype val
                                                const msda_tile_plan *plan,
                                                const void *plan_buffer, msda_stream_t stream);
 
+/*
+ * msda_forward_fused_tiled without a caller-provided plan buffer: the call
+ * chooses the plan (as msda_tile_plan_init with `halo` and `ctas_per_sm`),
+ * sorts the queries into it and runs the tiled fused forward, keeping the
+ * plan in a device array that belongs to the library.  Nothing in the pages
+ * corresponds to this call; it exists for callers that cannot give the
+ * library device memory beyond their inputs and outputs (a plugin whose host
+ * framework owns all device memory and offers no workspace, or a caller that
+ * may not call cudaMalloc, which can synchronise the device and fail under
+ * memory pressure).  It allocates nothing.
+ *
+ *  - The array holds plans of up to 4 MiB (plan.device_bytes; about a million
+ *    queries): larger problems return MSDA_ERR_UNSUPPORTED.  Every GPU that
+ *    loads the library keeps the array until the process exits.
+ *  - The first call on a device looks up the array's device address (with
+ *    that device current) and keeps it; make that first call before any
+ *    stream capture.
+ *  - Every call on a device uses the same array.  Each call rewrites every
+ *    entry it reads, so nothing needs clearing between calls, but calls whose
+ *    work overlaps on the GPU (other streams, other host threads) race on the
+ *    array and must be serialised by the caller.
+ *
+ * Arguments, outputs and errors are those of msda_forward_fused and
+ * msda_tile_plan_init; every check runs before any device work.
+ */
+MSDA_API msda_status msda_forward_fused_tiled_noalloc(
+    const void *value, msda_dtype value_dtype, const int64_t *spatial_shapes,
+    const int64_t *level_start_index, const float *reference_points, int reference_dim,
+    const float *offsets, const float *logits, float *out, float *sampling_locations_out,
+    float *attention_weights_out, msda_dims dims, int halo, int ctas_per_sm,
+    msda_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

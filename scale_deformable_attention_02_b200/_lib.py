@@ -64,6 +64,8 @@ SIGNATURES = {
     "msda_forward_tiled": (INT, [P, INT, P, P, P, P, P, Dims, P, P, P]),
     "msda_forward_fused_tiled": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, Dims, P, P, P]),
     "msda_backward_tiled": (INT, [P, INT, P, P, P, P, P, P, P, P, Dims, P, P, P]),
+    "msda_forward_fused_tiled_noalloc": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, Dims, INT,
+                                               INT, P]),
     "msda_backward_fused_tiled": (INT, [P, INT, P, P, P, INT, P, P, P, P, P, P, P, Dims, P, P,
                                         P]),
     "msda_debug_sample_points": (INT, [P, P, P, Dims, P, P, P, P, P, P, P]),
