@@ -45,10 +45,11 @@
  *    returns an error has launched nothing and written nothing.
  *
  * Limits of this build: L <= 32 and 1 <= L*K <= 128; D*sizeof(value
- * element) a multiple of 16 bytes (else MSDA_ERR_ALIGN) and at most 512
- * bytes; H_l, W_l, S*M*D below 2^31 (row offsets inside one batch entry are
- * 32-bit); N*Lq*M below 2^31 (the kernels split (query, head) item indices
- * in 32 bits).  Other calls beyond them return MSDA_ERR_UNSUPPORTED.  N = 0
+ * element) a multiple of 16 bytes (else MSDA_ERR_ALIGN), of any length up to
+ * the next limit (rows over 512 bytes are taken in passes of 512); H_l, W_l,
+ * M*D, S*M*D below 2^31 (row offsets inside one batch entry are 32-bit);
+ * N*Lq*M below 2^31 (the kernels split (query, head) item indices in 32
+ * bits).  Other calls beyond them return MSDA_ERR_UNSUPPORTED.  N = 0
  * or Lq = 0 is a valid empty problem (the backward then only zeroes
  * grad_value).
  */

@@ -86,10 +86,9 @@ msda_status check_dims(msda_dtype dt, const int64_t *shapes, const int64_t *star
     }
     if (acc != d.S) return MSDA_ERR_LEVELS;
     pr->esz = dt == MSDA_F32 ? 4 : 2;
-    if (d.D > 512) return MSDA_ERR_UNSUPPORTED;
+    if (d.D > kI32Max) return MSDA_ERR_UNSUPPORTED;
     const int64_t rowbytes = d.D * pr->esz;
     if (rowbytes % 16 != 0) return MSDA_ERR_ALIGN;
-    if (rowbytes > 512) return MSDA_ERR_UNSUPPORTED;  // at most one 16-byte chunk per lane
     if (d.Lq > kI32Max || d.M > kI32Max) return MSDA_ERR_UNSUPPORTED;
     int64_t smd, md, t;
     if (!mul_le(d.M, d.D, kI32Max, &md) || !mul_le(d.S, md, kI32Max, &smd))
@@ -103,8 +102,9 @@ msda_status check_dims(msda_dtype dt, const int64_t *shapes, const int64_t *star
     pr->samples = pr->items * d.L * d.K;
     pr->n_out = pr->items * d.D;
     pr->nchunks = (int)(rowbytes / 16);
+    // one 16-byte chunk per lane; rows of more than 32 chunks take passes of 32
     int lanes = 1;
-    while (lanes < pr->nchunks) lanes <<= 1;
+    while (lanes < pr->nchunks && lanes < 32) lanes <<= 1;
     pr->lanes = lanes;
     return MSDA_OK;
 }

@@ -33,7 +33,7 @@ struct Problem {
     int64_t n_out;    // N*Lq*M*D
     int esz;          // value element size
     int nchunks;      // 16-byte chunks per value row
-    int lanes;        // lanes per row: next power of two >= nchunks
+    int lanes;        // lanes per row: next power of two >= nchunks, at most 32
     Levels lv;
 };
 

@@ -107,6 +107,9 @@ __global__ void __launch_bounds__(kWarps * 32)
     const int cslot = lin / R;
     const int chunk = lin % R;
     const bool chunk_ok = chunk < p.nchunks;
+    // rows of more than R 16-byte chunks (R = 32: over 512 bytes) take passes
+    // of R chunks; pass 0 keeps its grad_out chunk in registers
+    const int npass = R == 32 ? (p.nchunks + R - 1) / R : 1;  // narrower rows: one pass
 
     float g[kVec];
     if (chunk_ok) {
@@ -221,6 +224,33 @@ __global__ void __launch_bounds__(kWarps * 32)
                             for (int i = 0; i < kVec; i += 4)
                                 red_add_v4(dst + i, aw * g[i], aw * g[i + 1], aw * g[i + 2],
                                            aw * g[i + 3]);
+                        }
+                        for (int ps = 1; ps < npass && e.off >= 0; ++ps) {
+                            const int ck = ps * R + chunk;
+                            if (ck >= p.nchunks) break;
+                            const int64_t eo = e.off + (int64_t)ps * R * kVec;
+                            if (!msda_in_map(p.check, p.check_limit, rowbase + eo, kVec))
+                                continue;
+                            float gp[kVec], x[kVec];
+                            const float4 *gq = reinterpret_cast<const float4 *>(
+                                p.grad_out + nq * (int64_t)(M * D) + m * D + (int64_t)ck * kVec);
+#pragma unroll
+                            for (int i = 0; i < kVec / 4; ++i) {
+                                const float4 q4 = __ldg(gq + i);
+                                gp[4 * i] = q4.x;
+                                gp[4 * i + 1] = q4.y;
+                                gp[4 * i + 2] = q4.z;
+                                gp[4 * i + 3] = q4.w;
+                            }
+                            Chunk<VT>::load(vbase + eo, x);
+#pragma unroll
+                            for (int i = 0; i < kVec; ++i) t = fmaf(x[i], gp[i], t);
+                            const float aw = a * e.w;
+                            float *dst = gvbase + eo;
+#pragma unroll
+                            for (int i = 0; i < kVec; i += 4)
+                                red_add_v4(dst + i, aw * gp[i], aw * gp[i + 1], aw * gp[i + 2],
+                                           aw * gp[i + 3]);
                         }
                         v[it] = fmaf(e.w, t, v[it]);
                         v[kBatch + it] = fmaf(e.dwx, t, v[kBatch + it]);

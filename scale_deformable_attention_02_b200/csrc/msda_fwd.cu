@@ -117,7 +117,9 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
     const int npairs = 4 * LK;
     const int slot = lane / R;
     const int chunk = lane % R;
-    const bool chunk_ok = kExact || chunk < p.nchunks;
+    // rows of more than R 16-byte chunks (R = 32: over 512 bytes) take passes
+    // of R chunks; the entries, which hold whole-row addresses, serve them all
+    const int npass = R == 32 ? (p.nchunks + R - 1) / R : 1;  // narrower rows: one pass
 
     // This CTA sweeps the contiguous item range [begin, end): neighbouring
     // queries sample neighbouring pixels, so the sweep keeps rows in L1.
@@ -185,22 +187,24 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
         }
         __syncwarp();
 
-        // ---- phase 2: gather, item by item --------------------------------
+        // ---- phase 2: gather, item by item, R chunks of the row per pass ----
 #pragma unroll 1
-        for (int it = 0; it < kItems; ++it) {
-            const int64_t item = item0 + it;
+        for (int it = 0; it < kItems * npass; ++it) {
+            const int64_t item = item0 + it / npass;
             if (item >= end) break;  // uniform across the warp
+            const int ck = (it % npass) * R + chunk;  // this lane's chunk of the row
+            const bool chunk_ok = kExact || ck < p.nchunks;
             const ItemIdx ix = msda_item_idx(item, p.dM, p.dLq);
             const int m = ix.m;
             const int64_t nq = ix.nq;
             // byte offset of this lane's chunk in a row; lanes past the last chunk
             // (D*size not a power-of-two multiple of 16 bytes) re-read chunk 0 and
             // their sums are discarded, so no lane reads past a row
-            const int lane_off = chunk_ok ? chunk * 16 : 0;
+            const int64_t lane_off = chunk_ok ? (int64_t)ck * 16 : 0;
             float2 acc[kNP];
 #pragma unroll
             for (int i = 0; i < kNP; ++i) acc[i] = make_float2(0.f, 0.f);
-            const Corner *ent = corners[warp][it];
+            const Corner *ent = corners[warp][it / npass];
             for (int t0 = 0; t0 < npairs; t0 += kB * kSlots) {
                 uint4 raw[kB];
                 float w[kB];
@@ -239,7 +243,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
                 }
             if (slot == 0 && chunk_ok) {
                 float4 *dst = reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D +
-                                                         chunk * (2 * kNP));
+                                                         (int64_t)ck * (2 * kNP));
 #pragma unroll
                 for (int i = 0; i < kNP / 2; ++i)
                     __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
@@ -459,11 +463,19 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
     const int nblk = (LK + 31) / 32;
     const int slot = lane / R;
     const int chunk = lane % R;
-    const bool chunk_ok = chunk < p.nchunks;
-    const int lane_elem = (chunk_ok ? chunk : 0) * EPL;
+    // rows of more than R 16-byte chunks (R = 32: over 512 bytes) take passes
+    // of R chunks, each a unit of work of its own; pass 0 stores the sampling
+    // locations and weights
+    const int npass = R == 32 ? (p.nchunks + R - 1) / R : 1;  // narrower rows: one pass
+    const int64_t units = p.items * npass;
 
-    for (int64_t item = (int64_t)blockIdx.x * kWarps + warp; item < p.items;
-         item += (int64_t)gridDim.x * kWarps) {
+    for (int64_t u = (int64_t)blockIdx.x * kWarps + warp; u < units;
+         u += (int64_t)gridDim.x * kWarps) {
+        const int64_t item = npass == 1 ? u : u / npass;
+        const int pass = (int)(u - item * npass);
+        const int ck = pass * R + chunk;  // this lane's chunk of the row
+        const bool chunk_ok = ck < p.nchunks;
+        const int64_t lane_elem = (int64_t)(chunk_ok ? ck : 0) * EPL;
         const ItemIdx ix = msda_item_idx(item, p.dM, p.dLq);
         const int m = ix.m;
         const int64_t nq = ix.nq;
@@ -504,9 +516,9 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
                         const float2 loc = msda_fused_location(p.ref, p.ref_dim, nq, o.x, o.y, H, W);
                         lx = loc.x;
                         ly = loc.y;
-                        if (p.loc_out && first_head)
+                        if (p.loc_out && first_head && pass == 0)
                             __stcs(reinterpret_cast<float2 *>(p.loc_out) + sl, make_float2(lx, ly));
-                        if (p.attn_out) __stcs(p.attn_out + si, a);
+                        if (p.attn_out && pass == 0) __stcs(p.attn_out + si, a);
                     } else {
                         const float2 t = __ldcs(reinterpret_cast<const float2 *>(p.loc) + sl);
                         lx = t.x;
@@ -568,7 +580,7 @@ __global__ void __launch_bounds__(kWarps * 32, 3)
             }
         if (slot == 0 && chunk_ok) {
             float4 *dst =
-                reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D + chunk * EPL);
+                reinterpret_cast<float4 *>(p.out + nq * (int64_t)MD + m * D + (int64_t)ck * EPL);
 #pragma unroll
             for (int i = 0; i < kNP / 2; ++i)
                 __stcs(dst + i, make_float4(acc[2 * i].x, acc[2 * i].y, acc[2 * i + 1].x,
@@ -583,8 +595,9 @@ cudaError_t launch_long(FwdParams p, cudaStream_t stream)
     const int lanes = (p.D + EPL - 1) / EPL;  // D*size is a multiple of 16 bytes
     p.nchunks = lanes;
     const dim3 block(kWarps * 32);
+    const int64_t units = p.items * ((lanes + 31) / 32);  // (item, pass of 32 lanes) pairs
     auto go = [&](auto kern) {
-        const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, p.items, kWarps);
+        const int64_t ctas = persistent_ctas((const void *)kern, kWarps * 32, units, kWarps);
         kern<<<(unsigned)ctas, block, 0, stream>>>(p);
         return cudaGetLastError();
     };
@@ -829,7 +842,7 @@ cudaError_t launch_fwd_vt(const FwdParams &p, int R, cudaStream_t stream)
         if (E16 != 4 && p.D % E16 == 0 && p.D / E16 <= 8)
             return launch_fast_lanes<VT, E16, kFused>(p, p.D / E16, stream);
     }
-    const bool exact = p.nchunks == R;
+    const bool exact = p.nchunks % R == 0;  // every lane holds a chunk in every pass
     switch (R) {
     case 1: return launch_r<VT, 1, kFused>(p, exact, stream);
     case 2: return launch_r<VT, 2, kFused>(p, exact, stream);

@@ -174,7 +174,8 @@ def test_forward_argument_errors(lib):
     # row sizes: fp32 D = 3 (12 B), bf16 D = 4 (8 B) are not 16-byte multiples
     assert fwd(lib, Prob(D=3)) == ALIGN
     assert fwd(lib, Prob(D=4, dtype=1)) == ALIGN
-    assert fwd(lib, Prob(D=256)) == UNSUP  # 1 KB rows
+    # int32 head offsets: M*D must stay below 2^31 (any row width below that)
+    assert fwd(lib, Prob(M=2, D=1 << 30)) == UNSUP
     # pointers
     assert lib.msda_forward(fake(0), 0, None, pr.st(), fake(1), fake(2), fake(3), pr.dims,
                             None) == NULL

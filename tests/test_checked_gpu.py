@@ -45,6 +45,7 @@ CASES = [
     (1, 12, 2, 32, 16, ((6, 8), (3, 4)), "f32"),                     # L*K = 32
     (1, 9, 2, 32, 16, ((6, 8), (3, 4), (2, 2)), "f32"),              # L*K = 48, blocks
     (1, 7, 2, 64, 9, ((5, 5), (3, 3), (2, 2), (1, 1)), "f32"),       # wide, L*K = 36
+    (1, 9, 2, 160, 2, ((5, 4), (2, 3)), "f32"),                      # 640-B rows, two passes
 ]
 IDS = [f"case{i}" for i in range(len(CASES))]
 
@@ -154,10 +155,12 @@ def test_checked_build_skips_and_reports_beyond_lowered_bound(case):
     for (st, cnt, first), what in zip(codes, ("forward", "fused forward", "backward")):
         assert st == DEVICE_CHECK, what
         assert limit <= first < total, (what, first)
-    # the unfused passes skip at least one access per (sample, corner) pair
-    # beyond the bound, and no more than one per lane
+    # the unfused calls skip at least one access per (sample, corner) pair
+    # beyond the bound, and no more than one per lane and pass of 32 chunks
+    esz = 2 if dt == "bf16" else 4
+    npass = -(-(D * esz // 16) // 32)
     for st, cnt, first in (codes[0], codes[2]):
-        assert pairs <= cnt <= 32 * pairs
+        assert pairs <= cnt <= 32 * npass * pairs
     # outputs: the method on the value map with the pixels beyond the bound zeroed
     vz = _zero_beyond(d["value"], limit)
     out, fo, (ogv, ogl, oga, mgl, mga) = _oracle_all(vz, d, A)
