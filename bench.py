@@ -66,7 +66,9 @@ def parse_args(argv=None):
     ap.add_argument("--workload", choices=sorted(WORKLOAD_TEXT), default="encoder")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer leg")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle leg")
-    ap.add_argument("--e2e-steps", type=int, default=10)
+    # the pipelined e2e steps: filling and draining the copy-in / compute /
+    # copy-out pipeline costs about one download, spread over these steps
+    ap.add_argument("--e2e-steps", type=int, default=40)
     ap.add_argument("--no-floors", action="store_true",
                     help="skip the memory-floor replay of the workload's corner rows")
     ap.add_argument("--graph", action="store_true",
@@ -177,6 +179,13 @@ def read_peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_key(workload: str, step: str, schedule: str) -> str:
+    """Entry of profiles/traffic.json for a bench configuration: the workload,
+    "/fused" for the fused step, "/tiled" for the tiled kernels."""
+    key = workload if step == "split" else workload + "/fused"
+    return key + "/tiled" if schedule == "tiled" else key
 
 
 def read_traffic(workload: str, kernel: str):
@@ -519,9 +528,7 @@ def run_ours(args):
     }
     for k in kernels.values():
         k["frac_of_" + peak_kind] = k["GB_s"] / peak
-    tkey = args.workload if args.step == "split" else args.workload + "/fused"
-    if schedule == "untiled":
-        tkey += "/untiled"
+    tkey = traffic_key(args.workload, args.step, schedule)
     roofline = {
         "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
         "frac": achieved / peak, "frac_of_nominal_8000": achieved / 8000.0,

@@ -66,3 +66,19 @@ def test_kernel_source_hash_ignores_comments_only(tmp_path, monkeypatch):
     assert bench.kernel_source_hash() == base
     f.write_text(text.replace("constexpr int kWarps = 8;", "constexpr int kWarps = 4;", 1))
     assert bench.kernel_source_hash() != base
+
+
+def test_traffic_entries_cover_the_default_configurations():
+    """The default line (split step, untiled calls) and the fused step look up
+    entries that profiles/traffic.json holds, and the tiled schedule never
+    reads the untiled kernels' counts."""
+    import json
+    import os
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        entries = json.load(f)
+    assert bench.traffic_key("encoder", "split", "untiled") == "encoder"
+    assert bench.traffic_key("encoder", "fused", "untiled") == "encoder/fused"
+    assert bench.traffic_key("encoder", "split", "tiled") == "encoder/tiled"
+    for key in ("encoder", "encoder/fused"):
+        assert {"fwd", "bwd"} <= set(entries[key]), key
+    assert "encoder/tiled" not in entries
