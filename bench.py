@@ -145,8 +145,16 @@ def algorithmic_bytes(w: wl.Workload, step: str = "split", touched_rows=None) ->
     return {"fwd": fwd, "bwd": bwd, "samples": samples}
 
 
-def kernel_source_hash() -> str:
-    """sha256 of the forward and backward kernels' device code: the kernel
+# Device sources behind each schedule's kernels (the tiled kernels include the
+# untiled ones' helpers).
+UNTILED_SOURCES = ("msda_fwd.cu", "msda_bwd.cu", "msda_common.cuh", "msda_rows.cuh",
+                   "msda_types.h")
+TILED_SOURCES = UNTILED_SOURCES + ("msda_fwd_tiled.cu", "msda_bwd_tiled.cu",
+                                   "msda_tile_plan.cu", "msda_tile.cuh", "msda_tma.cuh")
+
+
+def kernel_source_hash(schedule: str = "untiled") -> str:
+    """sha256 of one schedule's forward and backward device code: the kernel
     sources and device headers and the launch-parameter structs, with comments
     and blank space removed, so that a counter taken on those kernels stays
     valid across edits that do not touch them."""
@@ -158,14 +166,15 @@ def kernel_source_hash() -> str:
         text = re.sub(r"//[^\n]*", " ", text)
         return " ".join(text.split())
 
-    for f in ("msda_fwd.cu", "msda_bwd.cu", "msda_fwd_tiled.cu", "msda_bwd_tiled.cu",
-              "msda_tile_plan.cu", "msda_common.cuh", "msda_rows.cuh", "msda_tile.cuh",
-              "msda_tma.cuh", "msda_types.h"):
+    tiled = schedule == "tiled"
+    for f in TILED_SOURCES if tiled else UNTILED_SOURCES:
         with open(os.path.join(csrc, f), encoding="utf-8") as fh:
             h.update(f.encode() + b"\0" + norm(fh.read()).encode())
     with open(os.path.join(csrc, "msda_internal.h"), encoding="utf-8") as fh:
         internal = norm(fh.read())
-    for name in ("FwdParams", "BwdParams", "TileView", "FwdTiledParams", "BwdTiledParams"):
+    structs = ("FwdParams", "BwdParams") + (
+        ("TileView", "FwdTiledParams", "BwdTiledParams") if tiled else ())
+    for name in structs:
         m = re.search(r"struct " + name + r" \{.*?\};", internal)
         h.update(name.encode() + b"\0" + (m.group(0) if m else "").encode())
     return h.hexdigest()
@@ -196,7 +205,8 @@ def read_traffic(workload: str, kernel: str):
         with open(p) as f:
             d = json.load(f)
         e = d[workload][kernel]
-        if e.get("source_sha256") != kernel_source_hash():
+        schedule = "tiled" if workload.endswith("/tiled") else "untiled"
+        if e.get("source_sha256") != kernel_source_hash(schedule):
             return None
         return float(e["dram_bytes_per_launch"])
     except Exception:

@@ -69,7 +69,7 @@ __global__ void __launch_bounds__(kWarps * 32, kMinCtas)
     const int j = lane % P;
     const bool jact = j < LK;
     const int lvl = jact ? j / K : 0;
-    const int H = p.lv.H[lvl], W = p.lv.W[lvl], start = p.lv.start[lvl];
+    const int H = p.lv.H[lvl], W = p.lv.W[lvl];
     const int ww = t.ww[lvl], wh = t.wh[lvl];
     const int soff = t.soff[lvl];
 

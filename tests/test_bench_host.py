@@ -82,3 +82,19 @@ def test_traffic_entries_cover_the_default_configurations():
     for key in ("encoder", "encoder/fused"):
         assert {"fwd", "bwd"} <= set(entries[key]), key
     assert "encoder/tiled" not in entries
+
+
+def test_untiled_hash_ignores_the_tiled_sources(tmp_path, monkeypatch):
+    """Counters of the untiled kernels stay valid when only the tiled kernels
+    change, and the tiled schedule's hash tracks both."""
+    import os
+    import shutil
+    src = os.path.join(bench.ROOT, "scale_deformable_attention_02_b200", "csrc")
+    dst = tmp_path / "scale_deformable_attention_02_b200" / "csrc"
+    shutil.copytree(src, dst)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    untiled, tiled = bench.kernel_source_hash(), bench.kernel_source_hash("tiled")
+    f = dst / "msda_fwd_tiled.cu"
+    f.write_text(f.read_text().replace("namespace msda {", "namespace msda { int unused_x;", 1))
+    assert bench.kernel_source_hash() == untiled
+    assert bench.kernel_source_hash("tiled") != tiled
