@@ -880,7 +880,10 @@ cudaError_t launch_fast_r(const BwdParams &p, cudaStream_t stream)
     // P: a power of two >= L*K and >= the 8 samples of one batch
     const int LK = p.L * p.K;
     if (LK <= 8) return launch_fast<VT, R, 8, kFused>(p, stream);
-    if (LK <= 16) return launch_fast<VT, R, 16, kFused>(p, stream);
+    if (LK <= 16 && !one_item_rounds((const void *)bwd_kernel<VT, R, 16, kFused>,
+                                     (const void *)bwd_kernel<VT, R, 32, kFused>, kWarps,
+                                     p.items))
+        return launch_fast<VT, R, 16, kFused>(p, stream);
     return launch_fast<VT, R, 32, kFused>(p, stream);
 }
 

@@ -764,7 +764,10 @@ cudaError_t launch_fast_r(const FwdParams &p, cudaStream_t stream)
     // 8/R samples one warp instruction gathers
     const int LK = p.L * p.K;
     if (LK <= 8) return launch_fast<VT, EPL, R, 8, kFused>(p, stream);
-    if (LK <= 16) return launch_fast<VT, EPL, R, 16, kFused>(p, stream);
+    if (LK <= 16 && !one_item_rounds((const void *)fwd_kernel<VT, EPL, R, 16, kFused>,
+                                     (const void *)fwd_kernel<VT, EPL, R, 32, kFused>, kWarps,
+                                     p.items))
+        return launch_fast<VT, EPL, R, 16, kFused>(p, stream);
     return launch_fast<VT, EPL, R, 32, kFused>(p, stream);
 }
 

@@ -83,6 +83,15 @@ struct PointsParams {
 // current device, but no more than the rounds of `round` items there are.
 int64_t persistent_ctas(const void *kernel, int threads, int64_t items, int round);
 
+// Whether one item per warp round finishes sooner than two.  A persistent
+// grid whose last round of two-item steps holds only a few warps leaves the
+// rest of the GPU idle for a whole step; counted in item times per warp,
+// ceil(items / 2W) * 2 against ceil(items / W1) for W and W1 resident warps
+// of the two layouts.  True when the one-item layout needs at least 15%
+// fewer item times (the decoder backward: 3 against 4).
+bool one_item_rounds(const void *two_item_kernel, const void *one_item_kernel, int warps,
+                     int64_t items);
+
 // Launchers (return the launch's cudaError_t).
 cudaError_t launch_forward(const FwdParams &p, bool bf16, bool fused, int lanes_per_row,
                            cudaStream_t stream);

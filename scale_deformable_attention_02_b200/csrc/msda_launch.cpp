@@ -42,4 +42,15 @@ int64_t persistent_ctas(const void *kernel, int threads, int64_t items, int roun
     return want < 1 ? 1 : want;
 }
 
+bool one_item_rounds(const void *two_item_kernel, const void *one_item_kernel, int warps,
+                     int64_t items)
+{
+    constexpr int64_t kAll = INT64_C(1) << 40;  // more rounds than any grid holds
+    const int64_t w2 = persistent_ctas(two_item_kernel, warps * 32, kAll, 1) * warps;
+    const int64_t w1 = persistent_ctas(one_item_kernel, warps * 32, kAll, 1) * warps;
+    const int64_t t2 = (items + 2 * w2 - 1) / (2 * w2) * 2;
+    const int64_t t1 = (items + w1 - 1) / w1;
+    return t1 * 20 <= t2 * 17;
+}
+
 }  // namespace msda
