@@ -22,7 +22,7 @@ using msda::Levels;
 using msda::kMaxLK;
 using namespace msda::api;
 
-constexpr int kAbiVersion = 10200;  // 1.2.0: tiled entry points (msda_tiled.h)
+constexpr int kAbiVersion = 10300;  // 1.3.0: value rows of any width (1.2.0: tiled entry points)
 
 }  // namespace
 

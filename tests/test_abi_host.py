@@ -74,7 +74,7 @@ def test_library_exports_nothing_else(path, headers):
 def test_status_strings_and_version(lib):
     for code, name in _lib.STATUS_NAMES.items():
         assert lib.msda_status_string(code).decode().startswith(name)
-    assert lib.msda_abi_version() == 10200
+    assert lib.msda_abi_version() == 10300
 
 
 def test_checked_build_host_calls():
