@@ -1,5 +1,7 @@
 """Helpers shared by the GPU parity tests: device transfer and the
 elementwise tolerance check |gpu - oracle| <= atol + rtol * |oracle|."""
+import functools
+
 import numpy as np
 import torch
 
@@ -31,6 +33,15 @@ def grad_tol(groups: int, heads: int) -> dict:
     when every head has its own locations, else summed over the group's heads
     with atomics."""
     return PLAIN if groups == heads else GRAD
+
+
+@functools.lru_cache(maxsize=2)
+def cached_inputs(name: str) -> dict:
+    """make_inputs of a named workload, drawn once per test session (the
+    stress workload's draws take a minute of CPU).  Callers must not modify
+    the arrays."""
+    from scale_deformable_attention_02_b200 import workloads as wl
+    return wl.make_inputs(wl.WORKLOADS[name])
 
 
 def dev():

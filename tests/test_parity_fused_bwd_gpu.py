@@ -19,7 +19,8 @@ import oracle
 from scale_deformable_attention_02_b200 import msda_backward_fused, msda_forward_fused
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import GRAD, KAPPA, PLAIN, U32, assert_close, host, to_dev, value_grad_terms
+from gpu_util import (GRAD, KAPPA, PLAIN, U32, assert_close, cached_inputs, host, to_dev,
+                      value_grad_terms)
 
 pytestmark = pytest.mark.gpu
 
@@ -30,11 +31,15 @@ def _cuda():
         pytest.skip("no CUDA device")
 
 
-def _check(d, ref, off, logits, box: bool):
+def _check(d, ref, off, logits, box: bool, got=None):
+    """The fused backward of d's inputs (or `got`, its results computed by the
+    caller) against the oracle's backward and chain rule."""
     sh = d["spatial_shapes"]
     g = d["grad_out"]
-    gv, gr, go, gz = msda_backward_fused(to_dev(d["value"]), sh, None, to_dev(ref), to_dev(off),
-                                         to_dev(logits), to_dev(g))
+    if got is None:
+        got = msda_backward_fused(to_dev(d["value"]), sh, None, to_dev(ref), to_dev(off),
+                                  to_dev(logits), to_dev(g))
+    gv, gr, go, gz = got
     loc = oracle.locations_box_f32(ref, off) if box else oracle.locations_f32(ref, off, sh)
     A = oracle.softmax(logits)
     ogv, ogl, oga, mgl, mga = oracle.backward(d["value"], sh, loc, A.astype(np.float32), g,
@@ -156,3 +161,33 @@ def test_fused_backward_wide_rows(D, K, box):
                               rng.uniform(0.05, 0.5, (2, 9, 2))], axis=-1).astype(np.float32)
         off = (rng.standard_normal(off.shape) * 0.25).astype(np.float32)
     _check(d, ref, off, d["logits"], box=box)
+
+
+def test_fused_backward_stress():
+    """The stress configuration at full size (N = 8, bf16 value, K = 8, 5% of
+    the samples pushed out of range): grad_value satisfies the adjoint
+    identity over every batch entry, and one middle entry matches the oracle
+    in every gradient (entries are independent)."""
+    w = wl.STRESS
+    d = cached_inputs("stress")
+    sh = d["spatial_shapes"]
+    value = to_dev(d["value"])
+    ref, off, z, g = (to_dev(d[k]) for k in ("reference_points", "offsets", "logits",
+                                             "grad_out"))
+    got = msda_backward_fused(value, sh, None, ref, off, z, g)
+    out = msda_forward_fused(value, sh, None, ref, off, z)
+    torch.cuda.synchronize()
+    # out is linear in the value map: <grad_out, out> = <grad_value, value>
+    lhs = float((g.double() * out.double()).sum())
+    rhs = float((got[0].double() * value.double()).sum())
+    mass = float((g.double() * out.double()).abs().sum() +
+                 (got[0].double() * value.double()).abs().sum())
+    assert abs(lhs - rhs) <= 1e-5 * mass, ("fused stress adjoint", lhs, rhs, mass)
+    del out
+    n = w.N // 2 - 1
+    sl = slice(n, n + 1)
+    dn = {k: (np.ascontiguousarray(v[sl]) if k != "spatial_shapes" else v) for k, v in d.items()
+          if k in ("value", "spatial_shapes", "reference_points", "offsets", "logits",
+                   "grad_out")}
+    _check(dn, dn["reference_points"], dn["offsets"], dn["logits"], box=False,
+           got=tuple(x[sl] for x in got))

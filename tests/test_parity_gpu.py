@@ -19,8 +19,8 @@ from scale_deformable_attention_02_b200 import (msda_backward, msda_debug_sample
                                                 msda_forward, msda_forward_fused)
 from scale_deformable_attention_02_b200 import workloads as wl
 
-from gpu_util import (F32, GRAD, PLAIN, assert_bits_equal, assert_close, host, to_dev,
-                      value_grad_terms)
+from gpu_util import (F32, GRAD, PLAIN, assert_bits_equal, assert_close, cached_inputs, host,
+                      to_dev, value_grad_terms)
 
 pytestmark = pytest.mark.gpu
 
@@ -202,7 +202,7 @@ def test_encoder_backward():
 # ---------------------------------------------------------------------------
 def test_stress_forward_backward():
     w = wl.STRESS
-    d = wl.make_inputs(w)
+    d = cached_inputs("stress")
     sh = d["spatial_shapes"]
     value = to_dev(d["value"])
     out, loc_o, a_o = msda_forward_fused(value, sh, None, to_dev(d["reference_points"]),
