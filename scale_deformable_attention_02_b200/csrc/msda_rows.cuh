@@ -12,7 +12,7 @@
 
 namespace msda {
 
-// EPL consecutive value elements of one lane (16 or 8 bytes), widened to
+// EPL consecutive value elements of one lane (32, 16 or 8 bytes), widened to
 // float pairs when consumed.
 template <typename VT, int EPL>
 struct LaneLoad;
@@ -28,6 +28,34 @@ struct LaneLoad<float, 4> {
     {
         v[0] = make_float2(__uint_as_float(r.x), __uint_as_float(r.y));
         v[1] = make_float2(__uint_as_float(r.z), __uint_as_float(r.w));
+    }
+};
+
+// Eight fp32 elements (32 bytes) of one lane with one 256-bit load (sm_100).
+// The address must be 32-byte aligned: the launcher takes these lanes only
+// for rows of 32 elements (128 bytes) in a value map whose base is 32-byte
+// aligned.
+struct Raw8 {
+    uint32_t w[8];
+};
+
+template <>
+struct LaneLoad<float, 8> {
+    using Raw = Raw8;
+    __device__ __forceinline__ static Raw load(const float *p)
+    {
+        Raw r;
+        asm volatile("ld.global.nc.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]),
+                       "=r"(r.w[5]), "=r"(r.w[6]), "=r"(r.w[7])
+                     : "l"(p));
+        return r;
+    }
+    __device__ __forceinline__ static void widen(const Raw &r, float2 (&v)[4])
+    {
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            v[i] = make_float2(__uint_as_float(r.w[2 * i]), __uint_as_float(r.w[2 * i + 1]));
     }
 };
 

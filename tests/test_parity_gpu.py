@@ -381,3 +381,25 @@ def test_forward_deterministic_and_stream_ordered():
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+def test_forward_lane_width_follows_value_alignment():
+    """fp32 rows of 32 elements are gathered in 32-byte lanes when the value
+    map is 32-byte aligned and in 16-byte lanes when it is only 16-byte
+    aligned: both match the oracle."""
+    shapes = ((12, 15), (6, 8), (3, 4), (2, 2))
+    d = wl.make_random_problem(91, N=2, Lq=77, M=4, D=32, K=4, shapes=shapes)
+    sh = d["spatial_shapes"]
+    ref, off, z = (to_dev(d[k]) for k in ("reference_points", "offsets", "logits"))
+    ora, _, _ = oracle.forward_fused(d["value"], sh, d["reference_points"], d["offsets"],
+                                     d["logits"])
+    flat = torch.from_numpy(d["value"]).reshape(-1)
+    buf = torch.zeros(flat.numel() + 8, device="cuda")
+    for shift in (0, 4):  # 0 or 16 bytes past a 32-byte aligned base
+        assert buf.data_ptr() % 32 == 0
+        v = buf[shift:shift + flat.numel()]
+        v.copy_(flat.to("cuda"))
+        value = v.view(d["value"].shape)
+        assert (value.data_ptr() % 32 == 0) == (shift == 0)
+        out = msda_forward_fused(value, sh, None, ref, off, z)
+        assert_close(host(out), ora, **F32, what=f"forward, value at +{4 * shift} bytes")
