@@ -38,6 +38,9 @@
  *    nothing and gets zero gradient.  Locations outside [0,1] are not errors.
  *  - Attention weights are used as given (never renormalised).
  *  - Accumulation is fp32 for both value dtypes.
+ *  - `value` must be 16-byte aligned.  A 32-byte aligned fp32 map of D = 32
+ *    lets the forward gather rows with 256-bit loads (a few percent faster);
+ *    results agree with the 16-byte path to fp32 rounding.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream).  The library allocates no memory and never
  *    synchronises.  Outputs are fully overwritten.
